@@ -1,0 +1,422 @@
+"""Benchmark of the lightning-indexer decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl li|reference] [--no-sweep]
+
+One step = one DSA decode indexer pass over B=8 requests with 32768 cached
+FP8 keys each (H=64 heads, d=128): query quantisation + score of every cache
+position (one fused kernel) followed by the top-2048 select (one kernel).
+Inputs are synthetic (seeded, shaped as the pages' decode workload) and the
+key caches rotate over enough copies to exceed the 126 MB L2, so every step
+reads its keys from HBM.  Under torchrun each rank runs its own batch of
+requests (weak scaling, no collective on the data path); the time is the max
+over ranks.
+
+Prints ONE JSON line (rank 0).  `--impl reference` times the fp64 CPU oracle
+on the same workload instead (a bounded sample of it).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "indexer µs/decode-step and keys scored/s at 8K–128K; % of HBM / FP8-tensor roofline"
+WORKLOAD = "dsa_decode_b8_l32k"
+B, L, H, D, KTOP = 8, 32768, 64, 128, 2048
+L2_BYTES = 126 * 1024 * 1024
+SCORER_KERNEL = "stream_score_kernel"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def decode_bytes_per_key(d=D):
+    # key bytes + per-token scale + one fp32 score written
+    return d + 4 + 4
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def traffic_for(kernel: str, units: float):
+    """DRAM bytes per launch from the committed ncu summary, scaled to `units`
+    keys, or None when that summary was taken on a different kernel source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p)).get(kernel)
+        src = os.path.join(ROOT, d["source"])
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if h != d["source_sha256_16"]:
+            return None
+        return d["dram_bytes_per_unit"] * units
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the fp64 CPU oracle
+# ---------------------------------------------------------------------------
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    import oracle
+    from sparse_attention_lightning_score_b200 import synth
+    nthreads = oracle.nthreads_default()
+    case = synth.dsa_decode(B=B, L=L, k_top=KTOP, seed=1)
+    q8, sq, _ = oracle.quantize_query(case.q, case.w.numpy())
+    rows_per_step = 1  # bounded sample: one request of the batch per step
+    times = []
+    for step in range(args.warmup + args.steps):
+        r = step % B
+        t0 = time.perf_counter()
+        q8r, sqr, _ = oracle.quantize_query(case.q[r:r + 1], case.w[r:r + 1].numpy())
+        sc = oracle.index_score(q8r, oracle.E4M3, case.w[r:r + 1], case.k8[r], oracle.E4M3, q_scale=sqr,
+                                k_scale=case.ks[r], nthreads=nthreads)
+        oracle.topk(sc, KTOP)
+        t1 = time.perf_counter()
+        if step >= args.warmup:
+            times.append(t1 - t0)
+    t = sum(times) / len(times)
+    keys_s = rows_per_step * L / t
+    out = {"impl": "reference", "metric": METRIC, "value": keys_s, "unit": "keys/s", "n_gpus": args.gpus,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3 * B / rows_per_step,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": WORKLOAD, "B": B, "L": L, "H": H, "d": D, "k": KTOP},
+           "cpu_baseline": {"value": keys_s, "unit": "keys/s", "cores": nthreads, "kind": "oracle",
+                            "sample": f"1 of {B} requests per step (L={L}), quantise+score+top-{KTOP}; "
+                                      "ms_per_step extrapolated to the full batch"},
+           "e2e": {"value": keys_s, "unit": "keys/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def cpu_baseline_sample():
+    import oracle
+    from sparse_attention_lightning_score_b200 import synth
+    nthreads = oracle.nthreads_default()
+    case = synth.dsa_decode(B=2, L=L, k_top=KTOP, seed=1)
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        r = n % 2
+        q8r, sqr, _ = oracle.quantize_query(case.q[r:r + 1], case.w[r:r + 1].numpy())
+        sc = oracle.index_score(q8r, oracle.E4M3, case.w[r:r + 1], case.k8[r], oracle.E4M3, q_scale=sqr,
+                                k_scale=case.ks[r], nthreads=nthreads)
+        oracle.topk(sc, KTOP)
+        n += 1
+        if time.perf_counter() - t0 > 8.0 or n >= 16:
+            break
+    t = time.perf_counter() - t0
+    return {"value": n * L / t, "unit": "keys/s", "cores": nthreads, "kind": "oracle",
+            "sample": f"{n} request(s) of L={L} (quantise+score+top-{KTOP}) on the host, {t:.1f} s"}
+
+
+# ---------------------------------------------------------------------------
+# li arm
+# ---------------------------------------------------------------------------
+def make_sets(dev, Lx, seed):
+    """Key caches for B requests of length Lx, copied until they exceed 1.5x L2."""
+    from sparse_attention_lightning_score_b200 import synth
+    case = synth.dsa_decode(B=B, L=Lx, k_top=KTOP, seed=seed)
+    per_set = B * Lx * (D + 4)
+    nsets = max(2, math.ceil(1.5 * L2_BYTES / per_set))
+    k8 = case.k8.to(dev)
+    ks = case.ks.to(dev)
+    sets = [(k8, ks)] + [(k8.clone(), ks.clone()) for _ in range(nsets - 1)]
+    return case, sets, nsets * per_set
+
+
+def capture(fns):
+    """One CUDA graph replaying the given launches in order (decode steps run
+    under graphs in serving; the graph removes host submission from the timing)."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for f in fns:
+            f()
+    return g
+
+
+class DecodeBench:
+    """Decode-step launches over rotating key caches, as graphs."""
+
+    def __init__(self, dev, Lx, seed):
+        import torch
+        from sparse_attention_lightning_score_b200 import api
+        self.api = api
+        self.Lx = Lx
+        self.case, self.sets, self.set_bytes = make_sets(dev, Lx, seed)
+        self.n = len(self.sets)
+        self.q, self.w = self.case.q.to(dev), self.case.w.to(dev)
+        self.sc = torch.empty((B, Lx), dtype=torch.float32, device=dev)
+        self.idx = torch.empty((B, KTOP), dtype=torch.int32, device=dev)
+
+    def score(self, i):
+        kk, ss = self.sets[i % self.n]
+        self.api.li_index_score(self.q, self.w, kk, ss, scores=self.sc)
+
+    def topk(self):
+        self.api.li_topk(self.sc, KTOP, idx=self.idx)
+
+    def step(self, i):
+        self.score(i)
+        self.topk()
+
+    def build_graphs(self, warmup):
+        import torch
+        for i in range(warmup):
+            self.step(i)
+        torch.cuda.synchronize()
+        self.step_graphs = [capture([lambda i=i: self.step(i)]) for i in range(self.n)]
+        reps = max(1, 24 // self.n)
+        self.score_graph = capture([lambda i=i: self.score(i) for i in range(self.n * reps)])
+        self.score_launches = self.n * reps
+        self.topk_graph = capture([self.topk] * 16)
+        self.topk_launches = 16
+        for g in self.step_graphs:
+            g.replay()
+        self.score_graph.replay()
+        self.topk_graph.replay()
+        torch.cuda.synchronize()
+
+    def time_steps(self, steps):
+        import torch
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(steps):
+            self.step_graphs[i % self.n].replay()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    def time_kernel(self, which, reps=3):
+        import torch
+        g, n = (self.score_graph, self.score_launches) if which == "score" else (self.topk_graph, self.topk_launches)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / (reps * n)
+
+    def time_direct(self, steps):
+        import torch
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(steps):
+            self.step(i)
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+
+def run_li(args, rank, world, local_rank):
+    import torch
+    from sparse_attention_lightning_score_b200 import api
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    bench = DecodeBench(dev, L, seed=1 + rank)
+    bench.build_graphs(args.warmup)
+    assert api.li_get_last_error() == 0
+
+    clocks = ClockSampler(local_rank)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    ms = bench.time_steps(args.steps)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if dist:
+        dist.barrier()
+    score_ms = bench.time_kernel("score")
+    topk_ms = bench.time_kernel("topk")
+    direct_ms = bench.time_direct(args.steps)
+    if dist:
+        t = torch.tensor([ms, score_ms, topk_ms, direct_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, score_ms, topk_ms, direct_ms = t.tolist()
+    launches = 2 * args.steps
+
+    # ---- end to end through the public API: pinned host q/w in, indices out,
+    # direct calls (no graph), as a user would make them
+    q, w, sc, idx = bench.q, bench.w, bench.sc, bench.idx
+    qh = bench.case.q.pin_memory()
+    wh = bench.case.w.pin_memory()
+    idx_h = torch.empty((B, KTOP), dtype=torch.int32).pin_memory()
+
+    def e2e_step(i):
+        kk, ss = bench.sets[i % bench.n]
+        q.copy_(qh, non_blocking=True)
+        w.copy_(wh, non_blocking=True)
+        api.li_index_score(q, w, kk, ss, scores=sc)
+        api.li_topk(sc, KTOP, idx=idx)
+        idx_h.copy_(idx, non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record()
+    for i in range(args.steps):
+        e2e_step(i)
+    a1.record()
+    torch.cuda.synchronize()
+    e2e_ms = a0.elapsed_time(a1) / args.steps
+    if dist:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = t.item()
+    assert api.li_get_last_error() == 0
+
+    sweep = None
+    if not args.no_sweep and rank == 0:
+        sweep = {}
+        hbm, _ = peaks()
+        for Lx in (8192, 16384, 32768, 65536, 131072):
+            bx = DecodeBench(dev, Lx, seed=11)
+            bx.build_graphs(3)
+            st_ms = bx.time_steps(max(20, args.steps))
+            sc_ms = bx.time_kernel("score")
+            tk_ms = bx.time_kernel("topk")
+            sweep[str(Lx)] = {"us_per_step": round(st_ms * 1e3, 2), "score_us": round(sc_ms * 1e3, 2),
+                              "topk_us": round(tk_ms * 1e3, 2), "keys_per_s": B * Lx / (st_ms * 1e-3),
+                              "score_hbm_frac": round(B * Lx * decode_bytes_per_key() / (sc_ms * 1e-3) / 1e9 / hbm,
+                                                      3)}
+            del bx
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    hbm, which = peaks()
+    units = B * L
+    algo_bytes = units * decode_bytes_per_key() + B * H * D * 2 + B * H * 4
+    achieved = algo_bytes / (score_ms * 1e-3) / 1e9
+    keys_s = world * B * L / (ms * 1e-3)
+    out = {
+        "metric": METRIC, "value": keys_s, "unit": "keys/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "us_per_step": ms * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": B, "L": L, "H": H, "d": D, "k": KTOP,
+                   "l2": f"{bench.n} rotating key-cache copies, {bench.set_bytes / 1e6:.0f} MB > 126 MB L2",
+                   "launch": "CUDA graph per step (score + top-k)", "per_rank": "own batch of B requests"},
+        "roofline": {"bound": "hbm", "kernel": SCORER_KERNEL, "achieved": achieved, "peak": hbm,
+                     "peak_source": which, "unit": "GB/s", "frac": achieved / hbm,
+                     "traffic": traffic_for(SCORER_KERNEL, units), "algorithmic_bytes": algo_bytes,
+                     "kernel_us": score_ms * 1e3},
+        "topk": {"us": topk_ms * 1e3, "rows_per_s": B / (topk_ms * 1e-3), "row_len": L, "k": KTOP},
+        "direct_us_per_step": direct_ms * 1e3,
+        "e2e": {"value": world * B * L / (e2e_ms * 1e-3), "unit": "keys/s",
+                "h2d_bytes_per_step": B * H * D * 2 + B * H * 4, "d2h_bytes_per_step": B * KTOP * 4,
+                "ms_per_step": e2e_ms},
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    if sweep:
+        out["sweep"] = sweep
+    if world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline_sample()
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="li", choices=["li", "reference"])
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    run_li(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

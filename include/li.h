@@ -1,0 +1,207 @@
+/*
+ * li.h -- lightning-indexer scan for NVIDIA B200 (sm_100a): the C ABI.
+ *
+ * The lightning indexer of DeepSeek Sparse Attention gives every visible cache
+ * position s of a query token t one score and keeps the k highest-scoring
+ * positions for that layer's sparse attention ("scores the whole cache and
+ * keeps the k=2048 highest-scoring tokens", Multi-layer Indexer abstract;
+ * "one score per visible position ... before top-k", IndexCache explainer,
+ * Symbol Map).  The score computed here is
+ *
+ *     I[t,s] = sum_j w[t,j] * ReLU(q[t,j,:] . k[s,:])        (j < H heads)
+ *
+ * LatentIndex (LatentIndex abstract and Figure 1) replaces the per-layer key
+ * cache of a G-layer group by one shared latent cache c, defines layer keys
+ * through per-layer decoders k_j[s] = W_dec[j] c[s], and absorbs the decoder
+ * into the query (q~_j = W_dec[j]^T q_j) so that the shared cache is scored
+ * directly.  In hierarchical selection (HS) the anchor's full scan proposes a
+ * candidate set that every follower re-scores and re-selects.
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *     allocates no device memory and keeps no pointer after the call returns.
+ *   - Tensors are dense, row-major, in the layouts stated per argument.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream).  No call synchronises the host, except li_get_last_error.
+ *   - Arguments are validated on the host before anything is launched; a
+ *     rejected call returns LI_ERR_INVALID_ARG or LI_ERR_UNSUPPORTED and has no
+ *     effect.  LI_ERR_CUDA means a CUDA runtime call failed (no device, launch
+ *     failure); the CUDA error is then cleared.  No exception or exit crosses
+ *     this boundary.
+ *   - Kernels never trap: a bounded wait that runs out or an index out of range
+ *     sets a device-side error word, the kernel returns, and the next
+ *     li_get_last_error reports it.
+ */
+#ifndef LI_H_
+#define LI_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* li_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    LI_OK = 0,
+    LI_ERR_INVALID_ARG = 1, /* a size, pointer, stride or alignment the call does not accept */
+    LI_ERR_UNSUPPORTED = 2, /* a valid combination this build does not implement */
+    LI_ERR_CUDA = 3,        /* a CUDA runtime call failed */
+    LI_ERR_TIMEOUT = 4,     /* (device) a bounded wait inside a kernel ran out */
+    LI_ERR_BOUNDS = 5       /* (device) a kernel met an index outside its tensor */
+} li_status;
+
+typedef enum {
+    LI_DTYPE_F32 = 0,
+    LI_DTYPE_BF16 = 1,
+    LI_DTYPE_E4M3 = 2 /* OCP FP8 e4m3 ("fn": no infinities, max 448) */
+} li_dtype;
+
+/* Longest score row li_topk accepts, and the largest k. */
+#define LI_TOPK_MAX_LEN 262144
+
+/* Human-readable name of a status code (static storage). */
+const char* li_status_string(li_status s);
+
+/* Reads and clears the device error word of the current device after a
+ * cudaDeviceSynchronize.  Returns LI_OK, LI_ERR_TIMEOUT, LI_ERR_BOUNDS, or
+ * LI_ERR_CUDA when the synchronisation itself fails.  This is the only call
+ * that blocks the host. */
+li_status li_get_last_error(void);
+
+/* ------------------------------------------------------------------------ */
+/* Query quantisation (FP8 scoring needs an e4m3 query as well as e4m3 keys) */
+/* ------------------------------------------------------------------------ */
+/* The pages fix no query precision; the FP8 tensor-core score needs both
+ * operands in e4m3.  Per (row, head), in fp32:
+ *     sq     = absmax(q[r,j,:]) / 448        (1 when the head is all zero)
+ *     q8     = e4m3(q[r,j,:] / sq)           (IEEE division, nearest-even, saturating at +-448)
+ *     w_eff  = w[r,j] * sq
+ * li_index_score performs this internally; this call exposes its bytes.
+ *   q_bf16  [rows, heads, dim] bf16          w      [rows, heads] fp32
+ *   q_e4m3  [rows, heads, dim] bytes (out)   q_scale[rows, heads] fp32 (out)
+ *   w_eff   [rows, heads] fp32 (out; may be NULL together with w)
+ * dim must be a multiple of 4 and at most 1024. */
+li_status li_quantize_query(const void* q_bf16, const float* w, int rows, int heads, int dim,
+                            uint8_t* q_e4m3, float* q_scale, float* w_eff, li_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* DSA lightning-indexer score (decode and causal prefill)                   */
+/* ------------------------------------------------------------------------ */
+typedef struct {
+    int rows;          /* R: decode -> requests B (one query token each); prefill -> query tokens T */
+    int heads;         /* H indexer heads */
+    int dim;           /* d, the indexer key/query width */
+    int max_len;       /* L: positions per request cache (decode) or of the shared cache (prefill) */
+    int causal;        /* 0: row r sees positions s < len[r] (len NULL: s < L).
+                          1: row t sees positions s <= t + causal_offset (and s < L) */
+    int causal_offset; /* prefill: cache position of query row 0 */
+    li_dtype q_dtype;  /* LI_DTYPE_BF16: quantised per (row, head) as li_quantize_query, FP8 tensor cores.
+                          LI_DTYPE_F32 : exact fp32 scalar path (k_dtype must be LI_DTYPE_F32). */
+    li_dtype k_dtype;  /* LI_DTYPE_E4M3 (k_scale required) or LI_DTYPE_F32 (k_scale NULL) */
+} li_score_desc;
+
+/* Scores every visible cache position of every row:
+ *     scores[r * scores_ld + s] = sk[s] * sum_j w_eff[r,j] * ReLU(q8[r,j,:] . k8[s,:])
+ * which is I[r,s] of the header comment with q = q8*sq and k = k8*sk.
+ * The scan runs over "the whole cache" of each row (Multi-layer Indexer
+ * abstract); in prefill each token sees its prefix including its own position
+ * ("scans the prefix", IndexCache explainer, Why This Exists).
+ *   q        [rows, heads, dim] (q_dtype)     w [rows, heads] fp32
+ *   k        key rows of `dim` elements (k_dtype); request r's cache begins at row
+ *            r * cache_batch_rows (0 = every row reads the same cache)
+ *   k_scale  one fp32 per key row, same row numbering as k (E4M3 only)
+ *   len      [rows] int32 visible lengths (decode; NULL = max_len; each must lie in [0, max_len])
+ *   scores   fp32, row r at scores + r * scores_ld; only visible positions are written
+ * Tensor-core path: heads == 64, dim == 128, k base 16-byte aligned, k_dtype E4M3.
+ * workspace: li_index_score_workspace(desc) bytes (0 for decode; may be NULL then). */
+li_status li_index_score(const void* q, const float* w, const void* k, const float* k_scale,
+                         int64_t cache_batch_rows, const int32_t* len, float* scores, int64_t scores_ld,
+                         const li_score_desc* desc, void* workspace, size_t workspace_bytes,
+                         li_stream_t stream);
+
+/* Bytes of device workspace li_index_score needs for this descriptor. */
+size_t li_index_score_workspace(const li_score_desc* desc);
+
+/* ------------------------------------------------------------------------ */
+/* Top-k selection                                                           */
+/* ------------------------------------------------------------------------ */
+/* Keeps the k highest scores of each row (IndexCache explainer, Symbol Map:
+ * the selected set holds k positions; k = 2,048 in the pages' models).
+ * Order: larger score first, equal scores to the lower position, NaN below
+ * every number, -0.0 equal to +0.0.  Row r holds n_r valid scores:
+ * min(max_len, r + 1 + causal_offset) when causal, else len[r] (len NULL:
+ * max_len).  The min(k, n_r) selected positions are written in ascending
+ * position order, then -1 up to k.
+ *   scores [rows] x scores_ld fp32 (scores_ld a multiple of 4, base 16-byte aligned)
+ *   idx    [rows, k] int32 (out)      vals [rows, k] fp32 (out, nullable; pads -inf)
+ * 1 <= k <= LI_TOPK_MAX_LEN, max_len <= LI_TOPK_MAX_LEN. */
+li_status li_topk(const float* scores, int64_t scores_ld, const int32_t* len, int rows, int max_len, int causal,
+                  int causal_offset, int k, int32_t* idx, float* vals, li_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* LatentIndex: decoder absorption and latent-cache scoring                  */
+/* ------------------------------------------------------------------------ */
+/* Absorbs one layer's key decoder into its queries (LatentIndex abstract,
+ * Figure 1):  q~[b,j,:] = W_dec[j]^T q[b,j,:], accumulated in fp32 and rounded
+ * once to bf16.
+ *   q_bf16      [batch, heads, dim] bf16
+ *   w_dec_bf16  [heads, dim, latent_dim] bf16 (maps a latent row to head j's key)
+ *   q_tilde     [batch, heads, latent_dim] bf16 (out)
+ * dim <= 256, latent_dim a multiple of 64. */
+li_status li_absorb_query(const void* q_bf16, const void* w_dec_bf16, void* q_tilde_bf16, int batch, int heads,
+                          int dim, int latent_dim, li_stream_t stream);
+
+/* Scores the shared latent cache with absorbed queries:
+ *     scores[b * scores_ld + s] = sum_j w[b,j] * ReLU(q~[b,j,:] . c[b,s,:])   for s < len[b]
+ *   q_tilde [batch, heads, latent_dim] bf16     w [batch, heads] fp32
+ *   c       latent rows of latent_dim bf16; request b's rows begin at row b * cache_batch_rows
+ *   len     [batch] int32 or NULL (= max_len)
+ * Tensor-core path (bf16): heads == 64, latent_dim == 256, c base 16-byte aligned. */
+li_status li_latent_score(const void* q_tilde_bf16, const float* w, const void* c_bf16, int64_t cache_batch_rows,
+                          const int32_t* len, float* scores, int64_t scores_ld, int batch, int heads, int latent_dim,
+                          int max_len, li_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Hierarchical selection: followers refine the anchor's candidates         */
+/* ------------------------------------------------------------------------ */
+/* LatentIndex abstract: "followers independently refine a shared candidate
+ * set proposed by the anchor".  For every follower f and request b, each
+ * candidate latent row c[b, cand[b,i]] is gathered once and scored against all
+ * followers' absorbed queries,
+ *     I_f[b,i] = sum_j w[f,b,j] * ReLU(q~[f,b,j,:] . c[b, cand[b,i], :]),
+ * then the k best candidates by (score desc, cache position asc) are kept and
+ * written as cache positions in ascending order, padded with -1.  Negative
+ * candidates are padding and are never selected.  Candidates must be listed in
+ * ascending cache position (li_topk's output order), padding last.
+ *   c       latent rows as in li_latent_score     cand [batch, n_cand] int32
+ *   q_tilde [followers, batch, heads, latent_dim] bf16   w [followers, batch, heads] fp32
+ *   out_idx [followers, batch, k] int32 (out)
+ * Candidates outside [0, rows of c) are reported as LI_ERR_BOUNDS by
+ * li_get_last_error and are not read.  heads == 64, latent_dim == 256,
+ * followers * heads <= 256, n_cand <= LI_TOPK_MAX_LEN.
+ * workspace: li_hs_refine_workspace(...) bytes. */
+li_status li_hs_refine(const void* c_bf16, int64_t cache_batch_rows, int64_t cache_rows, const int32_t* cand,
+                       int batch, int n_cand, const void* q_tilde_bf16, const float* w, int followers, int heads,
+                       int latent_dim, int k, int32_t* out_idx, void* workspace, size_t workspace_bytes,
+                       li_stream_t stream);
+
+size_t li_hs_refine_workspace(int batch, int n_cand, int followers);
+
+/* ------------------------------------------------------------------------ */
+/* Diagnostics                                                               */
+/* ------------------------------------------------------------------------ */
+/* Launches one block whose only work is the library's bounded wait on an
+ * mbarrier that nothing ever arrives on, with the given limit in nanoseconds.
+ * The wait runs out, the kernel records LI_ERR_TIMEOUT and returns; the next
+ * li_get_last_error reports it.  Exercises the failure path of every
+ * pipeline wait without faulting or hanging the device. */
+li_status li_selftest_wait_timeout(uint64_t limit_ns, li_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LI_H_ */

@@ -1,0 +1,11 @@
+"""B200-native lightning-indexer scan (DSA) with LatentIndex extensions.
+
+The hot path runs in ``libli.so`` (hand-written sm_100a CUDA behind the C ABI
+in ``include/li.h``); ``api`` is its thin PyTorch binding and ``synth`` makes
+the seeded synthetic inputs.
+"""
+from .api import (LiError, li_absorb_query, li_get_last_error, li_hs_refine, li_index_score,  # noqa: F401
+                  li_latent_score, li_quantize_query, li_selftest_wait_timeout, li_topk)
+
+__all__ = ["LiError", "li_absorb_query", "li_get_last_error", "li_hs_refine", "li_index_score", "li_latent_score",
+           "li_quantize_query", "li_selftest_wait_timeout", "li_topk"]

@@ -1,0 +1,186 @@
+"""Thin PyTorch binding over the li C ABI: same names, argument marshalling only.
+
+Every function takes CUDA tensors, allocates the outputs (and any workspace)
+with torch on the tensors' device, passes raw device pointers and the current
+torch stream to ``libli.so``, and raises ``LiError`` on a non-OK status.  No
+step of the indexer path runs in Python or torch.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional
+
+import torch
+
+from . import _lib
+from ._lib import LiError, ScoreDesc  # noqa: F401  (re-exported)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+
+
+def _round4(n: int) -> int:
+    return (n + 3) // 4 * 4
+
+
+def li_get_last_error() -> int:
+    """Synchronise the device and return (and clear) the device error status."""
+    return int(_lib.load().li_get_last_error())
+
+
+def li_quantize_query(q: torch.Tensor, w: Optional[torch.Tensor] = None, stream=None):
+    """q bf16 [R,H,d] (+ w fp32 [R,H]) -> (q8 uint8 [R,H,d], sq fp32 [R,H], w_eff fp32 [R,H] or None)."""
+    _need(q, "q", torch.bfloat16)
+    R, H, d = q.shape
+    q8 = torch.empty((R, H, d), dtype=torch.uint8, device=q.device)
+    sq = torch.empty((R, H), dtype=torch.float32, device=q.device)
+    we = None
+    if w is not None:
+        _need(w, "w", torch.float32)
+        we = torch.empty((R, H), dtype=torch.float32, device=q.device)
+    st = _lib.load().li_quantize_query(_ptr(q), _ptr(w), R, H, d, _ptr(q8), _ptr(sq), _ptr(we), _stream(stream))
+    _lib.check("li_quantize_query", st)
+    return q8, sq, we
+
+
+def score_desc(rows, heads, dim, max_len, causal=False, causal_offset=0, q_dtype=_lib.LI_DTYPE_BF16,
+               k_dtype=_lib.LI_DTYPE_E4M3) -> ScoreDesc:
+    return ScoreDesc(int(rows), int(heads), int(dim), int(max_len), int(bool(causal)), int(causal_offset),
+                     int(q_dtype), int(k_dtype))
+
+
+def li_index_score(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, k_scale: Optional[torch.Tensor] = None, *,
+                   lens: Optional[torch.Tensor] = None, causal: bool = False, causal_offset: int = 0,
+                   scores: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None, stream=None):
+    """DSA lightning-indexer scores.
+
+    q: [R,H,d] bf16 (FP8 tensor-core path, k uint8/float8_e4m3fn + k_scale) or fp32
+    (exact path, k fp32).  k: [R,L,d] (one cache per row) or [L,d] (shared cache).
+    Returns scores fp32 [R, round4(L)]; positions a row cannot see are left unwritten.
+    """
+    _need(q, "q", (torch.bfloat16, torch.float32))
+    _need(w, "w", torch.float32)
+    _need(k, "k")
+    R, H, d = q.shape
+    if k.dtype == torch.float8_e4m3fn:
+        k = k.view(torch.uint8)
+    L = k.shape[-2]
+    batch_rows = k.shape[1] if k.dim() == 3 else 0
+    if q.dtype == torch.float32:
+        qd, kd = _lib.LI_DTYPE_F32, _lib.LI_DTYPE_F32
+    else:
+        qd, kd = _lib.LI_DTYPE_BF16, _lib.LI_DTYPE_E4M3
+        _need(k_scale, "k_scale", torch.float32)
+    if lens is not None:
+        _need(lens, "lens", torch.int32)
+    desc = score_desc(R, H, d, L, causal, causal_offset, qd, kd)
+    lib = _lib.load()
+    if scores is None:
+        scores = torch.empty((R, _round4(L)), dtype=torch.float32, device=q.device)
+    need = lib.li_index_score_workspace(ctypes.byref(desc))
+    if need and (workspace is None or workspace.numel() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    st = lib.li_index_score(_ptr(q), _ptr(w), _ptr(k), _ptr(k_scale), batch_rows, _ptr(lens), _ptr(scores),
+                            scores.stride(0), ctypes.byref(desc), _ptr(workspace) if need else None,
+                            need, _stream(stream))
+    _lib.check("li_index_score", st)
+    return scores
+
+
+def li_topk(scores: torch.Tensor, k: int, *, lens: Optional[torch.Tensor] = None, max_len: Optional[int] = None,
+            causal: bool = False, causal_offset: int = 0, with_values: bool = False, idx=None, vals=None,
+            stream=None):
+    """Per-row top-k -> idx int32 [rows, k] ascending (-1 pads) [, vals fp32 [rows, k]]."""
+    _need(scores, "scores", torch.float32)
+    rows, ld = scores.shape
+    if max_len is None:
+        max_len = ld
+    if lens is not None:
+        _need(lens, "lens", torch.int32)
+    if idx is None:
+        idx = torch.empty((rows, k), dtype=torch.int32, device=scores.device)
+    if with_values and vals is None:
+        vals = torch.empty((rows, k), dtype=torch.float32, device=scores.device)
+    st = _lib.load().li_topk(_ptr(scores), ld, _ptr(lens), rows, int(max_len), int(bool(causal)), int(causal_offset),
+                             int(k), _ptr(idx), _ptr(vals) if with_values else None, _stream(stream))
+    _lib.check("li_topk", st)
+    return (idx, vals) if with_values else idx
+
+
+def li_absorb_query(q: torch.Tensor, w_dec: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None):
+    """q bf16 [B,H,d], W_dec bf16 [H,d,dc] -> q~ bf16 [B,H,dc]."""
+    _need(q, "q", torch.bfloat16)
+    _need(w_dec, "w_dec", torch.bfloat16)
+    B, H, d = q.shape
+    dc = w_dec.shape[2]
+    if out is None:
+        out = torch.empty((B, H, dc), dtype=torch.bfloat16, device=q.device)
+    st = _lib.load().li_absorb_query(_ptr(q), _ptr(w_dec), _ptr(out), B, H, d, dc, _stream(stream))
+    _lib.check("li_absorb_query", st)
+    return out
+
+
+def li_latent_score(q_tilde: torch.Tensor, w: torch.Tensor, c: torch.Tensor, *, lens: Optional[torch.Tensor] = None,
+                    scores: Optional[torch.Tensor] = None, stream=None):
+    """q~ bf16 [B,H,dc], w fp32 [B,H], c bf16 [B,L,dc] (or shared [L,dc]) -> scores fp32 [B, round4(L)]."""
+    _need(q_tilde, "q_tilde", torch.bfloat16)
+    _need(w, "w", torch.float32)
+    _need(c, "c", torch.bfloat16)
+    B, H, dc = q_tilde.shape
+    L = c.shape[-2]
+    batch_rows = c.shape[1] if c.dim() == 3 else 0
+    if lens is not None:
+        _need(lens, "lens", torch.int32)
+    if scores is None:
+        scores = torch.empty((B, _round4(L)), dtype=torch.float32, device=c.device)
+    st = _lib.load().li_latent_score(_ptr(q_tilde), _ptr(w), _ptr(c), batch_rows, _ptr(lens), _ptr(scores),
+                                     scores.stride(0), B, H, dc, L, _stream(stream))
+    _lib.check("li_latent_score", st)
+    return scores
+
+
+def li_hs_refine(c: torch.Tensor, cand: torch.Tensor, q_tilde: torch.Tensor, w: torch.Tensor, k: int, *,
+                 out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None, stream=None):
+    """Followers re-score the anchor's candidates and keep their own top-k.
+
+    c bf16 [B,L,dc] (or shared [L,dc]); cand int32 [B,C] ascending, -1 padding last;
+    q~ bf16 [F,B,H,dc]; w fp32 [F,B,H] -> out int32 [F,B,k] cache positions.
+    """
+    _need(c, "c", torch.bfloat16)
+    _need(cand, "cand", torch.int32)
+    _need(q_tilde, "q_tilde", torch.bfloat16)
+    _need(w, "w", torch.float32)
+    F, B, H, dc = q_tilde.shape
+    C = cand.shape[1]
+    batch_rows = c.shape[1] if c.dim() == 3 else 0
+    cache_rows = c.numel() // dc
+    lib = _lib.load()
+    need = lib.li_hs_refine_workspace(B, C, F)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=c.device)
+    if out is None:
+        out = torch.empty((F, B, k), dtype=torch.int32, device=c.device)
+    st = lib.li_hs_refine(_ptr(c), batch_rows, cache_rows, _ptr(cand), B, C, _ptr(q_tilde), _ptr(w), F, H, dc, int(k),
+                          _ptr(out), _ptr(workspace), need, _stream(stream))
+    _lib.check("li_hs_refine", st)
+    return out
+
+
+def li_selftest_wait_timeout(limit_ns: int, stream=None):
+    st = _lib.load().li_selftest_wait_timeout(int(limit_ns), _stream(stream))
+    _lib.check("li_selftest_wait_timeout", st)

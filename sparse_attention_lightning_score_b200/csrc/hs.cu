@@ -1,0 +1,266 @@
+// Hierarchical selection (LatentIndex abstract): followers independently
+// refine the candidate set proposed by the anchor.  This kernel gathers each
+// candidate latent row c[b, cand[b,i]] ONCE and scores it against the
+// absorbed queries of all F followers in one tensor-core pass:
+//
+//     I_f[b,i] = sum_j w[f,b,j] * ReLU(q~[f,b,j,:] . c[b, cand[b,i], :])
+//
+// MMA tile: 128 gathered candidates (M) x F*64 follower-heads (N <= 256) x 256
+// latent dims (four 128-byte K blocks, 16 tcgen05.mma.kind::f16 with K = 16).
+// Rows are gathered with 16-byte cp.async into the 128-byte-swizzled K-major
+// layout the MMA reads; padding (negative) candidates are zero-filled and
+// scored -inf so the following top-k never prefers them; candidates outside
+// the cache are reported (LI_ERR_BOUNDS) and zero-filled, never read.
+//
+// Warps: 0..3 gather producers, 4 TMEM allocator + MMA issuer, 5..8 follower
+// query preparation and epilogue.  Output: scores [F*B, round4(C)] fp32.
+#include "li_common.cuh"
+#include "li_kernels.cuh"
+
+namespace li {
+
+namespace {
+
+constexpr int HS_M = 128;
+constexpr int HS_H = 64;
+constexpr int HS_DC = 256;
+constexpr int HS_KBLK = 4;
+constexpr int HS_STAGES = 6;
+constexpr int HS_STAGE_BYTES = HS_M * 128;
+constexpr int HS_FMAX = 4;
+constexpr int HS_DEPTH = 3;  // cp.async groups in flight per producer thread
+constexpr int HS_THREADS = 288;
+
+template <int F>
+struct HsCfg {
+    static constexpr int N = F * HS_H;
+    static constexpr int Q_BYTES = HS_KBLK * N * 128;
+    static constexpr int OFF_Q = HS_STAGES * HS_STAGE_BYTES;
+    static constexpr int OFF_W = OFF_Q + Q_BYTES;
+    static constexpr int OFF_BAR = OFF_W + N * 4;
+    static constexpr int NBAR = 2 * HS_STAGES + 2 + 2 + 1;
+    static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
+    static constexpr int SMEM = OFF_TMEM + 16 + 1024;
+    static constexpr int TMEM_COLS = (2 * N <= 128) ? 128 : ((2 * N <= 256) ? 256 : 512);
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+template <int F>
+__global__ void __launch_bounds__(HS_THREADS, 1) hs_rescore_kernel(const HsArgs a, int tiles_per_cta) {
+    using C = HsCfg<F>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    const int b = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ntiles = (a.C + HS_M - 1) / HS_M;
+    const int t0 = blockIdx.x * tiles_per_cta;
+    const int nt = min(t0 + tiles_per_cta, ntiles) - t0;
+    if (nt <= 0) return;
+    const int ldw = (a.C + 3) & ~3;
+
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* empty = full + HS_STAGES;
+    uint64_t* accf = empty + HS_STAGES;
+    uint64_t* acce = accf + 2;
+    uint64_t* qready = acce + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
+    float* wsm = reinterpret_cast<float*>(smem + C::OFF_W);
+    uint8_t* qsm = smem + C::OFF_Q;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < HS_STAGES; ++s) {
+            mbar_init(&full[s], 128);
+            mbar_init(&empty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&accf[i], 1);
+            mbar_init(&acce[i], 128);
+        }
+        mbar_init(qready, 128);
+        fence_mbar_init();
+    }
+    if (warp == 4) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int32_t* cand = a.cand + (size_t)b * a.C;
+    const long long rowbase = (long long)b * a.batch_rows;
+
+    if (warp < 4) {
+        // ------------------------------------------------------------ gather producers
+        // Thread p handles row (p) of every stage: 8 chunks of 16 bytes of one
+        // 128-byte K block, written at their swizzled positions.
+        const int p = threadIdx.x;  // 0..127 = row within the tile
+        int stage = 0;
+        uint32_t ph = 0;
+        int pending = 0;
+        int pend_stage[HS_DEPTH + 1];
+        bool ok = true;
+        for (int it = 0; ok && it < nt; ++it) {
+            const int i = (t0 + it) * HS_M + p;
+            int s = i < a.C ? __ldg(cand + i) : -1;
+            uint32_t nbytes = 16;
+            const long long lim = a.batch_rows > 0 ? min((long long)a.batch_rows, a.cache_rows - rowbase)
+                                                   : a.cache_rows;
+            if (s < 0) nbytes = 0;
+            else if (s >= lim) {
+                record_error(a.err, ERRBIT_BOUNDS);
+                nbytes = 0;
+            }
+            const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(a.c) +
+                                       (nbytes ? (size_t)(rowbase + s) * HS_DC : 0);
+            for (int kb = 0; kb < HS_KBLK; ++kb) {
+                if (!mbar_wait(&empty[stage], ph ^ 1u, a.err)) { ok = false; break; }
+                const uint32_t dst = smem_u32(smem + stage * HS_STAGE_BYTES);
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch)
+                    cp_async16(dst + sw128_offset(p, ch), src + kb * 64 + ch * 8, nbytes);
+                cp_async_commit();
+                pend_stage[pending++] = stage;
+                if (pending > HS_DEPTH) {
+                    cp_async_wait<HS_DEPTH>();
+                    fence_proxy_async_smem();
+                    mbar_arrive(&full[pend_stage[0]]);
+#pragma unroll
+                    for (int q = 0; q < HS_DEPTH; ++q) pend_stage[q] = pend_stage[q + 1];
+                    --pending;
+                }
+                if (++stage == HS_STAGES) { stage = 0; ph ^= 1u; }
+            }
+        }
+        cp_async_wait<0>();
+        fence_proxy_async_smem();
+        for (int q = 0; q < pending; ++q) mbar_arrive(&full[pend_stage[q]]);
+    } else if (warp == 4) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t IDESC = idesc_f32acc(HS_M, C::N, kFmtBF16);
+            bool ok = mbar_wait(qready, 0, a.err);
+            tc_fence_after();
+            const uint32_t qaddr = smem_u32(qsm);
+            int stage = 0;
+            uint32_t ph = 0;
+            for (int it = 0; ok && it < nt; ++it) {
+                const int acc = it & 1;
+                if (!mbar_wait(&acce[acc], ((it >> 1) & 1) ^ 1u, a.err)) break;
+                tc_fence_after();
+                const uint32_t dt = tmem_base + (uint32_t)(acc * C::N);
+                for (int kb = 0; kb < HS_KBLK; ++kb) {
+                    if (!mbar_wait(&full[stage], ph, a.err)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t aaddr = smem_u32(smem + stage * HS_STAGE_BYTES);
+                    const uint32_t baddr = qaddr + (uint32_t)(kb * C::N * 128);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16(dt, sw128_kmajor_desc(aaddr + kk * 32), sw128_kmajor_desc(baddr + kk * 32), IDESC,
+                                 (kb | kk) != 0);
+                    tc_commit(&empty[stage]);
+                    if (++stage == HS_STAGES) { stage = 0; ph ^= 1u; }
+                }
+                if (!ok) break;
+                tc_commit(&accf[acc]);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ follower queries
+        const int et = threadIdx.x - 160;  // 0..127
+        constexpr int CH = HS_KBLK * 8;    // 16-byte chunks per query row
+        for (int ci = et; ci < C::N * CH; ci += 128) {
+            const int r = ci / CH, cc = ci % CH;  // r = f * 64 + j
+            const int f = r / HS_H, j = r % HS_H;
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.qt) +
+                                                                 (((size_t)f * a.B + b) * HS_H + j) * HS_DC) + cc);
+            *reinterpret_cast<uint4*>(qsm + (cc >> 3) * (C::N * 128) + sw128_offset(r, cc & 7)) = v;
+        }
+        for (int r = et; r < C::N; r += 128) {
+            const int f = r / HS_H, j = r % HS_H;
+            wsm[r] = __ldg(a.w + ((size_t)f * a.B + b) * HS_H + j);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(qready);
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+
+        // ------------------------------------------------------------ epilogue
+        const int g = warp & 3;
+        for (int it = 0; it < nt; ++it) {
+            const int acc = it & 1;
+            const int i = (t0 + it) * HS_M + g * 32 + lane;
+            const int s = i < a.C ? __ldg(cand + i) : -1;
+            if (!mbar_wait(&accf[acc], (it >> 1) & 1, a.err)) break;
+            tc_fence_after();
+            float res[F];
+#pragma unroll
+            for (int f = 0; f < F; ++f) {
+                const uint32_t tb = tmem_base + ((uint32_t)(g * 32) << 16) + (uint32_t)(acc * C::N + f * HS_H);
+                uint32_t v0[32], v1[32];
+                tmem_ld32(tb, v0);
+                tmem_ld32(tb + 32, v1);
+                tmem_ld_wait();
+                res[f] = relu_dot32(v0, wsm + f * HS_H) + relu_dot32(v1, wsm + f * HS_H + 32);
+            }
+            tc_fence_before();
+            mbar_arrive(&acce[acc]);
+            if (i < a.C) {
+#pragma unroll
+                for (int f = 0; f < F; ++f)
+                    a.out[((size_t)f * a.B + b) * ldw + i] = s >= 0 ? res[f] : -INFINITY;
+            }
+        }
+    }
+    __syncwarp();
+    __syncthreads();
+    if (warp == 4) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+template <int F>
+li_status launch_f(const HsArgs& a, cudaStream_t st) {
+    using C = HsCfg<F>;
+    static bool attr_done[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_done[dev]) {
+        if (cudaFuncSetAttribute(hs_rescore_kernel<F>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
+            cudaSuccess)
+            return host_check_launch();
+        attr_done[dev] = true;
+    }
+    const int ntiles = (a.C + HS_M - 1) / HS_M;
+    const int sms = host_num_sms();
+    int cpr = max(1, sms / max(1, a.B));
+    int tpc = max(1, (ntiles + cpr - 1) / cpr);
+    cpr = (ntiles + tpc - 1) / tpc;
+    hs_rescore_kernel<F><<<dim3(cpr, a.B), HS_THREADS, C::SMEM, st>>>(a, tpc);
+    return host_check_launch();
+}
+
+}  // namespace
+
+li_status launch_hs_rescore(const HsArgs& a, cudaStream_t st) {
+    if (a.B <= 0 || a.C <= 0) return LI_OK;
+    switch (a.F) {
+    case 1: return launch_f<1>(a, st);
+    case 2: return launch_f<2>(a, st);
+    case 3: return launch_f<3>(a, st);
+    case 4: return launch_f<4>(a, st);
+    default: return LI_ERR_UNSUPPORTED;
+    }
+}
+
+}  // namespace li

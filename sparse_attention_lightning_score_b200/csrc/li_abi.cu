@@ -1,0 +1,310 @@
+// The exported C ABI of the li library (declared in include/li.h): argument
+// validation, TMA tensor-map encoding, workspace carving and dispatch to the
+// kernel launchers.  Nothing here allocates device memory or blocks the host
+// (except li_get_last_error).
+#include <cudaTypedefs.h>
+
+#include <cstring>
+
+#include "li_common.cuh"
+#include "li_kernels.cuh"
+
+namespace li {
+
+__device__ unsigned g_li_error_word;
+
+namespace {
+
+constexpr int kMaxDev = 64;
+
+int current_device() {
+    int d = 0;
+    cudaGetDevice(&d);
+    return d;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        else
+            cudaGetLastError();
+    }
+    return fn;
+}
+
+// 2-D tensor map over `rows` rows of `row_elems` elements (row pitch
+// `row_bytes`), box = [box_inner elements, box_rows rows], 128-byte swizzle.
+bool encode_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t row_elems, uint64_t rows,
+                   uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows) {
+    auto fn = tensor_map_encoder();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {row_elems, rows};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_inner, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace
+
+DevErr host_dev_err() {
+    static unsigned* addr[kMaxDev] = {};
+    const int d = current_device();
+    if (d < kMaxDev && !addr[d]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_li_error_word) == cudaSuccess) addr[d] = static_cast<unsigned*>(p);
+        else cudaGetLastError();
+    }
+    return DevErr{d < kMaxDev ? addr[d] : nullptr, kDefaultWaitLimitNs};
+}
+
+int host_num_sms() {
+    static int n[kMaxDev] = {};
+    const int d = current_device();
+    if (d < kMaxDev && n[d] == 0) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, d) != cudaSuccess) {
+            cudaGetLastError();
+            v = 148;
+        }
+        n[d] = v;
+    }
+    return d < kMaxDev ? n[d] : 148;
+}
+
+li_status host_check_launch() {
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? LI_OK : LI_ERR_CUDA;
+}
+
+// The device must answer before any launch: an absent device or a missing
+// error word becomes LI_ERR_CUDA instead of a fault.
+static li_status ready(DevErr* e) {
+    *e = host_dev_err();
+    if (!e->word) return LI_ERR_CUDA;
+    return LI_OK;
+}
+
+}  // namespace li
+
+using namespace li;
+
+extern "C" {
+
+const char* li_status_string(li_status s) {
+    switch (s) {
+    case LI_OK: return "LI_OK";
+    case LI_ERR_INVALID_ARG: return "LI_ERR_INVALID_ARG";
+    case LI_ERR_UNSUPPORTED: return "LI_ERR_UNSUPPORTED";
+    case LI_ERR_CUDA: return "LI_ERR_CUDA";
+    case LI_ERR_TIMEOUT: return "LI_ERR_TIMEOUT";
+    case LI_ERR_BOUNDS: return "LI_ERR_BOUNDS";
+    }
+    return "LI_ERR_UNKNOWN";
+}
+
+li_status li_get_last_error(void) {
+    DevErr e;
+    if (ready(&e) != LI_OK) return LI_ERR_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess) {
+        cudaGetLastError();
+        return LI_ERR_CUDA;
+    }
+    unsigned v = 0;
+    if (cudaMemcpy(&v, e.word, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) {
+        cudaGetLastError();
+        return LI_ERR_CUDA;
+    }
+    const unsigned zero = 0;
+    if (v && cudaMemcpy(e.word, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) {
+        cudaGetLastError();
+        return LI_ERR_CUDA;
+    }
+    if (v & ERRBIT_TIMEOUT) return LI_ERR_TIMEOUT;
+    if (v & ERRBIT_BOUNDS) return LI_ERR_BOUNDS;
+    return LI_OK;
+}
+
+li_status li_quantize_query(const void* q_bf16, const float* w, int rows, int heads, int dim, uint8_t* q_e4m3,
+                            float* q_scale, float* w_eff, li_stream_t stream) {
+    if (rows < 0 || heads <= 0 || dim <= 0 || dim > 1024 || (dim % 4) != 0) return LI_ERR_INVALID_ARG;
+    if (rows == 0) return LI_OK;
+    if (!q_bf16 || !q_e4m3 || !q_scale || (w_eff && !w)) return LI_ERR_INVALID_ARG;
+    if (dim == 128 && !aligned(q_bf16, 8)) return LI_ERR_INVALID_ARG;
+    if (!aligned(q_bf16, 2) || (dim == 128 && !aligned(q_e4m3, 4))) return LI_ERR_INVALID_ARG;
+    DevErr e;
+    if (ready(&e) != LI_OK) return LI_ERR_CUDA;
+    return launch_quantize_query(q_bf16, w, rows, heads, dim, q_e4m3, q_scale, w_eff, stream);
+}
+
+size_t li_index_score_workspace(const li_score_desc* d) {
+    if (!d || !d->causal || d->q_dtype != LI_DTYPE_BF16 || d->k_dtype != LI_DTYPE_E4M3 || d->rows <= 0) return 0;
+    const size_t nh = (size_t)d->rows * d->heads;
+    return align_up(nh * d->dim, 256) + 2 * align_up(nh * sizeof(float), 256);
+}
+
+li_status li_index_score(const void* q, const float* w, const void* k, const float* k_scale,
+                         int64_t cache_batch_rows, const int32_t* len, float* scores, int64_t scores_ld,
+                         const li_score_desc* desc, void* workspace, size_t workspace_bytes, li_stream_t stream) {
+    if (!desc) return LI_ERR_INVALID_ARG;
+    const li_score_desc d = *desc;
+    if (d.rows < 0 || d.heads <= 0 || d.dim <= 0 || d.max_len < 0 || cache_batch_rows < 0) return LI_ERR_INVALID_ARG;
+    if (d.rows == 0 || d.max_len == 0) return LI_OK;
+    if (!q || !w || !k || !scores || scores_ld < d.max_len) return LI_ERR_INVALID_ARG;
+    if (d.causal && (cache_batch_rows != 0 || len)) return LI_ERR_INVALID_ARG;
+    if (d.causal && (d.causal_offset < 0)) return LI_ERR_INVALID_ARG;
+    DevErr e;
+    if (ready(&e) != LI_OK) return LI_ERR_CUDA;
+
+    if (d.q_dtype == LI_DTYPE_F32 && d.k_dtype == LI_DTYPE_F32) {
+        if (k_scale || (size_t)d.heads * d.dim > 12000) return LI_ERR_UNSUPPORTED;
+        SimtArgs a{static_cast<const float*>(q), w, static_cast<const float*>(k), len, scores, scores_ld,
+                   cache_batch_rows, d.rows, d.heads, d.dim, d.max_len, d.causal, d.causal_offset, e};
+        return launch_simt_score(a, stream);
+    }
+    if (d.q_dtype != LI_DTYPE_BF16 || d.k_dtype != LI_DTYPE_E4M3) return LI_ERR_UNSUPPORTED;
+    if (!k_scale) return LI_ERR_INVALID_ARG;
+    if (d.heads != 64 || d.dim != 128) return LI_ERR_UNSUPPORTED;
+    if (!aligned(k, 16) || !aligned(q, 16)) return LI_ERR_INVALID_ARG;
+    const uint64_t total_rows = cache_batch_rows > 0 ? (uint64_t)(d.rows - 1) * cache_batch_rows + d.max_len
+                                                     : (uint64_t)d.max_len;
+    if (total_rows >= (1ull << 31)) return LI_ERR_UNSUPPORTED;
+    CUtensorMap kmap;
+    if (!encode_map_2d(&kmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, k, 128, total_rows, 128, 128, 128)) return LI_ERR_CUDA;
+
+    if (!d.causal) {
+        StreamArgs a{};
+        a.q = q;
+        a.w = w;
+        a.kscale = k_scale;
+        a.len = len;
+        a.scores = scores;
+        a.scores_ld = scores_ld;
+        a.batch_rows = cache_batch_rows;
+        a.max_len = d.max_len;
+        a.err = e;
+        const int ntiles = (d.max_len + 127) / 128;
+        return launch_stream_score_fp8(kmap, a, d.rows, ntiles, stream);
+    }
+    // causal prefill: quantise all query rows into the workspace, then score
+    const size_t need = li_index_score_workspace(&d);
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return LI_ERR_INVALID_ARG;
+    const size_t nh = (size_t)d.rows * d.heads;
+    uint8_t* q8 = static_cast<uint8_t*>(workspace);
+    float* sq = reinterpret_cast<float*>(q8 + align_up(nh * d.dim, 256));
+    float* weff = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(sq) + align_up(nh * sizeof(float), 256));
+    li_status s = launch_quantize_query(q, w, d.rows, d.heads, d.dim, q8, sq, weff, stream);
+    if (s != LI_OK) return s;
+    CUtensorMap qmap;
+    if (!encode_map_2d(&qmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, q8, 128, nh, 128, 128, 256)) return LI_ERR_CUDA;
+    PrefillArgs pa{weff, k_scale, scores, scores_ld, d.rows, d.max_len, d.causal_offset, e};
+    return launch_prefill_score(qmap, kmap, pa, stream);
+}
+
+li_status li_topk(const float* scores, int64_t scores_ld, const int32_t* len, int rows, int max_len, int causal,
+                  int causal_offset, int k, int32_t* idx, float* vals, li_stream_t stream) {
+    if (rows < 0 || max_len < 0 || k < 1 || k > LI_TOPK_MAX_LEN || max_len > LI_TOPK_MAX_LEN) return LI_ERR_INVALID_ARG;
+    if (rows == 0) return LI_OK;
+    if (!idx || (!scores && max_len > 0) || scores_ld < max_len || (scores_ld % 4) != 0) return LI_ERR_INVALID_ARG;
+    if (scores && !aligned(scores, 16)) return LI_ERR_INVALID_ARG;
+    if (causal && len) return LI_ERR_INVALID_ARG;
+    DevErr e;
+    if (ready(&e) != LI_OK) return LI_ERR_CUDA;
+    TopkArgs a{scores, scores_ld, len, rows, max_len, causal ? 1 : 0, causal_offset, k, idx, vals, nullptr, 0, 1, e};
+    return launch_topk(a, stream);
+}
+
+li_status li_absorb_query(const void* q_bf16, const void* w_dec_bf16, void* q_tilde_bf16, int batch, int heads,
+                          int dim, int latent_dim, li_stream_t stream) {
+    if (batch < 0 || heads <= 0 || dim <= 0 || dim > 256 || latent_dim <= 0 || (latent_dim % 64) != 0 ||
+        heads > 65535)
+        return LI_ERR_INVALID_ARG;
+    if (batch == 0) return LI_OK;
+    if (!q_bf16 || !w_dec_bf16 || !q_tilde_bf16 || !aligned(w_dec_bf16, 4) || !aligned(q_tilde_bf16, 4))
+        return LI_ERR_INVALID_ARG;
+    DevErr e;
+    if (ready(&e) != LI_OK) return LI_ERR_CUDA;
+    return launch_absorb(q_bf16, w_dec_bf16, q_tilde_bf16, batch, heads, dim, latent_dim, stream);
+}
+
+li_status li_latent_score(const void* q_tilde_bf16, const float* w, const void* c_bf16, int64_t cache_batch_rows,
+                          const int32_t* len, float* scores, int64_t scores_ld, int batch, int heads, int latent_dim,
+                          int max_len, li_stream_t stream) {
+    if (batch < 0 || heads <= 0 || latent_dim <= 0 || max_len < 0 || cache_batch_rows < 0) return LI_ERR_INVALID_ARG;
+    if (batch == 0 || max_len == 0) return LI_OK;
+    if (!q_tilde_bf16 || !w || !c_bf16 || !scores || scores_ld < max_len) return LI_ERR_INVALID_ARG;
+    if (heads != 64 || latent_dim != 256) return LI_ERR_UNSUPPORTED;
+    if (!aligned(c_bf16, 16) || !aligned(q_tilde_bf16, 16)) return LI_ERR_INVALID_ARG;
+    DevErr e;
+    if (ready(&e) != LI_OK) return LI_ERR_CUDA;
+    const uint64_t total_rows = cache_batch_rows > 0 ? (uint64_t)(batch - 1) * cache_batch_rows + max_len
+                                                     : (uint64_t)max_len;
+    if (total_rows >= (1ull << 31)) return LI_ERR_UNSUPPORTED;
+    CUtensorMap cmap;
+    if (!encode_map_2d(&cmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c_bf16, 256, total_rows, 512, 64, 128))
+        return LI_ERR_CUDA;
+    StreamArgs a{};
+    a.q = q_tilde_bf16;
+    a.w = w;
+    a.kscale = nullptr;
+    a.len = len;
+    a.scores = scores;
+    a.scores_ld = scores_ld;
+    a.batch_rows = cache_batch_rows;
+    a.max_len = max_len;
+    a.err = e;
+    return launch_stream_score_bf16(cmap, a, batch, (max_len + 127) / 128, stream);
+}
+
+size_t li_hs_refine_workspace(int batch, int n_cand, int followers) {
+    if (batch <= 0 || n_cand <= 0 || followers <= 0) return 0;
+    return (size_t)followers * batch * align_up((size_t)n_cand, 4) * sizeof(float);
+}
+
+li_status li_hs_refine(const void* c_bf16, int64_t cache_batch_rows, int64_t cache_rows, const int32_t* cand,
+                       int batch, int n_cand, const void* q_tilde_bf16, const float* w, int followers, int heads,
+                       int latent_dim, int k, int32_t* out_idx, void* workspace, size_t workspace_bytes,
+                       li_stream_t stream) {
+    if (batch < 0 || n_cand < 0 || followers <= 0 || heads <= 0 || latent_dim <= 0 || k < 1 ||
+        k > LI_TOPK_MAX_LEN || n_cand > LI_TOPK_MAX_LEN || cache_batch_rows < 0 || cache_rows < 0)
+        return LI_ERR_INVALID_ARG;
+    if (batch == 0) return LI_OK;
+    if (!out_idx) return LI_ERR_INVALID_ARG;
+    if (heads != 64 || latent_dim != 256 || followers * heads > 256) return LI_ERR_UNSUPPORTED;
+    DevErr e;
+    if (ready(&e) != LI_OK) return LI_ERR_CUDA;
+    if (n_cand == 0) {
+        TopkArgs t{nullptr, 4, nullptr, followers * batch, 0, 0, 0, k, out_idx, nullptr, nullptr, 0, 1, e};
+        return launch_topk(t, stream);
+    }
+    if (!c_bf16 || !cand || !q_tilde_bf16 || !w || !aligned(c_bf16, 16) || !aligned(q_tilde_bf16, 16))
+        return LI_ERR_INVALID_ARG;
+    const size_t need = li_hs_refine_workspace(batch, n_cand, followers);
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) return LI_ERR_INVALID_ARG;
+    const int ldw = (int)align_up((size_t)n_cand, 4);
+    float* sc = static_cast<float*>(workspace);
+    HsArgs h{c_bf16, cache_batch_rows, cache_rows, cand, batch, n_cand, followers, q_tilde_bf16, w, sc, e};
+    li_status s = launch_hs_rescore(h, stream);
+    if (s != LI_OK) return s;
+    TopkArgs t{sc, ldw, nullptr, followers * batch, n_cand, 0, 0, k, out_idx, nullptr, cand, n_cand, batch, e};
+    return launch_topk(t, stream);
+}
+
+li_status li_selftest_wait_timeout(uint64_t limit_ns, li_stream_t stream) {
+    DevErr e;
+    if (ready(&e) != LI_OK) return LI_ERR_CUDA;
+    return launch_selftest_wait(limit_ns, stream);
+}
+
+}  // extern "C"

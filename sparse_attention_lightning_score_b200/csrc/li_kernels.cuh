@@ -1,0 +1,101 @@
+// Kernel launchers of the li library (host-callable, internal).  Arguments are
+// validated by the C-ABI layer (li_abi.cu) before any of these is reached.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "li.h"
+#include "li_common.cuh"
+
+namespace li {
+
+// ---------------------------------------------------------------- streaming scorer
+struct StreamArgs {
+    const void* q;          // FP8 kind: bf16 [B,64,128]; BF16 kind: bf16 [B,64,256]
+    const float* w;         // [B,64]
+    const float* kscale;    // FP8 kind: one per cache row
+    const int32_t* len;     // [B] or nullptr
+    float* scores;
+    long long scores_ld;
+    long long batch_rows;   // cache rows between requests (0 = shared cache)
+    int max_len;
+    int tiles_per_cta;      // set by the launcher
+    DevErr err;
+};
+li_status launch_stream_score_fp8(const CUtensorMap& map, const StreamArgs& args, int batch, int ntiles_max,
+                                  cudaStream_t st);
+li_status launch_stream_score_bf16(const CUtensorMap& map, const StreamArgs& args, int batch, int ntiles_max,
+                                   cudaStream_t st);
+
+// ---------------------------------------------------------------- causal prefill scorer
+struct PrefillArgs {
+    const float* w_eff;     // [T,64] (w * per-(token, head) query scale)
+    const float* kscale;    // [L]
+    float* scores;
+    long long scores_ld;
+    int T, L;
+    int causal_offset;
+    DevErr err;
+};
+li_status launch_prefill_score(const CUtensorMap& qmap, const CUtensorMap& kmap, const PrefillArgs& args,
+                               cudaStream_t st);
+
+// ---------------------------------------------------------------- query quantiser
+li_status launch_quantize_query(const void* q, const float* w, int rows, int heads, int dim, uint8_t* q8, float* sq,
+                                float* w_eff, cudaStream_t st);
+
+// ---------------------------------------------------------------- exact fp32 scorer
+struct SimtArgs {
+    const float* q;         // [R,H,d]
+    const float* w;         // [R,H]
+    const float* k;         // rows of d
+    const int32_t* len;
+    float* scores;
+    long long scores_ld;
+    long long batch_rows;
+    int R, H, d, L;
+    int causal, causal_offset;
+    DevErr err;
+};
+li_status launch_simt_score(const SimtArgs& a, cudaStream_t st);
+
+// ---------------------------------------------------------------- top-k
+struct TopkArgs {
+    const float* scores;
+    long long ld;
+    const int32_t* len;
+    int rows, max_len, causal, causal_offset, k;
+    int32_t* idx;
+    float* vals;
+    // optional position map (hierarchical selection): row r's slot i reports
+    // map[(r % map_rows) * map_ld + i] instead of i
+    const int32_t* map;
+    long long map_ld;
+    int map_rows;
+    DevErr err;
+};
+li_status launch_topk(const TopkArgs& a, cudaStream_t st);
+
+// ---------------------------------------------------------------- absorption
+li_status launch_absorb(const void* q, const void* wdec, void* qt, int B, int H, int d, int dc, cudaStream_t st);
+
+// ---------------------------------------------------------------- HS gather + rescore
+struct HsArgs {
+    const void* c;          // bf16 latent rows of 256
+    long long batch_rows;
+    long long cache_rows;   // rows addressable from c
+    const int32_t* cand;    // [B, C]
+    int B, C, F;
+    const void* qt;         // bf16 [F,B,64,256]
+    const float* w;         // [F,B,64]
+    float* out;             // [F,B,C] candidate scores (workspace)
+    DevErr err;
+};
+li_status launch_hs_rescore(const HsArgs& a, cudaStream_t st);
+
+// ---------------------------------------------------------------- diagnostics
+li_status launch_selftest_wait(unsigned long long limit_ns, cudaStream_t st);
+
+}  // namespace li

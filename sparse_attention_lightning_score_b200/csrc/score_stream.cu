@@ -1,0 +1,255 @@
+// Streaming indexer scorer for decode: one query token per request scans its
+// whole cache ("scores the whole cache", Multi-layer Indexer abstract).
+//
+//   FP8 kind (DSA decode):   I[b,s] = sk[s] * sum_j w_eff[b,j] * ReLU(q8[b,j,:] . k8[s,:])
+//                            q8/w_eff come from the bf16 query, quantised per
+//                            (request, head) inside the prologue.
+//   BF16 kind (LatentIndex): I[b,s] = sum_j w[b,j] * ReLU(q~[b,j,:] . c[s,:])
+//                            scoring the shared latent cache with the absorbed
+//                            query (LatentIndex abstract and Figure 1).
+//
+// The logits q.k form a [128 keys x 64 heads] tile per step: a dense
+// contraction, so it runs on the tcgen05 tensor cores with the keys as the
+// M=128 operand (one TMEM lane per key) and the heads as N=64.  The head
+// reduction, ReLU and key scale happen in registers after one tcgen05.ld per
+// 32 columns, so the [H, L] logits never reach HBM; only one fp32 score per
+// key is written.
+//
+// Warp roles (192 threads):
+//   warp 0      TMA producer: 128-key x 128-byte tiles of the cache, 128-byte
+//               swizzle, into a STAGES-deep ring of shared-memory stages.
+//   warp 1      TMEM allocator and MMA issuer (one thread): per key tile, the
+//               K/32 (FP8) or K/16 (bf16) MMAs into one of NACC accumulators.
+//   warps 2..5  query preparation, then the epilogue: TMEM -> registers ->
+//               weighted ReLU sum -> one score per key.
+// Grid: (CTAs per request, requests).  Each CTA streams a contiguous range of
+// key tiles of one request; sized for two CTAs per SM.
+#include "li_common.cuh"
+#include "li_kernels.cuh"
+
+namespace li {
+
+namespace {
+
+template <bool FP8, int KBLK, int STAGES, int NACC>
+struct StreamCfg {
+    static constexpr int H = 64;                       // heads = MMA N
+    static constexpr int M = 128;                      // keys per tile = MMA M = TMEM lanes
+    static constexpr int STAGE_BYTES = M * 128;        // one 128-byte K block of 128 keys
+    static constexpr int Q_BYTES = KBLK * H * 128;     // query operand, same K blocks
+    static constexpr int OFF_Q = STAGES * STAGE_BYTES;
+    static constexpr int OFF_W = OFF_Q + Q_BYTES;
+    static constexpr int OFF_BAR = OFF_W + H * 4;
+    static constexpr int NBAR = 2 * STAGES + 2 * NACC + 1;
+    static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
+    static constexpr int SMEM = OFF_TMEM + 16 + 1024;  // + slack to align the base to 1024
+    static constexpr int TMEM_COLS = NACC * H;
+    static constexpr int THREADS = 192;
+    static constexpr int ELEMS_PER_KBLOCK = FP8 ? 128 : 64;
+    static_assert(TMEM_COLS == 128 || TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM columns");
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+template <bool FP8, int KBLK, int STAGES, int NACC>
+__global__ void __launch_bounds__(192) stream_score_kernel(const __grid_constant__ CUtensorMap kmap,
+                                                           const StreamArgs a) {
+    using C = StreamCfg<FP8, KBLK, STAGES, NACC>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+
+    const int b = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int len_b = a.len ? __ldg(a.len + b) : a.max_len;
+    if (len_b < 0 || len_b > a.max_len) {
+        if (threadIdx.x == 0 && blockIdx.x == 0) record_error(a.err, ERRBIT_BOUNDS);
+        len_b = len_b < 0 ? 0 : a.max_len;
+    }
+    const int ntiles = (len_b + C::M - 1) / C::M;
+    const int t0 = blockIdx.x * a.tiles_per_cta;
+    const int nt = min(t0 + a.tiles_per_cta, ntiles) - t0;
+    if (nt <= 0) return;  // uniform over the CTA
+
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* empty = full + STAGES;
+    uint64_t* accf = empty + STAGES;
+    uint64_t* acce = accf + NACC;
+    uint64_t* qready = acce + NACC;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
+    float* wsm = reinterpret_cast<float*>(smem + C::OFF_W);
+    uint8_t* qsm = smem + C::OFF_Q;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int i = 0; i < NACC; ++i) {
+            mbar_init(&accf[i], 1);
+            mbar_init(&acce[i], 128);
+        }
+        mbar_init(qready, 128);
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            tma_prefetch_desc(&kmap);
+            const uint64_t pol = l2_policy_evict_first();
+            const long long rowbase = (long long)b * a.batch_rows;
+            int stage = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int it = 0; ok && it < nt; ++it) {
+                const int y = (int)(rowbase + (long long)(t0 + it) * C::M);
+                for (int kb = 0; kb < KBLK; ++kb) {
+                    if (!mbar_wait(&empty[stage], ph ^ 1u, a.err)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+                    tma_load_2d(smem + stage * C::STAGE_BYTES, &kmap, kb * C::ELEMS_PER_KBLOCK, y, &full[stage],
+                                pol);
+                    if (++stage == STAGES) { stage = 0; ph ^= 1u; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t IDESC = idesc_f32acc(C::M, C::H, FP8 ? kFmtE4M3 : kFmtBF16);
+            bool ok = mbar_wait(qready, 0, a.err);
+            tc_fence_after();
+            const uint32_t qaddr = smem_u32(qsm);
+            int stage = 0;
+            uint32_t ph = 0;
+            for (int it = 0; ok && it < nt; ++it) {
+                const int acc = it % NACC;
+                const uint32_t aph = (uint32_t)(it / NACC) & 1u;
+                if (!mbar_wait(&acce[acc], aph ^ 1u, a.err)) break;
+                tc_fence_after();
+                const uint32_t dt = tmem_base + (uint32_t)(acc * C::H);
+                for (int kb = 0; kb < KBLK; ++kb) {
+                    if (!mbar_wait(&full[stage], ph, a.err)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t aaddr = smem_u32(smem + stage * C::STAGE_BYTES);
+                    const uint32_t baddr = qaddr + (uint32_t)(kb * C::H * 128);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {  // 32-byte K slices of the 128-byte row
+                        const uint64_t ad = sw128_kmajor_desc(aaddr + kk * 32);
+                        const uint64_t bd = sw128_kmajor_desc(baddr + kk * 32);
+                        if constexpr (FP8) mma_e4m3(dt, ad, bd, IDESC, (kb | kk) != 0);
+                        else mma_bf16(dt, ad, bd, IDESC, (kb | kk) != 0);
+                    }
+                    tc_commit(&empty[stage]);
+                    if (++stage == STAGES) { stage = 0; ph ^= 1u; }
+                }
+                if (!ok) break;
+                tc_commit(&accf[acc]);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ query prep
+        const int et = threadIdx.x - 64;  // 0..127
+        const int ew = et >> 5;
+        if constexpr (FP8) {
+            const __nv_bfloat16* q = reinterpret_cast<const __nv_bfloat16*>(a.q) + (size_t)b * C::H * 128;
+            for (int j = ew; j < C::H; j += 4) {
+                const uint2 raw = __ldg(reinterpret_cast<const uint2*>(q + (size_t)j * 128) + lane);
+                float sq;
+                const uint32_t packed = quantize_head128(raw, &sq);
+                *reinterpret_cast<uint32_t*>(qsm + sw128_offset(j, lane >> 2) + (lane & 3) * 4) = packed;
+                if (lane == 0) wsm[j] = __ldg(a.w + (size_t)b * C::H + j) * sq;
+            }
+        } else {
+            constexpr int CH = KBLK * 8;  // 16-byte chunks per query row
+            const uint4* src =
+                reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.q) + (size_t)b * C::H * KBLK * 64);
+            for (int ci = et; ci < C::H * CH; ci += 128) {
+                const int r = ci / CH, cc = ci % CH;
+                const uint4 v = __ldg(src + ci);
+                *reinterpret_cast<uint4*>(qsm + (cc >> 3) * (C::H * 128) + sw128_offset(r, cc & 7)) = v;
+            }
+            for (int j = et; j < C::H; j += 128) wsm[j] = __ldg(a.w + (size_t)b * C::H + j);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(qready);
+        asm volatile("bar.sync 1, 128;" ::: "memory");  // w_eff visible to every epilogue thread
+
+        // ------------------------------------------------------------ epilogue
+        const int g = warp & 3;  // TMEM lane quarter this warp may access
+        const long long srow = (long long)b * a.batch_rows;
+        float* out = a.scores + (size_t)b * a.scores_ld;
+        for (int it = 0; it < nt; ++it) {
+            const int acc = it % NACC;
+            const uint32_t aph = (uint32_t)(it / NACC) & 1u;
+            const int s = (t0 + it) * C::M + g * 32 + lane;
+            float sk = 1.f;
+            if (FP8 && s < len_b) sk = __ldg(a.kscale + srow + s);
+            if (!mbar_wait(&accf[acc], aph, a.err)) break;
+            tc_fence_after();
+            const uint32_t tb = tmem_base + ((uint32_t)(g * 32) << 16) + (uint32_t)(acc * C::H);
+            uint32_t v0[32], v1[32];
+            tmem_ld32(tb, v0);
+            tmem_ld32(tb + 32, v1);
+            tmem_ld_wait();
+            tc_fence_before();
+            mbar_arrive(&acce[acc]);
+            const float sum = relu_dot32(v0, wsm) + relu_dot32(v1, wsm + 32);
+            if (s < len_b) out[s] = FP8 ? sum * sk : sum;
+        }
+    }
+    __syncwarp();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+template <bool FP8, int KBLK, int STAGES, int NACC>
+li_status launch_impl(const CUtensorMap& map, const StreamArgs& args, int batch, int ntiles_max, cudaStream_t st) {
+    using C = StreamCfg<FP8, KBLK, STAGES, NACC>;
+    auto kern = stream_score_kernel<FP8, KBLK, STAGES, NACC>;
+    static bool attr_done[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_done[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+            return host_check_launch();
+        attr_done[dev] = true;
+    }
+    const int sms = host_num_sms();
+    // two CTAs per SM in total, spread over the requests; contiguous tile ranges
+    int cpr = max(1, (2 * sms) / max(1, batch));
+    int tpc = (ntiles_max + cpr - 1) / cpr;
+    tpc = max(tpc, 1);
+    cpr = (ntiles_max + tpc - 1) / tpc;
+    StreamArgs a = args;
+    a.tiles_per_cta = tpc;
+    dim3 grid(max(cpr, 1), batch);
+    kern<<<grid, C::THREADS, C::SMEM, st>>>(map, a);
+    return host_check_launch();
+}
+
+}  // namespace
+
+li_status launch_stream_score_fp8(const CUtensorMap& map, const StreamArgs& args, int batch, int ntiles_max,
+                                  cudaStream_t st) {
+    return launch_impl<true, 1, 6, 4>(map, args, batch, ntiles_max, st);
+}
+
+li_status launch_stream_score_bf16(const CUtensorMap& map, const StreamArgs& args, int batch, int ntiles_max,
+                                   cudaStream_t st) {
+    return launch_impl<false, 4, 4, 4>(map, args, batch, ntiles_max, st);
+}
+
+}  // namespace li

@@ -1,0 +1,71 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every symbol include/li.h declares, and rejects bad arguments before it touches
+the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_attention_lightning_score_b200 import _lib
+
+HDR = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "li.h")
+
+
+def declared_symbols():
+    src = open(HDR).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\**\s*(li_[a-z0-9_]+)\s*\(", src, re.M)))
+
+
+def test_header_declares_the_boundary():
+    syms = declared_symbols()
+    for name in ["li_absorb_query", "li_index_score", "li_topk", "li_latent_score", "li_hs_refine",
+                 "li_get_last_error", "li_quantize_query"]:
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _lib.load()
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+        assert name in _lib.SIGNATURES, name
+
+
+def test_status_strings():
+    assert _lib.status_string(_lib.LI_OK) == "LI_OK"
+    assert _lib.status_string(_lib.LI_ERR_TIMEOUT) == "LI_ERR_TIMEOUT"
+
+
+def test_invalid_arguments_rejected_on_host():
+    lib = _lib.load()
+    p = ctypes.c_void_p(16)
+    # k out of range, negative sizes, unaligned leading dimension, null descriptor
+    assert lib.li_topk(p, 4, None, 1, 4, 0, 0, 0, p, None, None) == _lib.LI_ERR_INVALID_ARG
+    assert lib.li_topk(p, 4, None, 1, 4, 0, 0, _lib.LI_TOPK_MAX_LEN + 1, p, None, None) == _lib.LI_ERR_INVALID_ARG
+    assert lib.li_topk(p, 6, None, 1, 6, 0, 0, 2, p, None, None) == _lib.LI_ERR_INVALID_ARG
+    assert lib.li_topk(p, 4, None, -1, 4, 0, 0, 2, p, None, None) == _lib.LI_ERR_INVALID_ARG
+    assert lib.li_index_score(p, p, p, p, 0, None, p, 8, None, None, 0, None) == _lib.LI_ERR_INVALID_ARG
+    d = _lib.ScoreDesc(2, 64, 128, 100, 0, 0, _lib.LI_DTYPE_BF16, _lib.LI_DTYPE_E4M3)
+    assert lib.li_index_score(p, p, p, p, 0, None, p, 50, ctypes.byref(d), None, 0, None) == _lib.LI_ERR_INVALID_ARG
+    d.causal = 1
+    assert lib.li_index_score(p, p, p, p, 100, None, p, 100, ctypes.byref(d), None, 0, None) == _lib.LI_ERR_INVALID_ARG
+    assert lib.li_absorb_query(p, p, p, 1, 64, 128, 100, None) == _lib.LI_ERR_INVALID_ARG
+    assert lib.li_hs_refine(p, 0, 10, p, 1, 8, p, p, 0, 64, 256, 4, p, p, 0, None) == _lib.LI_ERR_INVALID_ARG
+
+
+def test_zero_sized_calls_are_no_ops():
+    lib = _lib.load()
+    p = ctypes.c_void_p(16)
+    assert lib.li_topk(p, 4, None, 0, 4, 0, 0, 2, p, None, None) == _lib.LI_OK
+    d = _lib.ScoreDesc(0, 64, 128, 100, 0, 0, _lib.LI_DTYPE_BF16, _lib.LI_DTYPE_E4M3)
+    assert lib.li_index_score(p, p, p, p, 0, None, p, 100, ctypes.byref(d), None, 0, None) == _lib.LI_OK
+
+
+def test_workspace_sizes():
+    lib = _lib.load()
+    d = _lib.ScoreDesc(8192, 64, 128, 8192, 1, 0, _lib.LI_DTYPE_BF16, _lib.LI_DTYPE_E4M3)
+    assert lib.li_index_score_workspace(ctypes.byref(d)) >= 8192 * 64 * (128 + 8)
+    d.causal = 0
+    assert lib.li_index_score_workspace(ctypes.byref(d)) == 0
+    assert lib.li_hs_refine_workspace(16, 8192, 3) == 3 * 16 * 8192 * 4

@@ -1,0 +1,209 @@
+"""GPU parity: every CUDA path against the fp64 oracle on the same seeded inputs.
+
+Integer work (quantised bytes, top-k indices on identical fp32 inputs, HS
+gathers) must match bit for bit; floating-point scores must match within the
+tolerance of tests/_checks.py.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_attention_lightning_score_b200 import api, synth
+from sparse_attention_lightning_score_b200._lib import LI_ERR_BOUNDS, LI_ERR_TIMEOUT, LI_OK, LiError
+from tests._checks import assert_scores_close, assert_topk_equivalent
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _np(t):
+    return t.detach().cpu().numpy()
+
+
+# ---------------------------------------------------------------------------
+# query quantisation: bit-exact bytes, scales and folded weights
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("R,H,d", [(8, 64, 128), (3, 5, 96), (1, 64, 128)])
+def test_quantize_query_bit_exact(R, H, d):
+    g = torch.Generator().manual_seed(R * 100 + d)
+    q = (torch.randn(R, H, d, generator=g) * torch.exp(torch.randn(R, H, 1, generator=g) * 3)).to(torch.bfloat16)
+    q[0, 0] = 0.0                      # all-zero head
+    q[0, 1 % H, :4] = torch.tensor([1.0, -2.0, 0.5, 4.0])
+    q[-1, -1] *= 1e-30                 # tiny values (bf16 keeps the exponent range)
+    w = torch.randn(R, H, generator=g)
+    q8_o, sq_o, we_o = oracle.quantize_query(q, w.numpy())
+    q8, sq, we = api.li_quantize_query(q.to(DEV), w.to(DEV))
+    assert np.array_equal(_np(q8), q8_o)
+    assert np.array_equal(_np(sq).view(np.uint32), sq_o.view(np.uint32))
+    assert np.array_equal(_np(we).view(np.uint32), we_o.view(np.uint32))
+
+
+# ---------------------------------------------------------------------------
+# tiny fp32 case: exact scalar path, tolerance 1e-4
+# ---------------------------------------------------------------------------
+def test_tiny_fp32_score_and_topk():
+    case = synth.tiny_fp32()
+    ref, mag = oracle.index_score(case.q, oracle.F32, case.w, case.k, oracle.F32, with_mag=True)
+    sc = api.li_index_score(case.q.to(DEV), case.w.to(DEV), case.k.to(DEV))
+    L = case.k.shape[0]
+    assert_scores_close(_np(sc)[:, :L], ref, mag, 1e-4)
+    idx = api.li_topk(sc, case.k_top, max_len=L)
+    ridx, _ = oracle.topk(ref, case.k_top)
+    assert_topk_equivalent(_np(idx), ridx, ref, 1e-4)
+    assert set(case.planted.tolist()) <= set(_np(idx)[0].tolist())
+
+
+# ---------------------------------------------------------------------------
+# DSA decode scorer (FP8, tcgen05)
+# ---------------------------------------------------------------------------
+def _oracle_decode(case, rows=None):
+    q8, sq, _ = oracle.quantize_query(case.q, case.w.numpy())
+    L = case.k8.shape[1]
+    return oracle.index_score(q8, oracle.E4M3, case.w, case.k8, oracle.E4M3, q_scale=sq, k_scale=case.ks,
+                              k_batch_rows=L, L=L, lens=case.lens.numpy(), rows=rows, with_mag=True)
+
+
+@pytest.mark.parametrize("B,L,lens", [(3, 1000, [1000, 517, 129]), (2, 4096, None), (5, 300, [0, 1, 127, 128, 300])])
+def test_dsa_decode_scores(B, L, lens):
+    case = synth.dsa_decode(B=B, L=L, seed=21, lens=lens)
+    ref, mag = _oracle_decode(case)
+    sc = api.li_index_score(case.q.to(DEV), case.w.to(DEV), case.k8.to(DEV), case.ks.to(DEV),
+                            lens=case.lens.to(DEV))
+    assert_scores_close(_np(sc)[:, :L], ref, mag, 1e-2)
+    assert api.li_get_last_error() == LI_OK
+
+
+def test_dsa_decode_shared_cache():
+    case = synth.dsa_decode(B=4, L=777, seed=22)
+    k8, ks = case.k8[0], case.ks[0]
+    q8, sq, _ = oracle.quantize_query(case.q, case.w.numpy())
+    ref, mag = oracle.index_score(q8, oracle.E4M3, case.w, k8, oracle.E4M3, q_scale=sq, k_scale=ks, with_mag=True)
+    sc = api.li_index_score(case.q.to(DEV), case.w.to(DEV), k8.to(DEV), ks.to(DEV))
+    assert_scores_close(_np(sc)[:, :777], ref, mag, 1e-2)
+
+
+def test_dsa_decode_bench_config_full():
+    """The benchmarked decode step at full size (B=8, L=32768): every score and
+    every top-2048 selection against the oracle."""
+    case = synth.dsa_decode()  # B=8, L=32768, k=2048
+    ref, mag = _oracle_decode(case)
+    q, w, k8, ks = case.q.to(DEV), case.w.to(DEV), case.k8.to(DEV), case.ks.to(DEV)
+    sc = api.li_index_score(q, w, k8, ks)
+    assert_scores_close(_np(sc)[:, :32768], ref, mag, 1e-2)
+    idx = api.li_topk(sc, 2048, max_len=32768)
+    ridx, _ = oracle.topk(ref, 2048)
+    assert_topk_equivalent(_np(idx), ridx, ref, 1e-2)
+    assert api.li_get_last_error() == LI_OK
+
+
+# ---------------------------------------------------------------------------
+# top-k: bit-exact against the oracle on identical fp32 rows
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("rows,L,k,ties", [(8, 32768, 2048, 0), (1, 131072, 8192, 0), (16, 131072, 2048, 0),
+                                           (3, 5000, 100, 7), (200, 3000, 64, 0), (2, 262144, 2048, 3),
+                                           (4, 4096, 4096, 0), (6, 100, 2048, 0), (1, 9, 3, 2)])
+def test_topk_bit_exact(rows, L, k, ties):
+    s = synth.score_rows(rows, L, seed=rows + L + k, ties=ties)
+    ld = (L + 3) // 4 * 4
+    buf = torch.full((rows, ld), float("nan"))
+    buf[:, :L] = s
+    idx, vals = api.li_topk(buf.to(DEV), k, max_len=L, with_values=True)
+    ridx, rvals = oracle.topk(s.double().numpy(), k)
+    assert np.array_equal(_np(idx), ridx)
+    assert np.array_equal(_np(vals).astype(np.float64), rvals)
+
+
+def test_topk_ragged_and_causal_rows():
+    rows, L, k = 300, 2500, 256
+    s = synth.score_rows(rows, L, seed=31)
+    lens = torch.randint(0, L + 1, (rows,), generator=torch.Generator().manual_seed(3), dtype=torch.int32)
+    lens[:4] = torch.tensor([0, 1, k, k + 1], dtype=torch.int32)
+    sd = s.to(DEV)
+    idx = api.li_topk(sd, k, lens=lens.to(DEV), max_len=L)
+    ridx, _ = oracle.topk(s.double().numpy(), k, lens=lens.numpy())
+    assert np.array_equal(_np(idx), ridx)
+    idx = api.li_topk(sd, k, causal=True, causal_offset=5, max_len=L)
+    ridx, _ = oracle.topk(s.double().numpy(), k, causal=True, causal_offset=5, max_len=L)
+    assert np.array_equal(_np(idx), ridx)
+
+
+def test_topk_special_values():
+    row = torch.tensor([[float("nan"), -0.0, 0.0, float("-inf"), 1.0, float("nan"), 0.0, -0.0]])
+    for k in (1, 2, 3, 5, 7):
+        idx = api.li_topk(row.to(DEV), k)
+        ridx, _ = oracle.topk(row.double().numpy(), k)
+        assert np.array_equal(_np(idx), ridx), k
+    eq = torch.full((2, 40000), 1.5)
+    idx = api.li_topk(eq.to(DEV), 2048)
+    assert np.array_equal(_np(idx), np.tile(np.arange(2048, dtype=np.int32), (2, 1)))
+
+
+# ---------------------------------------------------------------------------
+# LatentIndex: absorption and latent scoring
+# ---------------------------------------------------------------------------
+def test_absorb_matches_oracle():
+    case = synth.latent_group(B=5, L=8, seed=41)
+    for layer in range(2):
+        qt = api.li_absorb_query(case.q[layer].to(DEV), case.w_dec[layer].to(DEV))
+        ref = oracle.absorb(case.q[layer], case.w_dec[layer])
+        got = qt.float().cpu().double().numpy()
+        absq = np.abs(case.q[layer].double().numpy())
+        absw = np.abs(case.w_dec[layer].double().numpy())
+        cond = np.einsum("bjd,jdc->bjc", absq, absw)
+        # one round-to-nearest into bf16 (8 significant bits: relative error <= 2^-8)
+        # plus fp32 accumulation over d terms
+        assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-5 * cond)
+
+
+@pytest.mark.parametrize("B,L,lens", [(3, 1000, [1000, 333, 1]), (2, 5000, None)])
+def test_latent_scores(B, L, lens):
+    case = synth.latent_group(B=B, L=L, seed=42, lens=lens, plant_frac=0.01)
+    qt = api.li_absorb_query(case.q[0].to(DEV), case.w_dec[0].to(DEV))
+    ref, mag = oracle.latent_score(qt.cpu(), oracle.BF16, case.w[0], case.c, lens=case.lens.numpy(), with_mag=True)
+    sc = api.li_latent_score(qt, case.w[0].to(DEV), case.c.to(DEV), lens=case.lens.to(DEV))
+    assert_scores_close(_np(sc)[:, :L], ref, mag, 1e-2)
+    assert api.li_get_last_error() == LI_OK
+
+
+def test_latent_group_step_against_fp64_definition():
+    """One G=4 group step at reduced length: absorb -> score -> top-k per layer,
+    against the oracle's fp64 absorption (no bf16 rounding of q~)."""
+    case = synth.latent_group(B=2, L=6000, seed=43)
+    c = case.c.to(DEV)
+    for layer in range(4):
+        qt = api.li_absorb_query(case.q[layer].to(DEV), case.w_dec[layer].to(DEV))
+        sc = api.li_latent_score(qt, case.w[layer].to(DEV), c)
+        idx = api.li_topk(sc, 512, max_len=6000)
+        qt64 = oracle.absorb(case.q[layer], case.w_dec[layer])
+        ref, mag = oracle.latent_score(qt64, oracle.F64, case.w[layer], case.c, with_mag=True)
+        assert_scores_close(_np(sc)[:, :6000], ref, mag, 1e-2)
+        ridx, _ = oracle.topk(ref, 512)
+        assert_topk_equivalent(_np(idx), ridx, ref, 1e-2)
+
+
+# ---------------------------------------------------------------------------
+# failure path: bounded waits and out-of-range lengths report, never trap
+# ---------------------------------------------------------------------------
+def test_bounded_wait_reports_timeout():
+    assert api.li_get_last_error() == LI_OK
+    api.li_selftest_wait_timeout(1_000_000)  # 1 ms
+    assert api.li_get_last_error() == LI_ERR_TIMEOUT
+    assert api.li_get_last_error() == LI_OK
+
+
+def test_bad_length_reports_bounds():
+    case = synth.dsa_decode(B=2, L=256, seed=5)
+    lens = torch.tensor([256, 9999], dtype=torch.int32, device=DEV)
+    api.li_index_score(case.q.to(DEV), case.w.to(DEV), case.k8.to(DEV), case.ks.to(DEV), lens=lens)
+    assert api.li_get_last_error() == LI_ERR_BOUNDS
+    assert api.li_get_last_error() == LI_OK
+
+
+def test_unsupported_shapes_raise():
+    q = torch.zeros(2, 32, 128, dtype=torch.bfloat16, device=DEV)
+    w = torch.zeros(2, 32, device=DEV)
+    k = torch.zeros(2, 64, 128, dtype=torch.uint8, device=DEV)
+    ks = torch.ones(2, 64, device=DEV)
+    with pytest.raises(LiError):
+        api.li_index_score(q, w, k, ks)
