@@ -283,11 +283,8 @@ def run_li(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    from sparse_attention_lightning_score_b200 import dist as li_dist
+    dist = li_dist.init("nccl", device=dev) if world > 1 else None
 
     bench = DecodeBench(dev, L, seed=1 + rank)
     bench.build_graphs(args.warmup)
@@ -307,10 +304,7 @@ def run_li(args, rank, world, local_rank):
     score_ms = bench.time_kernel("score")
     topk_ms = bench.time_kernel("topk")
     direct_ms = bench.time_direct(args.steps)
-    if dist:
-        t = torch.tensor([ms, score_ms, topk_ms, direct_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, score_ms, topk_ms, direct_ms = t.tolist()
+    ms, score_ms, topk_ms, direct_ms = li_dist.max_over_ranks([ms, score_ms, topk_ms, direct_ms], device=dev)
     launches = 2 * args.steps
 
     # ---- end to end through the public API: pinned host q/w in, indices out,
@@ -340,10 +334,7 @@ def run_li(args, rank, world, local_rank):
     a1.record()
     torch.cuda.synchronize()
     e2e_ms = a0.elapsed_time(a1) / args.steps
-    if dist:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = t.item()
+    (e2e_ms,) = li_dist.max_over_ranks([e2e_ms], device=dev)
     assert api.li_get_last_error() == 0
 
     sweep = None
@@ -409,9 +400,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    from sparse_attention_lightning_score_b200.dist import env_rank
+    rank, world, local_rank = env_rank()
     if args.impl == "reference":
         run_reference(args, rank)
         return
