@@ -190,6 +190,30 @@ li_status li_hs_refine(const void* c_bf16, int64_t cache_batch_rows, int64_t cac
 
 size_t li_hs_refine_workspace(int batch, int n_cand, int followers);
 
+/* Capacity, in floats (4 MiB), of the fixed scratch behind li_hs_refine_noalloc. */
+#define LI_HS_NOALLOC_MAX_SCRATCH_FLOATS 1048576
+
+/* li_hs_refine without a workspace argument, for callers that cannot
+ * allocate device memory: for example code inside an engine that owns and
+ * budgets all device memory and forbids allocation while serving, or a
+ * plugin that receives only its inputs and outputs.  The pages have no
+ * counterpart to this call; it exists only for such callers.
+ *
+ * Same arguments, results and errors as li_hs_refine.  The followers'
+ * candidate scores go to a file-scope device array of
+ * LI_HS_NOALLOC_MAX_SCRATCH_FLOATS floats that every GPU loading the library
+ * holds until the process exits; the call allocates nothing.
+ *   - followers * batch * round_up(n_cand, 4) above that capacity returns
+ *     LI_ERR_INVALID_ARG before anything is launched.
+ *   - The array is shared by all calls on a device and keeps the last call's
+ *     contents; nothing in it needs to start at zero.  Calls that overlap on
+ *     the GPU (unordered streams) race on it: serialise them.
+ *   - The first call on a device looks up the array's device address; make
+ *     that first call before any stream capture begins. */
+li_status li_hs_refine_noalloc(const void* c_bf16, int64_t cache_batch_rows, int64_t cache_rows, const int32_t* cand,
+                               int batch, int n_cand, const void* q_tilde_bf16, const float* w, int followers,
+                               int heads, int latent_dim, int k, int32_t* out_idx, li_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Diagnostics                                                               */
 /* ------------------------------------------------------------------------ */

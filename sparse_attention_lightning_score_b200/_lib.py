@@ -14,6 +14,7 @@ LIB_PATH = os.path.join(_PKG, "libli.so")
 LI_OK, LI_ERR_INVALID_ARG, LI_ERR_UNSUPPORTED, LI_ERR_CUDA, LI_ERR_TIMEOUT, LI_ERR_BOUNDS = range(6)
 LI_DTYPE_F32, LI_DTYPE_BF16, LI_DTYPE_E4M3 = 0, 1, 2
 LI_TOPK_MAX_LEN = 262144
+LI_HS_NOALLOC_MAX_SCRATCH_FLOATS = 1048576
 
 vp = ctypes.c_void_p
 i32 = ctypes.c_int
@@ -38,6 +39,7 @@ SIGNATURES = {
     "li_latent_score": (i32, [vp, vp, vp, i64, vp, vp, i64, i32, i32, i32, i32, vp]),
     "li_hs_refine": (i32, [vp, i64, i64, vp, i32, i32, vp, vp, i32, i32, i32, i32, vp, vp, sz, vp]),
     "li_hs_refine_workspace": (sz, [i32, i32, i32]),
+    "li_hs_refine_noalloc": (i32, [vp, i64, i64, vp, i32, i32, vp, vp, i32, i32, i32, i32, vp, vp]),
     "li_selftest_wait_timeout": (i32, [ctypes.c_uint64, vp]),
 }
 
