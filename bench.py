@@ -389,6 +389,226 @@ def run_li(args, rank, world, local_rank):
     print(json.dumps(out), flush=True)
 
 
+# ---------------------------------------------------------------------------
+# other configurations (parity-test workloads; timed on request with --workload)
+# ---------------------------------------------------------------------------
+def fp8_peak_tflops():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        # FP8 dense = 2 x the measured bf16 dense rate (nominal 4.5 : 2.25 PF ratio)
+        return 2.0 * float(d["bf16_tflops"]), 2.0 * float(d["bf16_tflops_sustained"]), "measured bf16 x 2"
+    return 2 * 1590.0, 2 * 1400.0, "fallback bf16 x 2"
+
+
+class PrefillBench:
+    """Causal prefill: T = L = 8192, quantise + score (s <= t) + top-2048 per row."""
+
+    def __init__(self, dev):
+        import torch
+        from sparse_attention_lightning_score_b200 import api, synth
+        self.api = api
+        self.T = self.L = 8192
+        case = synth.dsa_prefill(T=self.T, L=self.L)
+        self.q, self.w = case.q.to(dev), case.w.to(dev)
+        self.k8, self.ks = case.k8.to(dev), case.ks.to(dev)
+        self.sc = torch.empty((self.T, self.L), dtype=torch.float32, device=dev)
+        self.idx = torch.empty((self.T, KTOP), dtype=torch.int32, device=dev)
+        from sparse_attention_lightning_score_b200 import _lib
+        desc = api.score_desc(self.T, H, D, self.L, causal=True)
+        import ctypes
+        self.ws = torch.empty(_lib.load().li_index_score_workspace(ctypes.byref(desc)), dtype=torch.uint8, device=dev)
+        self.pairs = self.T * (self.T + 1) // 2
+
+    def score(self):
+        self.api.li_index_score(self.q, self.w, self.k8, self.ks, causal=True, scores=self.sc, workspace=self.ws)
+
+    def topk(self):
+        self.api.li_topk(self.sc, KTOP, causal=True, max_len=self.L, idx=self.idx)
+
+    def run(self, steps, warmup):
+        import torch
+        for _ in range(warmup):
+            self.score()
+            self.topk()
+        torch.cuda.synchronize()
+        gs = capture([self.score, self.topk])
+        g_sc = capture([self.score])
+        g_tk = capture([self.topk])
+        res = {}
+        for name, g in (("step", gs), ("score", g_sc), ("topk", g_tk)):
+            g.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(steps):
+                g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            res[name] = e0.elapsed_time(e1) / steps
+        return res
+
+
+class LatentBench:
+    """LatentIndex G=4 group decode: 4 x (absorb + latent score + top-2048), B=4, L=65536."""
+
+    def __init__(self, dev, B=4, Lx=65536):
+        import torch
+        from sparse_attention_lightning_score_b200 import api, synth
+        self.api = api
+        self.B, self.L = B, Lx
+        case = synth.latent_group(B=B, L=Lx)
+        self.c = [case.c.to(dev)]
+        per = case.c.numel() * 2
+        while len(self.c) * per < 1.5 * L2_BYTES:
+            self.c.append(self.c[0].clone())
+        self.q = [case.q[l].to(dev) for l in range(4)]
+        self.wd = [case.w_dec[l].to(dev) for l in range(4)]
+        self.w = [case.w[l].to(dev) for l in range(4)]
+        self.qt = torch.empty((B, H, 256), dtype=torch.bfloat16, device=dev)
+        self.sc = torch.empty((B, Lx), dtype=torch.float32, device=dev)
+        self.idx = torch.empty((4, B, KTOP), dtype=torch.int32, device=dev)
+
+    def layer(self, i, l):
+        self.api.li_absorb_query(self.q[l], self.wd[l], out=self.qt)
+        self.api.li_latent_score(self.qt, self.w[l], self.c[i % len(self.c)], scores=self.sc)
+        self.api.li_topk(self.sc, KTOP, idx=self.idx[l])
+
+    def run(self, steps, warmup):
+        import torch
+        for i in range(warmup):
+            for l in range(4):
+                self.layer(i, l)
+        torch.cuda.synchronize()
+        graphs = [capture([lambda i=i, l=l: self.layer(i, l) for l in range(4)]) for i in range(len(self.c))]
+        g_sc = capture([lambda i=i: self.api.li_latent_score(self.qt, self.w[0], self.c[i % len(self.c)], scores=self.sc)
+                        for i in range(8)])
+        for g in graphs:
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(steps):
+            graphs[i % len(graphs)].replay()
+        e1.record()
+        torch.cuda.synchronize()
+        step = e0.elapsed_time(e1) / steps
+        e0.record()
+        g_sc.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        return {"step": step, "score": e0.elapsed_time(e1) / 8}
+
+
+class HsBench:
+    """HS decode at L=131072: anchor absorb + scan + top-8192, 3 follower absorbs + refine."""
+
+    def __init__(self, dev, B):
+        import torch
+        from sparse_attention_lightning_score_b200 import api, synth
+        self.api = api
+        self.B, self.L, self.C = B, 131072, 8192
+        case = synth.latent_hs(B=B, L=self.L)
+        self.c = [case.c.to(dev)]
+        per = case.c.numel() * 2
+        while len(self.c) * per < 1.5 * L2_BYTES:
+            self.c.append(self.c[0].clone())
+        self.q = [case.q[l].to(dev) for l in range(4)]
+        self.wd = [case.w_dec[l].to(dev) for l in range(4)]
+        self.w0 = case.w[0].to(dev)
+        self.wf = case.w[1:].contiguous().to(dev)
+        self.qt0 = torch.empty((B, H, 256), dtype=torch.bfloat16, device=dev)
+        self.qtf = torch.empty((3, B, H, 256), dtype=torch.bfloat16, device=dev)
+        self.sc = torch.empty((B, self.L), dtype=torch.float32, device=dev)
+        self.cand = torch.empty((B, self.C), dtype=torch.int32, device=dev)
+        self.out = torch.empty((3, B, KTOP), dtype=torch.int32, device=dev)
+        self.ws = torch.empty(3 * B * self.C * 4, dtype=torch.uint8, device=dev)
+
+    def step(self, i):
+        c = self.c[i % len(self.c)]
+        self.api.li_absorb_query(self.q[0], self.wd[0], out=self.qt0)
+        self.api.li_latent_score(self.qt0, self.w0, c, scores=self.sc)
+        self.api.li_topk(self.sc, self.C, idx=self.cand)
+        for f in range(3):
+            self.api.li_absorb_query(self.q[1 + f], self.wd[1 + f], out=self.qtf[f])
+        self.api.li_hs_refine(c, self.cand, self.qtf, self.wf, KTOP, out=self.out, workspace=self.ws)
+
+    def run(self, steps, warmup):
+        import torch
+        for i in range(warmup):
+            self.step(i)
+        torch.cuda.synchronize()
+        graphs = [capture([lambda i=i: self.step(i)]) for i in range(len(self.c))]
+        for g in graphs:
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(steps):
+            graphs[i % len(graphs)].replay()
+        e1.record()
+        torch.cuda.synchronize()
+        return {"step": e0.elapsed_time(e1) / steps}
+
+
+def run_other(args, rank, world, local_rank):
+    import torch
+    from sparse_attention_lightning_score_b200 import api
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    hbm, which = peaks()
+    fp8_burst, fp8_sust, fp8_src = fp8_peak_tflops()
+    clocks = ClockSampler(local_rank)
+    if args.workload == "prefill":
+        bx = PrefillBench(dev)
+        clocks.start()
+        r = bx.run(args.steps, args.warmup)
+        clk = clocks.stop()
+        flops = bx.pairs * 2 * H * D
+        achieved = flops / (r["score"] * 1e-3) / 1e12
+        out = {"metric": METRIC, "value": bx.pairs / (r["step"] * 1e-3), "unit": "keys/s (visible pairs)",
+               "ms_per_step": r["step"], "higher_is_better": True, "dtype": "e4m3",
+               "config": {"workload": "dsa_prefill_t8k", "T": bx.T, "L": bx.L, "H": H, "d": D, "k": KTOP},
+               "roofline": {"bound": "tensor", "kernel": "quantize_query_kernel + prefill_score_kernel",
+                            "achieved": achieved, "peak": fp8_burst, "peak_source": fp8_src, "unit": "TFLOP/s",
+                            "frac": achieved / fp8_burst, "frac_of_sustained": achieved / fp8_sust,
+                            "score_ms": r["score"]},
+               "topk": {"ms": r["topk"], "rows_per_s": bx.T / (r["topk"] * 1e-3)}, "clocks": clk}
+    elif args.workload == "latent":
+        bx = LatentBench(dev)
+        clocks.start()
+        r = bx.run(args.steps, args.warmup)
+        clk = clocks.stop()
+        per_layer_bytes = bx.B * bx.L * (512 + 4)
+        achieved = per_layer_bytes / (r["score"] * 1e-3) / 1e9
+        out = {"metric": METRIC, "value": 4 * bx.B * bx.L / (r["step"] * 1e-3), "unit": "keys/s",
+               "ms_per_step": r["step"], "us_per_layer": r["step"] * 1e3 / 4, "higher_is_better": True,
+               "dtype": "bf16", "config": {"workload": "latent_g4_b4_l64k", "B": bx.B, "L": bx.L, "G": 4,
+                                           "d_c": 256, "k": KTOP, "l2": f"{len(bx.c)} rotating cache copies"},
+               "roofline": {"bound": "hbm", "kernel": "stream_score_kernel<bf16>", "achieved": achieved,
+                            "peak": hbm, "peak_source": which, "unit": "GB/s", "frac": achieved / hbm,
+                            "kernel_us": r["score"] * 1e3}, "clocks": clk}
+    else:
+        Bx = 1 if args.workload == "hs_b1" else 16
+        bx = HsBench(dev, Bx)
+        clocks.start()
+        r = bx.run(args.steps, args.warmup)
+        clk = clocks.stop()
+        algo = bx.B * bx.L * (512 + 8) + bx.B * bx.C * (512 + 4 + 3 * 8)
+        out = {"metric": METRIC, "value": bx.B * bx.L / (r["step"] * 1e-3), "unit": "keys/s (anchor scan)",
+               "ms_per_step": r["step"], "us_per_step": r["step"] * 1e3, "higher_is_better": True,
+               "dtype": "bf16", "config": {"workload": f"latent_hs_b{Bx}_l128k", "B": Bx, "L": bx.L, "C": bx.C,
+                                           "followers": 3, "k": KTOP, "l2": f"{len(bx.c)} rotating cache copies"},
+               "roofline": {"bound": "hbm", "kernel": "whole HS step", "achieved": algo / (r["step"] * 1e-3) / 1e9,
+                            "peak": hbm, "peak_source": which, "unit": "GB/s",
+                            "frac": algo / (r["step"] * 1e-3) / 1e9 / hbm}, "clocks": clk}
+    assert api.li_get_last_error() == 0
+    out.update({"n_gpus": world, "steps": args.steps, "warmup": args.warmup, "scaling": "weak", "vs_baseline": None,
+                "data": "synthetic"})
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -397,6 +617,9 @@ def main():
     ap.add_argument("--impl", default="li", choices=["li", "reference"])
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "latent", "hs_b1", "hs_b16"],
+                    help="decode (default) is the benchmarked configuration; the others time the other "
+                         "configurations of the parity tests")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -405,7 +628,10 @@ def main():
     if args.impl == "reference":
         run_reference(args, rank)
         return
-    run_li(args, rank, world, local_rank)
+    if args.workload == "decode":
+        run_li(args, rank, world, local_rank)
+    else:
+        run_other(args, rank, world, local_rank)
 
 
 if __name__ == "__main__":

@@ -179,12 +179,24 @@ __global__ void __launch_bounds__(HS_THREADS, 1) hs_rescore_kernel(const HsArgs 
         // ------------------------------------------------------------ follower queries
         const int et = threadIdx.x - 160;  // 0..127
         constexpr int CH = HS_KBLK * 8;    // 16-byte chunks per query row
-        for (int ci = et; ci < C::N * CH; ci += 128) {
-            const int r = ci / CH, cc = ci % CH;  // r = f * 64 + j
-            const int f = r / HS_H, j = r % HS_H;
-            const uint4 v = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.qt) +
-                                                                 (((size_t)f * a.B + b) * HS_H + j) * HS_DC) + cc);
-            *reinterpret_cast<uint4*>(qsm + (cc >> 3) * (C::N * 128) + sw128_offset(r, cc & 7)) = v;
+        constexpr int PER = C::N * CH / 128;  // 16 chunks per thread per follower
+#pragma unroll 1
+        for (int g0 = 0; g0 < PER; g0 += 8) {  // loads of a batch are all in flight together
+            uint4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int ci = et + 128 * (g0 + u);
+                const int r = ci / CH, cc = ci % CH;  // r = f * 64 + j
+                const int f = r / HS_H, j = r % HS_H;
+                v[u] = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.qt) +
+                                                            (((size_t)f * a.B + b) * HS_H + j) * HS_DC) + cc);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int ci = et + 128 * (g0 + u);
+                const int r = ci / CH, cc = ci % CH;
+                *reinterpret_cast<uint4*>(qsm + (cc >> 3) * (C::N * 128) + sw128_offset(r, cc & 7)) = v[u];
+            }
         }
         for (int r = et; r < C::N; r += 128) {
             const int f = r / HS_H, j = r % HS_H;

@@ -161,24 +161,44 @@ __global__ void __launch_bounds__(192) stream_score_kernel(const __grid_constant
         const int et = threadIdx.x - 64;  // 0..127
         const int ew = et >> 5;
         if constexpr (FP8) {
+            // 16 heads per warp; all loads are issued before any is consumed
+            constexpr int HPW = C::H / 4;
             const __nv_bfloat16* q = reinterpret_cast<const __nv_bfloat16*>(a.q) + (size_t)b * C::H * 128;
-            for (int j = ew; j < C::H; j += 4) {
-                const uint2 raw = __ldg(reinterpret_cast<const uint2*>(q + (size_t)j * 128) + lane);
+            uint2 raw[HPW];
+            float wv[HPW];
+#pragma unroll
+            for (int i = 0; i < HPW; ++i) {
+                const int j = ew + 4 * i;
+                raw[i] = __ldg(reinterpret_cast<const uint2*>(q + (size_t)j * 128) + lane);
+                wv[i] = __ldg(a.w + (size_t)b * C::H + j);
+            }
+#pragma unroll
+            for (int i = 0; i < HPW; ++i) {
+                const int j = ew + 4 * i;
                 float sq;
-                const uint32_t packed = quantize_head128(raw, &sq);
+                const uint32_t packed = quantize_head128(raw[i], &sq);
                 *reinterpret_cast<uint32_t*>(qsm + sw128_offset(j, lane >> 2) + (lane & 3) * 4) = packed;
-                if (lane == 0) wsm[j] = __ldg(a.w + (size_t)b * C::H + j) * sq;
+                if (lane == 0) wsm[j] = wv[i] * sq;
             }
         } else {
-            constexpr int CH = KBLK * 8;  // 16-byte chunks per query row
+            constexpr int CH = KBLK * 8;                // 16-byte chunks per query row
+            constexpr int PER = C::H * CH / 128;        // chunks per thread
+            static_assert(PER % 8 == 0, "query copy batches");
             const uint4* src =
                 reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.q) + (size_t)b * C::H * KBLK * 64);
-            for (int ci = et; ci < C::H * CH; ci += 128) {
-                const int r = ci / CH, cc = ci % CH;
-                const uint4 v = __ldg(src + ci);
-                *reinterpret_cast<uint4*>(qsm + (cc >> 3) * (C::H * 128) + sw128_offset(r, cc & 7)) = v;
+#pragma unroll
+            for (int g0 = 0; g0 < PER; g0 += 8) {
+                uint4 v[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) v[u] = __ldg(src + et + 128 * (g0 + u));
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int ci = et + 128 * (g0 + u);
+                    const int r = ci / CH, cc = ci % CH;
+                    *reinterpret_cast<uint4*>(qsm + (cc >> 3) * (C::H * 128) + sw128_offset(r, cc & 7)) = v[u];
+                }
             }
-            for (int j = et; j < C::H; j += 128) wsm[j] = __ldg(a.w + (size_t)b * C::H + j);
+            if (et < C::H) wsm[et] = __ldg(a.w + (size_t)b * C::H + et);
         }
         fence_proxy_async_smem();
         mbar_arrive(qready);
