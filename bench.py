@@ -111,13 +111,19 @@ def traffic_for(kernel: str, units: float):
         return None
     try:
         d = json.load(open(p)).get(kernel)
-        src = os.path.join(ROOT, d["source"])
-        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-        if h != d["source_sha256_16"]:
+        if sources_sha256_16(d["sources"]) != d["sources_sha256_16"]:
             return None
         return d["dram_bytes_per_unit"] * units
     except Exception:
         return None
+
+
+def sources_sha256_16(paths):
+    """Hash of the kernel's source files (repo-relative), to detect stale counters."""
+    h = hashlib.sha256()
+    for rel in paths:
+        h.update(open(os.path.join(ROOT, rel), "rb").read())
+    return h.hexdigest()[:16]
 
 
 # ---------------------------------------------------------------------------
@@ -307,34 +313,34 @@ def run_li(args, rank, world, local_rank):
     ms, score_ms, topk_ms, direct_ms = li_dist.max_over_ranks([ms, score_ms, topk_ms, direct_ms], device=dev)
     launches = 2 * args.steps
 
-    # ---- end to end through the public API: pinned host q/w in, indices out,
-    # direct calls (no graph), as a user would make them
-    q, w, sc, idx = bench.q, bench.w, bench.sc, bench.idx
-    qh = bench.case.q.pin_memory()
-    wh = bench.case.w.pin_memory()
-    idx_h = torch.empty((B, KTOP), dtype=torch.int32).pin_memory()
-
-    def e2e_step(i):
-        kk, ss = bench.sets[i % bench.n]
-        q.copy_(qh, non_blocking=True)
-        w.copy_(wh, non_blocking=True)
-        api.li_index_score(q, w, kk, ss, scores=sc)
-        api.li_topk(sc, KTOP, idx=idx)
-        idx_h.copy_(idx, non_blocking=True)
-
+    # ---- end to end through the public API: each step copies the pinned host
+    # query/weights in, scores + selects, and copies the indices out, as one
+    # graph-captured DecodeIndexer step (one indexer per rotating cache copy)
+    from sparse_attention_lightning_score_b200.step import DecodeIndexer
+    indexers = [DecodeIndexer(kk, ss, H, KTOP) for kk, ss in bench.sets]
+    for ix in indexers:
+        ix.q_host.copy_(bench.case.q)
+        ix.w_host.copy_(bench.case.w)
     for i in range(args.warmup):
-        e2e_step(i)
+        indexers[i % len(indexers)].step(sync=False)
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
     a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a0.record()
     for i in range(args.steps):
-        e2e_step(i)
+        indexers[i % len(indexers)].step(sync=False)
     a1.record()
     torch.cuda.synchronize()
     e2e_ms = a0.elapsed_time(a1) / args.steps
     (e2e_ms,) = li_dist.max_over_ranks([e2e_ms], device=dev)
+    # the selections that came back to the host match the device-side graph's
+    ref_idx = bench.idx.clone()
+    bench.step_graphs[(args.steps - 1) % bench.n].replay()
+    torch.cuda.synchronize()
+    assert torch.equal(indexers[(args.steps - 1) % len(indexers)].idx_host, bench.idx.cpu())
+    h2d, d2h = indexers[0].h2d_bytes, indexers[0].d2h_bytes
+    del indexers, ref_idx
     assert api.li_get_last_error() == 0
 
     sweep = None
@@ -377,8 +383,8 @@ def run_li(args, rank, world, local_rank):
         "topk": {"us": topk_ms * 1e3, "rows_per_s": B / (topk_ms * 1e-3), "row_len": L, "k": KTOP},
         "direct_us_per_step": direct_ms * 1e3,
         "e2e": {"value": world * B * L / (e2e_ms * 1e-3), "unit": "keys/s",
-                "h2d_bytes_per_step": B * H * D * 2 + B * H * 4, "d2h_bytes_per_step": B * KTOP * 4,
-                "ms_per_step": e2e_ms},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "api": "DecodeIndexer.step (graph: H2D q,w -> score -> top-k -> D2H indices)"},
         "gpu_launches": launches,
         "clocks": clk,
     }

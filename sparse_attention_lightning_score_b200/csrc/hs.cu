@@ -27,7 +27,6 @@ constexpr int HS_DC = 256;
 constexpr int HS_KBLK = 4;
 constexpr int HS_STAGES = 6;
 constexpr int HS_STAGE_BYTES = HS_M * 128;
-constexpr int HS_FMAX = 4;
 constexpr int HS_DEPTH = 3;  // cp.async groups in flight per producer thread
 constexpr int HS_THREADS = 288;
 

@@ -10,6 +10,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "li.h"
 
 namespace li {
@@ -32,6 +34,32 @@ li_status host_check_launch();      // maps cudaGetLastError() to li_status
 int host_num_sms();
 
 constexpr unsigned long long kDefaultWaitLimitNs = 2000000000ull; // 2 s
+
+// Launch with programmatic stream serialisation (and an optional cluster shape).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, int cluster_x,
+                       Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+    if (cluster_x > 1) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = cluster_x;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 #if defined(__CUDACC__)
 
@@ -94,6 +122,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
         }
     }
 }
+
+// Programmatic dependent launch.  A kernel launched with the programmatic
+// stream-serialisation attribute may start while the previous kernel of the
+// stream is still running; pdl_wait() blocks the calling thread until that
+// kernel has completed and its memory is visible (a no-op without the
+// attribute).  pdl_trigger() lets the next kernel of the stream be scheduled.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // Make generic-proxy writes to shared memory visible to the async proxy
 // (TMA, tcgen05.mma operand reads).
@@ -239,6 +275,31 @@ __device__ __forceinline__ float relu_dot32(const uint32_t (&v)[32], const float
     return (a0 + a1) + (a2 + a3);
 }
 
+// acc.{x,y} += a.{0,1} * b.{0,1} with one packed fp32x2 FMA (same rounding as two fmaf).
+__device__ __forceinline__ void ffma2(float2& acc, float a0, float a1, float b0, float b1) {
+    asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %5};\n\t"
+        "mov.b64 rc, {%0, %1};\n\t"
+        "fma.rn.f32x2 rc, ra, rb, rc;\n\t"
+        "mov.b64 {%0, %1}, rc;\n\t}"
+        : "+f"(acc.x), "+f"(acc.y)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// Weighted ReLU reduction over 32 head values with packed FMAs:
+// sum_j wj * max(v_j, 0), 1.5 instructions per value (FMNMX + half an FFMA2).
+__device__ __forceinline__ float relu_dot32_x2(const uint32_t (&v)[32], const float* __restrict__ wsm) {
+    float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) {
+        const float4 w4 = *reinterpret_cast<const float4*>(wsm + j);
+        ffma2(a0, fmaxf(__uint_as_float(v[j + 0]), 0.f), fmaxf(__uint_as_float(v[j + 1]), 0.f), w4.x, w4.y);
+        ffma2(a1, fmaxf(__uint_as_float(v[j + 2]), 0.f), fmaxf(__uint_as_float(v[j + 3]), 0.f), w4.z, w4.w);
+    }
+    return (a0.x + a0.y) + (a1.x + a1.y);
+}
+
 // Per-(row, head) e4m3 quantisation of one 128-element bf16 head vector held
 // as 4 consecutive elements per lane of a warp.  Returns the packed 4 bytes
 // of this lane and writes the head scale to *sq (all lanes).
@@ -256,6 +317,37 @@ __device__ __forceinline__ uint32_t quantize_head128(uint2 raw, float* sq_out) {
     const uint32_t b2 = __nv_cvt_float_to_fp8(__fdiv_rn(x2, sq), __NV_SATFINITE, __NV_E4M3);
     const uint32_t b3 = __nv_cvt_float_to_fp8(__fdiv_rn(x3, sq), __NV_SATFINITE, __NV_E4M3);
     return b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+}
+
+// Same quantisation with 8 lanes per head: the lane holds 16 consecutive bf16
+// elements (16*l8 .. 16*l8+15 of the head, `lo` then `hi`) and returns their 16
+// e4m3 bytes; *sq_out receives the head scale.  All 32 lanes of the warp must
+// call it (the absmax reduction shuffles within aligned groups of 8 lanes).
+__device__ __forceinline__ uint4 quantize_head128_g8(uint4 lo, uint4 hi, float* sq_out) {
+    float x[16];
+    const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        x[2 * i] = __uint_as_float(w[i] << 16);
+        x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+    float m = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(x[i]));
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float sq = m > 0.f ? __fdiv_rn(m, 448.f) : 1.f;
+    *sq_out = sq;
+    uint32_t b[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t b0 = __nv_cvt_float_to_fp8(__fdiv_rn(x[4 * i + 0], sq), __NV_SATFINITE, __NV_E4M3);
+        const uint32_t b1 = __nv_cvt_float_to_fp8(__fdiv_rn(x[4 * i + 1], sq), __NV_SATFINITE, __NV_E4M3);
+        const uint32_t b2 = __nv_cvt_float_to_fp8(__fdiv_rn(x[4 * i + 2], sq), __NV_SATFINITE, __NV_E4M3);
+        const uint32_t b3 = __nv_cvt_float_to_fp8(__fdiv_rn(x[4 * i + 3], sq), __NV_SATFINITE, __NV_E4M3);
+        b[i] = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+    }
+    return make_uint4(b[0], b[1], b[2], b[3]);
 }
 
 #endif  // __CUDACC__

@@ -15,8 +15,11 @@
 // (32 KB e4m3) stays in shared memory while its key tiles stream past it
 // through a ring of TMA stages; keys of the shared cache are re-read from L2.
 //
-// Warps: 0 TMA producer, 1 TMEM allocator + MMA issuer, 2..9 epilogue (two
-// warps per TMEM lane quarter, each handling two of the four tokens).
+// Warps: 0 TMA producer, 1 TMEM allocator + MMA issuer, 2..17 epilogue (four
+// warps per TMEM lane quarter, one per token).  The epilogue is exact fp32:
+// ReLU as FMNMX and the head-weighted sum as packed fp32x2 FMAs, 1.5
+// instructions per logit; sixteen warps keep enough of them in flight to
+// overlap the next tile's MMA.
 #include "li_common.cuh"
 #include "li_kernels.cuh"
 
@@ -37,8 +40,8 @@ constexpr int PF_OFF_BAR = PF_OFF_W + 2 * PF_N * 4;
 constexpr int PF_NBAR = 2 * PF_STAGES + 2 + 2 + 2 + 2;
 constexpr int PF_OFF_TMEM = PF_OFF_BAR + PF_NBAR * 8;
 constexpr int PF_SMEM = PF_OFF_TMEM + 16 + 1024;
-constexpr int PF_THREADS = 320;
-constexpr int PF_EPI_THREADS = 256;
+constexpr int PF_THREADS = 576;
+constexpr int PF_EPI_THREADS = 512;
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -160,9 +163,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_score_kernel(const __gr
             }
         }
     } else {
-        const int e = warp - 2;         // 0..7
+        const int e = warp - 2;         // 0..15
         const int g = warp & 3;         // TMEM lane quarter
-        const int u0 = (e >> 2) * 2;    // first of this warp's two tokens
+        const int u = e >> 2;           // this warp's token within the block
         const int et = threadIdx.x - 64;
         uint32_t tc = 0;
         bool ok = true;
@@ -171,11 +174,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_score_kernel(const __gr
             if (qb < 0) break;
             const int t0 = qb * PF_NT;
             float* wb = wbuf + (bi & 1) * PF_N;
-            {
+            if (et < PF_N) {
                 const int t = t0 + et / PF_H;
                 wb[et] = t < a.T ? __ldg(a.w_eff + (size_t)t0 * PF_H + et) : 0.f;
             }
-            asm volatile("bar.sync 1, 256;" ::: "memory");
+            asm volatile("bar.sync 1, 512;" ::: "memory");
             const int nt = pf_ntiles(qb, a);
             for (int kt = 0; kt < nt; ++kt, ++tc) {
                 const uint32_t acc = tc & 1u;
@@ -183,20 +186,16 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_score_kernel(const __gr
                 const float sk = s < a.L ? __ldg(a.kscale + s) : 0.f;
                 if (!mbar_wait(&accf[acc], (tc >> 1) & 1u, a.err)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t tb = tmem_base + ((uint32_t)(g * 32) << 16) + acc * PF_N + u0 * PF_H;
-                uint32_t v0[32], v1[32], v2[32], v3[32];
+                const uint32_t tb = tmem_base + ((uint32_t)(g * 32) << 16) + acc * PF_N + u * PF_H;
+                uint32_t v0[32], v1[32];
                 tmem_ld32(tb, v0);
                 tmem_ld32(tb + 32, v1);
-                tmem_ld32(tb + 64, v2);
-                tmem_ld32(tb + 96, v3);
                 tmem_ld_wait();
                 tc_fence_before();
                 mbar_arrive(&acce[acc]);
-                const float s0 = relu_dot32(v0, wb + u0 * PF_H) + relu_dot32(v1, wb + u0 * PF_H + 32);
-                const float s1 = relu_dot32(v2, wb + (u0 + 1) * PF_H) + relu_dot32(v3, wb + (u0 + 1) * PF_H + 32);
-                const int ta = t0 + u0, tb2 = t0 + u0 + 1;
-                if (ta < a.T && s <= ta + a.causal_offset && s < a.L) a.scores[(size_t)ta * a.scores_ld + s] = s0 * sk;
-                if (tb2 < a.T && s <= tb2 + a.causal_offset && s < a.L) a.scores[(size_t)tb2 * a.scores_ld + s] = s1 * sk;
+                const float sum = relu_dot32_x2(v0, wb + u * PF_H) + relu_dot32_x2(v1, wb + u * PF_H + 32);
+                const int t = t0 + u;
+                if (t < a.T && s <= t + a.causal_offset && s < a.L) a.scores[(size_t)t * a.scores_ld + s] = sum * sk;
             }
         }
     }

@@ -44,7 +44,9 @@ struct StreamCfg {
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_TMEM + 16 + 1024;  // + slack to align the base to 1024
     static constexpr int TMEM_COLS = NACC * H;
-    static constexpr int THREADS = 192;
+    // FP8: warps 6..9 only help quantise the query in the prologue
+    static constexpr int PRO_WARPS = FP8 ? 8 : 4;
+    static constexpr int THREADS = 64 + 32 * PRO_WARPS;
     static constexpr int ELEMS_PER_KBLOCK = FP8 ? 128 : 64;
     static_assert(TMEM_COLS == 128 || TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM columns");
 };
@@ -54,7 +56,7 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 }
 
 template <bool FP8, int KBLK, int STAGES, int NACC>
-__global__ void __launch_bounds__(192) stream_score_kernel(const __grid_constant__ CUtensorMap kmap,
+__global__ void __launch_bounds__(StreamCfg<FP8, KBLK, STAGES, NACC>::THREADS, 2) stream_score_kernel(const __grid_constant__ CUtensorMap kmap,
                                                            const StreamArgs a) {
     using C = StreamCfg<FP8, KBLK, STAGES, NACC>;
     extern __shared__ uint8_t smem_raw[];
@@ -62,15 +64,8 @@ __global__ void __launch_bounds__(192) stream_score_kernel(const __grid_constant
 
     const int b = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    int len_b = a.len ? __ldg(a.len + b) : a.max_len;
-    if (len_b < 0 || len_b > a.max_len) {
-        if (threadIdx.x == 0 && blockIdx.x == 0) record_error(a.err, ERRBIT_BOUNDS);
-        len_b = len_b < 0 ? 0 : a.max_len;
-    }
-    const int ntiles = (len_b + C::M - 1) / C::M;
-    const int t0 = blockIdx.x * a.tiles_per_cta;
-    const int nt = min(t0 + a.tiles_per_cta, ntiles) - t0;
-    if (nt <= 0) return;  // uniform over the CTA
+    pdl_trigger();  // the next kernel of the stream may be scheduled; it waits for this one itself
+    if (blockIdx.x * a.tiles_per_cta >= (a.max_len + C::M - 1) / C::M) return;  // no tile for any length
 
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* empty = full + STAGES;
@@ -90,7 +85,7 @@ __global__ void __launch_bounds__(192) stream_score_kernel(const __grid_constant
             mbar_init(&accf[i], 1);
             mbar_init(&acce[i], 128);
         }
-        mbar_init(qready, 128);
+        mbar_init(qready, 32 * C::PRO_WARPS);
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -101,6 +96,18 @@ __global__ void __launch_bounds__(192) stream_score_kernel(const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+
+    // everything above overlaps the previous kernel; inputs are read only after it completed
+    pdl_wait();
+    int len_b = a.len ? __ldg(a.len + b) : a.max_len;
+    if (len_b < 0 || len_b > a.max_len) {
+        if (threadIdx.x == 0 && blockIdx.x == 0) record_error(a.err, ERRBIT_BOUNDS);
+        len_b = len_b < 0 ? 0 : a.max_len;
+    }
+    const int ntiles = (len_b + C::M - 1) / C::M;
+    const int t0 = blockIdx.x * a.tiles_per_cta;
+    const int nt = min(t0 + a.tiles_per_cta, ntiles) - t0;
+    if (nt <= 0) goto done;  // uniform over the CTA
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -158,27 +165,32 @@ __global__ void __launch_bounds__(192) stream_score_kernel(const __grid_constant
         }
     } else {
         // ------------------------------------------------------------ query prep
-        const int et = threadIdx.x - 64;  // 0..127
+        const int et = threadIdx.x - 64;  // 0 .. 32*PRO_WARPS-1
         const int ew = et >> 5;
         if constexpr (FP8) {
-            // 16 heads per warp; all loads are issued before any is consumed
-            constexpr int HPW = C::H / 4;
+            // 8 heads per warp, four at a time (8 lanes per head, 16 elements per
+            // lane); all loads are issued before any is consumed
+            constexpr int HPW = C::H / C::PRO_WARPS;
+            constexpr int IT = HPW / 4;
+            const int g8 = lane >> 3, l8 = lane & 7;
             const __nv_bfloat16* q = reinterpret_cast<const __nv_bfloat16*>(a.q) + (size_t)b * C::H * 128;
-            uint2 raw[HPW];
-            float wv[HPW];
+            uint4 raw[IT][2];
+            float wv[IT];
 #pragma unroll
-            for (int i = 0; i < HPW; ++i) {
-                const int j = ew + 4 * i;
-                raw[i] = __ldg(reinterpret_cast<const uint2*>(q + (size_t)j * 128) + lane);
+            for (int i = 0; i < IT; ++i) {
+                const int j = HPW * ew + 4 * i + g8;
+                const uint4* src = reinterpret_cast<const uint4*>(q + (size_t)j * 128) + 2 * l8;
+                raw[i][0] = __ldg(src);
+                raw[i][1] = __ldg(src + 1);
                 wv[i] = __ldg(a.w + (size_t)b * C::H + j);
             }
 #pragma unroll
-            for (int i = 0; i < HPW; ++i) {
-                const int j = ew + 4 * i;
+            for (int i = 0; i < IT; ++i) {
+                const int j = HPW * ew + 4 * i + g8;
                 float sq;
-                const uint32_t packed = quantize_head128(raw[i], &sq);
-                *reinterpret_cast<uint32_t*>(qsm + sw128_offset(j, lane >> 2) + (lane & 3) * 4) = packed;
-                if (lane == 0) wsm[j] = wv[i] * sq;
+                const uint4 packed = quantize_head128_g8(raw[i][0], raw[i][1], &sq);
+                *reinterpret_cast<uint4*>(qsm + sw128_offset(j, l8)) = packed;
+                if (l8 == 0) wsm[j] = wv[i] * sq;
             }
         } else {
             constexpr int CH = KBLK * 8;                // 16-byte chunks per query row
@@ -202,7 +214,9 @@ __global__ void __launch_bounds__(192) stream_score_kernel(const __grid_constant
         }
         fence_proxy_async_smem();
         mbar_arrive(qready);
-        asm volatile("bar.sync 1, 128;" ::: "memory");  // w_eff visible to every epilogue thread
+        // w_eff visible to every epilogue thread
+        asm volatile("bar.sync 1, %0;" ::"n"(32 * C::PRO_WARPS) : "memory");
+        if (warp >= 6) goto done;  // prologue helpers: nothing more to do
 
         // ------------------------------------------------------------ epilogue
         const int g = warp & 3;  // TMEM lane quarter this warp may access
@@ -227,6 +241,7 @@ __global__ void __launch_bounds__(192) stream_score_kernel(const __grid_constant
             if (s < len_b) out[s] = FP8 ? sum * sk : sum;
         }
     }
+done:
     __syncwarp();
     __syncthreads();
     if (warp == 1) {
@@ -256,7 +271,7 @@ li_status launch_impl(const CUtensorMap& map, const StreamArgs& args, int batch,
     StreamArgs a = args;
     a.tiles_per_cta = tpc;
     dim3 grid(max(cpr, 1), batch);
-    kern<<<grid, C::THREADS, C::SMEM, st>>>(map, a);
+    if (launch_pdl(kern, grid, dim3(C::THREADS), C::SMEM, st, 1, map, a) != cudaSuccess) return host_check_launch();
     return host_check_launch();
 }
 

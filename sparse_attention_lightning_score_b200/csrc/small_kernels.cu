@@ -18,14 +18,32 @@ __global__ void __launch_bounds__(256) quantize_query_kernel(const __nv_bfloat16
                                                              float* __restrict__ w_eff) {
     const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
+    if (dim == 128) {  // four heads per warp, 8 lanes per head
+        const long long head = gw * 4 + (lane >> 3);
+        if (gw * 4 >= nheads) return;  // whole warp
+        const bool live = head < nheads;
+        const int l8 = lane & 7;
+        uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
+        if (live) {
+            const uint4* src = reinterpret_cast<const uint4*>(q + head * 128) + 2 * l8;
+            lo = __ldg(src);
+            hi = __ldg(src + 1);
+        }
+        float s;
+        const uint4 packed = quantize_head128_g8(lo, hi, &s);  // all lanes take part in the shuffles
+        if (live) {
+            reinterpret_cast<uint4*>(q8 + head * 128)[l8] = packed;
+            if (l8 == 0) {
+                sq[head] = s;
+                if (w_eff) w_eff[head] = w[head] * s;
+            }
+        }
+        return;
+    }
     if (gw >= nheads) return;  // whole warp
     const __nv_bfloat16* src = q + gw * dim;
     float s;
-    if (dim == 128) {
-        const uint2 raw = __ldg(reinterpret_cast<const uint2*>(src) + lane);
-        const uint32_t packed = quantize_head128(raw, &s);
-        reinterpret_cast<uint32_t*>(q8 + gw * 128)[lane] = packed;
-    } else {
+    {
         float m = 0.f;
         for (int e = lane; e < dim; e += 32) m = fmaxf(m, fabsf(__bfloat162float(src[e])));
 #pragma unroll
@@ -143,7 +161,8 @@ li_status launch_quantize_query(const void* q, const float* w, int rows, int hea
                                 float* w_eff, cudaStream_t st) {
     const long long nh = (long long)rows * heads;
     if (nh == 0) return LI_OK;
-    const long long blocks = (nh * 32 + 255) / 256;
+    const long long warps = dim == 128 ? (nh + 3) / 4 : nh;
+    const long long blocks = (warps * 32 + 255) / 256;
     quantize_query_kernel<<<(unsigned)blocks, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(q), w, nh, dim, q8,
                                                             sq, w_eff);
     return host_check_launch();

@@ -5,17 +5,32 @@
 // below every number; -0.0 equals +0.0.  The selected positions are written in
 // ascending order (then -1 pads when a row holds fewer than k scores).
 //
-// Method: MSB-first radix select (8-bit digits) on an order-preserving
-// uint32 image of the fp32 bits, as in Alabi et al., "Fast k-Selection
-// Algorithms for Graphics Processing Units" (2012).  A row is split over a
-// thread-block cluster of CS CTAs; each CTA keeps its slice of the row in
-// shared memory, so HBM is read once.  Per digit, each CTA builds a 256-bin
-// histogram of the still-undecided keys with warp-aggregated shared-memory
-// atomics (__match_any_sync groups lanes holding the same digit, one atomic
-// per group), the histograms are summed across the cluster through
-// distributed shared memory, and every CTA takes the same decision.  The
-// final compaction is an ordered scan (CTA prefix over the cluster, block
-// prefix inside the CTA), so the output does not depend on atomic order.
+// Method: MSB-first radix select on an order-preserving uint32 image of the
+// fp32 bits, as in Alabi et al., "Fast k-Selection Algorithms for Graphics
+// Processing Units" (2012).  A pass stops the select early when the bin that
+// holds the k-th key is taken whole (no tie to break), which for real scores
+// happens after 22-24 bits.
+//
+// Each CTA keeps its slice of the row in shared memory, so the scores are read
+// from HBM (or L2) once.  Many rows (causal prefill): one CTA per row, 11-bit
+// digits (three passes at most), every pass a shared-memory histogram plus
+// block barriers.  Few rows (decode): each row is split over a thread-block
+// cluster so that about 4K keys land on each CTA and every sweep runs on many
+// SMs; the CTAs' histograms are summed through distributed shared memory after
+// one cluster barrier per pass, with 8-bit digits so that a merge moves 256
+// bins (measured: merging 2048-bin histograms cost more than the extra pass).
+//
+// Histograms: warp w adds into private copy w % NCOPY with plain shared-memory
+// atomics, which spreads the few hot bins a pass of real scores concentrates
+// on (aggregating lanes by digit with __match_any_sync was measured 6x slower
+// on B200); a warp ballot skips warps with no undecided key.  Each owner
+// thread folds the copies of its bins, merges them over the cluster and feeds
+// a block-wide scan (warp shuffles) that finds the digit of the k-th key.
+//
+// Compaction: the slice's counts above / at the threshold are exchanged over
+// the cluster once, then the slice is written in order, 4 keys per thread per
+// tile, positions from a block-wide scan.  No output depends on the order of
+// any atomic operation.
 #include <cooperative_groups.h>
 
 #include "li_common.cuh"
@@ -27,11 +42,9 @@ namespace li {
 
 namespace {
 
-constexpr int TK_THREADS = 512;
-constexpr int TK_WARPS = TK_THREADS / 32;
-constexpr int TK_IPT = 4;                     // keys per thread per compaction tile
-constexpr int TK_TILE = TK_THREADS * TK_IPT;  // 2048
-constexpr int TK_MAX_SMEM = 160 * 1024;       // key slice budget per CTA
+constexpr int TK_SMEM_ROW = 40960;  // longest slice held by one CTA (160 KB of keys)
+constexpr int TK_MAX_CS = 8;        // largest cluster
+constexpr int TK_SLICE = 4096;      // target slice of a row per cluster CTA
 
 __device__ __forceinline__ uint32_t order_key(float f) {
     if (f != f) return 0u;  // NaN: the only key mapped to 0, below -inf (0x007FFFFF)
@@ -40,31 +53,32 @@ __device__ __forceinline__ uint32_t order_key(float f) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Inclusive prefix sum over the 512 threads of the block; *total receives the
-// block sum.  Contains __syncthreads; call from all threads.
-__device__ __forceinline__ uint32_t block_incl_scan(uint32_t v, uint32_t* wsum, uint32_t* total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+__device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v, int lane) {
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const uint32_t t = __shfl_up_sync(0xffffffffu, v, o);
         if (lane >= o) v += t;
     }
-    if (lane == 31) wsum[warp] = v;
+    return v;
+}
+
+// Block-wide inclusive scan with one __syncthreads.  wsum must not be reused
+// before every thread has passed the next block-wide barrier.
+template <int NW>
+__device__ __forceinline__ uint32_t block_scan1(uint32_t v, uint32_t* wsum, uint32_t* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t incl = warp_incl_scan(v, lane);
+    if (lane == 31) wsum[warp] = incl;
     __syncthreads();
-    if (warp == 0) {
-        uint32_t x = lane < TK_WARPS ? wsum[lane] : 0u;
+    uint32_t off = 0u, tot = 0u;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t t = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += t;
-        }
-        if (lane < TK_WARPS) wsum[lane] = x;
+    for (int w = 0; w < NW; ++w) {
+        const uint32_t x = wsum[w];
+        off += w < warp ? x : 0u;
+        tot += x;
     }
-    __syncthreads();
-    const uint32_t add = warp > 0 ? wsum[warp - 1] : 0u;
-    *total = wsum[TK_WARPS - 1];
-    __syncthreads();
-    return v + add;
+    *total = tot;
+    return incl + off;
 }
 
 template <bool CLUSTER>
@@ -79,16 +93,48 @@ __device__ __forceinline__ const uint32_t* cl_peer(uint32_t* p, int rank) {
     else return p;
 }
 
-template <bool CLUSTER>
-__global__ void __launch_bounds__(TK_THREADS) topk_kernel(const TopkArgs a, int row0, int chunk) {
+// Kernel shape: NT threads, DBITS-bit digits (11 for a row held by one CTA:
+// three passes, no merge; 8 for a row split over a cluster: up to four
+// passes, but each cluster merge moves 256 bins instead of 2048).
+template <int NT, bool CLUSTER>
+struct TopkShape {
+    static constexpr int WARPS = NT / 32;
+    static constexpr int DBITS = CLUSTER ? 8 : 11;
+    static constexpr int BINS = 1 << DBITS;
+    static constexpr int PASSES = (32 + DBITS - 1) / DBITS;
+    static constexpr int OWNERS = BINS < NT ? BINS : NT;  // threads that own bins
+    static constexpr int BPT = BINS / OWNERS;              // bins per owner
+    static constexpr int NCOPY = CLUSTER ? 8 : (NT >= 1024 ? 4 : 2);  // private histogram copies
+    static constexpr int TILE = NT * 4;                    // compaction tile (4 keys per thread)
+    // dynamic shared memory: keys, NCOPY histogram copies, then (cluster) the
+    // double-buffered merged histogram the peers read
+    static size_t smem(int chunk) {
+        return (size_t)((chunk + 3) & ~3) * 4 + (size_t)NCOPY * BINS * 4 + (CLUSTER ? 2 * BINS * 4 : 0);
+    }
+    __device__ static int shift(int p) { return 32 - DBITS * (p + 1) > 0 ? 32 - DBITS * (p + 1) : 0; }
+    __device__ static uint32_t digits(int p) {
+        const int lo = shift(p), hi = 32 - DBITS * p;  // bits [lo, hi)
+        return (hi - lo >= 32) ? 0xffffffffu : ((1u << (hi - lo)) - 1u);
+    }
+};
+
+// Thread t < OWNERS owns the BPT contiguous bins BINS-BPT(t+1) .. BINS-BPT*t-1
+// (descending positions BPT*t .. BPT*t+BPT-1).
+template <int NT, bool CLUSTER>
+__global__ void __launch_bounds__(NT) topk_kernel(const TopkArgs a, int row0, int chunk) {
+    using S = TopkShape<NT, CLUSTER>;
+    constexpr int BPT = S::BPT, NW = S::WARPS, NCOPY = S::NCOPY, BINS = S::BINS;
+    static_assert(BPT == 1 || BPT == 2 || BPT == 4 || BPT == 8, "bins per owner");
     extern __shared__ uint4 tk_dyn[];
     uint32_t* keys = reinterpret_cast<uint32_t*>(tk_dyn);
-    __shared__ uint32_t hist[2][256];
-    __shared__ uint32_t tot[256];
-    __shared__ uint32_t wsum[TK_WARPS];
+    uint32_t* hcopy = keys + ((chunk + 3) & ~3);     // [NCOPY][BINS]
+    uint32_t* pub = hcopy + NCOPY * BINS;            // [2][BINS], cluster only
+    __shared__ uint32_t wsum[2][32];
     __shared__ uint32_t bc[4];
     __shared__ uint32_t xch[2];
 
+    pdl_trigger();
+    pdl_wait();  // the scores come from the previous kernel of the stream
     const int r = row0 + blockIdx.y;
     const int CS = gridDim.x;
     const int c = blockIdx.x;  // == cluster rank: the cluster spans gridDim.x
@@ -107,12 +153,12 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const TopkArgs a, int 
     const int32_t* mrow = a.map ? a.map + (size_t)(r % a.map_rows) * a.map_ld : nullptr;
 
     if (n <= k) {  // every score is selected; the branch is uniform over the cluster
-        for (int i = threadIdx.x; i < cnt; i += TK_THREADS) {
+        for (int i = threadIdx.x; i < cnt; i += NT) {
             const int p = base + i;
             oidx[p] = mrow ? __ldg(mrow + p) : p;
             if (oval) oval[p] = __ldg(srow + p);
         }
-        for (int p = n + c * TK_THREADS + threadIdx.x; p < k; p += CS * TK_THREADS) {
+        for (int p = n + c * NT + threadIdx.x; p < k; p += CS * NT) {
             oidx[p] = -1;
             if (oval) oval[p] = -INFINITY;
         }
@@ -122,93 +168,138 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const TopkArgs a, int 
     // ---- load this CTA's slice (row start and slice start are 16-byte aligned)
     const float4* s4 = reinterpret_cast<const float4*>(srow + base);
     const int nvec = (cnt + 3) >> 2;
-    for (int i = threadIdx.x; i < nvec; i += TK_THREADS) {
+    for (int i = threadIdx.x; i < nvec; i += NT) {
         const float4 v = __ldg(s4 + i);
         tk_dyn[i] = make_uint4(order_key(v.x), order_key(v.y), order_key(v.z), order_key(v.w));
     }
-    for (int i = threadIdx.x; i < 512; i += TK_THREADS) (&hist[0][0])[i] = 0u;
+    for (int i = threadIdx.x; i < NCOPY * BINS; i += NT) hcopy[i] = 0u;
     __syncthreads();
 
     // ---- radix select, most significant digit first
     uint32_t prefix = 0u, mask = 0u;
     int krem = k;
     bool ties = true;
-    const int cnt32 = (cnt + 31) & ~31;
-    for (int pass = 0; pass < 4; ++pass) {
-        const int shift = 24 - 8 * pass;
-        uint32_t* h = hist[pass & 1];
-        for (int i0 = warp * 32; i0 < cnt32; i0 += TK_THREADS) {
-            const int i = i0 + lane;
-            bool act = false;
-            uint32_t dig = 0u;
-            if (i < cnt) {
-                const uint32_t kk = keys[i];
-                act = (kk & mask) == prefix;
-                dig = (kk >> shift) & 255u;
-            }
-            const uint32_t am = __ballot_sync(0xffffffffu, act);
-            if (act) {
-                const uint32_t peers = __match_any_sync(am, dig);
-                if (lane == __ffs(peers) - 1) atomicAdd(&h[dig], (uint32_t)__popc(peers));
-            }
-        }
-        cl_sync<CLUSTER>();
-        if (threadIdx.x < 256) {
-            uint32_t t = 0u;
-            for (int q = 0; q < CS; ++q) t += cl_peer<CLUSTER>(h, q)[threadIdx.x];
-            tot[threadIdx.x] = t;
-            hist[(pass + 1) & 1][threadIdx.x] = 0u;  // read by peers one pass ago: free again
+    const bool owner = threadIdx.x < S::OWNERS;
+    const int b0 = BINS - BPT * (threadIdx.x + 1);  // an owner's bins b0 .. b0+BPT-1
+    uint32_t* hmine = hcopy + (warp % NCOPY) * BINS;
+    for (int pass = 0; pass < S::PASSES; ++pass) {
+        const int shift = S::shift(pass);
+        const uint32_t dm = S::digits(pass);
+        for (int i = threadIdx.x; i < ((cnt + 31) & ~31); i += NT) {
+            const uint32_t kk = i < cnt ? keys[i] : 0u;
+            const bool act = i < cnt && (kk & mask) == prefix;
+            if (__ballot_sync(0xffffffffu, act) == 0u) continue;  // nothing undecided in this warp
+            if (act) atomicAdd(&hmine[(kk >> shift) & dm], 1u);
         }
         __syncthreads();
-        const uint32_t v = threadIdx.x < 256 ? tot[255 - threadIdx.x] : 0u;
+        // fold the private copies of an owner's bins (and clear them for the next pass);
+        // tot[i]: bin b0+BPT-1-i (descending position BPT*t + i) summed over the cluster
+        uint32_t tot[BPT];
+#pragma unroll
+        for (int i = 0; i < BPT; ++i) tot[i] = 0u;
+        if (owner) {
+            uint32_t mine[BPT];
+#pragma unroll
+            for (int v = 0; v < BPT; ++v) mine[v] = 0u;
+#pragma unroll
+            for (int cp = 0; cp < NCOPY; ++cp) {
+#pragma unroll
+                for (int v = 0; v < BPT; ++v) {
+                    mine[v] += hcopy[cp * BINS + b0 + v];
+                    hcopy[cp * BINS + b0 + v] = 0u;
+                }
+            }
+            if constexpr (!CLUSTER) {
+#pragma unroll
+                for (int i = 0; i < BPT; ++i) tot[i] = mine[BPT - 1 - i];
+            } else {
+                uint32_t* pb = pub + (pass & 1) * BINS;  // read by the peers one pass ago: free again
+#pragma unroll
+                for (int v = 0; v < BPT; ++v) pb[b0 + v] = mine[v];
+            }
+        }
+        if constexpr (CLUSTER) {
+            cl_sync<true>();
+            if (owner) {
+                const uint32_t* pb = pub + (pass & 1) * BINS;
+                uint32_t pv[TK_MAX_CS][BPT];
+#pragma unroll
+                for (int q = 0; q < TK_MAX_CS; ++q)
+                    if (q < CS) {
+                        const uint32_t* src = cl_peer<true>(const_cast<uint32_t*>(pb), q) + b0;
+#pragma unroll
+                        for (int v = 0; v < BPT; ++v) pv[q][v] = src[v];
+                    }
+#pragma unroll
+                for (int q = 0; q < TK_MAX_CS; ++q)
+                    if (q < CS) {
+#pragma unroll
+                        for (int i = 0; i < BPT; ++i) tot[i] += pv[q][BPT - 1 - i];
+                    }
+            }
+        }
+        uint32_t s = 0u;
+#pragma unroll
+        for (int i = 0; i < BPT; ++i) s += tot[i];
         uint32_t total;
-        const uint32_t incl = block_incl_scan(v, wsum, &total);
-        if (threadIdx.x < 256 && v > 0u && incl >= (uint32_t)krem && incl - v < (uint32_t)krem) {
-            bc[0] = 255u - threadIdx.x;  // the digit holding the k-th largest key
-            bc[1] = incl - v;            // keys above that digit
-            bc[2] = v;                   // keys in that digit
+        const uint32_t incl = block_scan1<NW>(s, wsum[pass & 1], &total);
+        const uint32_t excl = incl - s;
+        if (owner && excl < (uint32_t)krem && incl >= (uint32_t)krem) {
+            uint32_t run = excl;
+#pragma unroll
+            for (int i = 0; i < BPT; ++i) {
+                if (run < (uint32_t)krem && run + tot[i] >= (uint32_t)krem) {
+                    bc[0] = (uint32_t)(BINS - 1 - (BPT * threadIdx.x + i));  // digit of the k-th key
+                    bc[1] = run;                                             // keys above that digit
+                    bc[2] = tot[i];                                          // keys in that digit
+                }
+                run += tot[i];
+            }
         }
         __syncthreads();
         const uint32_t digit = bc[0], above = bc[1], inbin = bc[2];
-        prefix |= digit << shift;
-        mask |= 255u << shift;
         krem -= (int)above;
-        __syncthreads();
-        if ((int)inbin == krem) {  // the whole bin is taken: no tie to break
+        prefix |= digit << shift;
+        mask |= dm << shift;
+        if ((int)inbin == krem) {  // the k-th key's bin is taken entirely: no tie
             ties = false;
             break;
         }
     }
     const uint32_t T = prefix;
 
-    // ---- counts of this slice, exchanged over the cluster
+    // ---- counts of this slice; with a cluster, exchanged for the CTA's output offset
     uint32_t my = 0u;
-    for (int i = threadIdx.x; i < cnt; i += TK_THREADS) {
+    for (int i = threadIdx.x; i < cnt; i += NT) {
         const uint32_t kk = keys[i];
         if (ties ? kk > T : kk >= T) my += 1u << 16;
         else if (ties && kk == T) my += 1u;
     }
-    // per-thread counts fit 16 bits (cnt <= 32768 per slice, 64 per thread here)
     uint32_t ctot;
-    (void)block_incl_scan(my, wsum, &ctot);
-    if (threadIdx.x == 0) {
-        xch[0] = ctot >> 16;
-        xch[1] = ctot & 0xffffu;
-    }
-    cl_sync<CLUSTER>();
+    (void)block_scan1<NW>(my, wsum[0], &ctot);  // per-thread counts < 2^16: slices <= 40960 keys
     uint32_t gt_before = 0u, eq_before = 0u;
-    for (int q = 0; q < c; ++q) {
-        const uint32_t* px = cl_peer<CLUSTER>(xch, q);
-        gt_before += px[0];
-        eq_before += px[1];
+    if constexpr (CLUSTER) {
+        if (threadIdx.x == 0) {
+            xch[0] = ctot >> 16;
+            xch[1] = ctot & 0xffffu;
+        }
+        cl_sync<true>();
+        for (int q = 0; q < c; ++q) {
+            const uint32_t* px = cl_peer<true>(xch, q);
+            gt_before += px[0];
+            eq_before += px[1];
+        }
+        // peers read this CTA's shared memory no more; they may leave after the wait below
+        asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
     }
     const int quota = ties ? max(0, krem - (int)eq_before) : 0;
     const int out_base = (int)gt_before + (ties ? min((int)eq_before, krem) : 0);
 
-    // ---- ordered compaction of this slice
+    // ---- ordered compaction of the slice in tiles of 4 keys per thread
     int carry_gt = 0, carry_eq = 0;
-    for (int tb = 0; tb < cnt; tb += TK_TILE) {
-        const int i0 = tb + threadIdx.x * TK_IPT;
+    int tile = 1;  // wsum[1] is free from here on; tiles alternate 1, 0, 1, ...
+    for (int tb = 0; tb < cnt; tb += S::TILE, tile ^= 1) {
+        const int i0 = tb + threadIdx.x * 4;
         uint4 kv = make_uint4(0u, 0u, 0u, 0u);
         if (i0 < cnt) kv = tk_dyn[i0 >> 2];
         const uint32_t kk[4] = {kv.x, kv.y, kv.z, kv.w};
@@ -221,7 +312,7 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const TopkArgs a, int 
         }
         const uint32_t packed = ((uint32_t)__popc(gm) << 16) | (uint32_t)__popc(em);
         uint32_t ttot;
-        const uint32_t excl = block_incl_scan(packed, wsum, &ttot) - packed;
+        const uint32_t excl = block_scan1<NW>(packed, wsum[tile], &ttot) - packed;
         int gb = carry_gt + (int)(excl >> 16);
         int eb = carry_eq + (int)(excl & 0xffffu);
 #pragma unroll
@@ -247,52 +338,47 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const TopkArgs a, int 
         carry_gt += (int)(ttot >> 16);
         carry_eq += (int)(ttot & 0xffffu);
     }
-    cl_sync<CLUSTER>();  // no CTA leaves while a peer may still read its shared memory
+    if constexpr (CLUSTER) asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+template <int NT, bool CLUSTER>
+cudaError_t launch_one(const TopkArgs& a, int row0, int nr, int cs, int chunk, cudaStream_t st) {
+    using S = TopkShape<NT, CLUSTER>;
+    static bool attr_done[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_done[dev]) {
+        cudaFuncSetAttribute(topk_kernel<NT, CLUSTER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)S::smem(TK_SMEM_ROW));
+        attr_done[dev] = true;
+    }
+    return launch_pdl(topk_kernel<NT, CLUSTER>, dim3(CLUSTER ? cs : 1, nr), dim3(NT), S::smem(chunk), st,
+                      CLUSTER ? cs : 1, a, row0, chunk);
 }
 
 }  // namespace
 
 li_status launch_topk(const TopkArgs& a, cudaStream_t st) {
     if (a.rows <= 0) return LI_OK;
-    const int sms = host_num_sms();
     const int maxl = max(a.max_len, 1);
-    int cs = 1;
-    if (a.rows < sms) cs = min(8, (2 * sms + a.rows - 1) / a.rows);
+    const int sms = host_num_sms();
     auto chunk_of = [&](int csz) { return (((maxl + csz - 1) / csz) + 3) & ~3; };
-    while (cs < 8 && chunk_of(cs) * 4 > TK_MAX_SMEM) ++cs;
-    // keep small rows on few CTAs: a slice below one compaction tile wastes the cluster
-    while (cs > 1 && chunk_of(cs) < TK_TILE / 2 && chunk_of(cs / 2) * 4 <= TK_MAX_SMEM) cs /= 2;
+    // few rows: split each row over a cluster so that about 4K keys land on each CTA
+    // (the load and every sweep run on many SMs); many rows: one CTA per row
+    int cs = 1;
+    if (a.rows < sms)
+        while (cs < TK_MAX_CS && chunk_of(cs) > TK_SLICE) cs *= 2;
+    while (cs < TK_MAX_CS && chunk_of(cs) > TK_SMEM_ROW) cs *= 2;
     const int chunk = chunk_of(cs);
-    if (chunk * 4 > TK_MAX_SMEM || chunk > 32768) return LI_ERR_UNSUPPORTED;
-    const size_t smem = (size_t)chunk * 4;
-
-    static bool attr_done[64][2] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !attr_done[dev][cs > 1]) {
-        if (cs > 1) cudaFuncSetAttribute(topk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, TK_MAX_SMEM);
-        else cudaFuncSetAttribute(topk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, TK_MAX_SMEM);
-        attr_done[dev][cs > 1] = true;
-    }
+    if (chunk > TK_SMEM_ROW) return LI_ERR_UNSUPPORTED;
+    const bool small = chunk <= 8192;
     for (int row0 = 0; row0 < a.rows; row0 += 65535) {
         const int nr = min(65535, a.rows - row0);
-        if (cs == 1) {
-            topk_kernel<false><<<dim3(1, nr), TK_THREADS, smem, st>>>(a, row0, chunk);
-        } else {
-            cudaLaunchConfig_t cfg = {};
-            cfg.gridDim = dim3(cs, nr);
-            cfg.blockDim = dim3(TK_THREADS);
-            cfg.dynamicSmemBytes = smem;
-            cfg.stream = st;
-            cudaLaunchAttribute attr[1];
-            attr[0].id = cudaLaunchAttributeClusterDimension;
-            attr[0].val.clusterDim.x = cs;
-            attr[0].val.clusterDim.y = 1;
-            attr[0].val.clusterDim.z = 1;
-            cfg.attrs = attr;
-            cfg.numAttrs = 1;
-            if (cudaLaunchKernelEx(&cfg, topk_kernel<true>, a, row0, chunk) != cudaSuccess) return host_check_launch();
-        }
+        cudaError_t e;
+        if (cs == 1) e = small ? launch_one<256, false>(a, row0, nr, cs, chunk, st)
+                               : launch_one<1024, false>(a, row0, nr, cs, chunk, st);
+        else e = launch_one<512, true>(a, row0, nr, cs, chunk, st);
+        if (e != cudaSuccess) return host_check_launch();
         const li_status s = host_check_launch();
         if (s != LI_OK) return s;
     }

@@ -207,3 +207,25 @@ def test_unsupported_shapes_raise():
     ks = torch.ones(2, 64, device=DEV)
     with pytest.raises(LiError):
         api.li_index_score(q, w, k, ks)
+
+
+# ---------------------------------------------------------------------------
+# graph-captured decode step (public API): host inputs in, selections out
+# ---------------------------------------------------------------------------
+def test_decode_indexer_graph_step():
+    from sparse_attention_lightning_score_b200.step import DecodeIndexer
+    case = synth.dsa_decode(B=3, L=5000, k_top=300, seed=23, lens=[5000, 2100, 40])
+    ix = DecodeIndexer(case.k8.to(DEV), case.ks.to(DEV), heads=64, k=300, lens=case.lens.to(DEV))
+    ref, _ = _oracle_decode(case)
+    ridx, _ = oracle.topk(ref, 300, lens=case.lens.numpy())
+    got = ix.step(case.q, case.w).numpy().copy()
+    assert_topk_equivalent(got, ridx, ref, 1e-2, n_valid=case.lens.numpy())
+    # a second step with new inputs through the same graph
+    case2 = synth.dsa_decode(B=3, L=5000, k_top=300, seed=24, lens=[5000, 2100, 40])
+    case2.k8, case2.ks = case.k8, case.ks
+    ref2, _ = _oracle_decode(case2)
+    ridx2, _ = oracle.topk(ref2, 300, lens=case.lens.numpy())
+    got2 = ix.step(case2.q, case2.w).numpy().copy()
+    assert_topk_equivalent(got2, ridx2, ref2, 1e-2, n_valid=case.lens.numpy())
+    assert ix.h2d_bytes == 3 * 64 * 128 * 2 + 3 * 64 * 4 and ix.d2h_bytes == 3 * 300 * 4
+    assert api.li_get_last_error() == LI_OK
