@@ -210,7 +210,13 @@ def capture(fns):
 
 
 class DecodeBench:
-    """Decode-step launches over rotating key caches, as graphs."""
+    """Decode-step launches over rotating key caches, as graphs.
+
+    A step is li_decode_select: the scorer (which also counts each row's first
+    radix digit into a histogram) and the top-k that starts from it.  The two
+    kernels are also timed alone through the call's two halves: the scorer
+    into a scratch histogram, the top-k from a saved histogram restored by a
+    device copy before each launch (the copy's own time is subtracted)."""
 
     def __init__(self, dev, Lx, seed):
         import torch
@@ -222,17 +228,31 @@ class DecodeBench:
         self.q, self.w = self.case.q.to(dev), self.case.w.to(dev)
         self.sc = torch.empty((B, Lx), dtype=torch.float32, device=dev)
         self.idx = torch.empty((B, KTOP), dtype=torch.int32, device=dev)
+        self.ws = api.li_decode_select_workspace(B, dev)
+        nh = B * 2048
+        self.hist_scratch = api.li_decode_select_workspace(B, dev).view(torch.int32)[:nh]
+        # scores + their histogram for the top-k-only timing
+        self.sc_t = torch.empty_like(self.sc)
+        self.idx_t = torch.empty_like(self.idx)
+        self.hist_saved = api.li_decode_select_workspace(B, dev).view(torch.int32)[:nh]
+        self.hist_t = api.li_decode_select_workspace(B, dev).view(torch.int32)[:nh]
+        kk, ss = self.sets[0]
+        api.li_decode_score_hist(self.q, self.w, kk, ss, self.hist_saved, scores=self.sc_t)
 
     def score(self, i):
         kk, ss = self.sets[i % self.n]
-        self.api.li_index_score(self.q, self.w, kk, ss, scores=self.sc)
+        self.api.li_decode_score_hist(self.q, self.w, kk, ss, self.hist_scratch, scores=self.sc)
+
+    def restore(self):
+        self.hist_t.copy_(self.hist_saved)
 
     def topk(self):
-        self.api.li_topk(self.sc, KTOP, idx=self.idx)
+        self.restore()
+        self.api.li_topk_hist(self.sc_t, KTOP, self.hist_t, idx=self.idx_t)
 
     def step(self, i):
-        self.score(i)
-        self.topk()
+        kk, ss = self.sets[i % self.n]
+        self.api.li_decode_select(self.q, self.w, kk, ss, KTOP, scores=self.sc, workspace=self.ws, idx=self.idx)
 
     def build_graphs(self, warmup):
         import torch
@@ -240,18 +260,39 @@ class DecodeBench:
             self.step(i)
         torch.cuda.synchronize()
         self.step_graphs = [capture([lambda i=i: self.step(i)]) for i in range(self.n)]
+        # one graph holding a step over every rotating set, back to back (as the
+        # indexer's kernels sit inside a model's decode graph)
+        self.loop_graph = capture([lambda i=i: self.step(i) for i in range(self.n)])
         reps = max(1, 24 // self.n)
         self.score_graph = capture([lambda i=i: self.score(i) for i in range(self.n * reps)])
         self.score_launches = self.n * reps
         self.topk_graph = capture([self.topk] * 16)
         self.topk_launches = 16
+        self.restore_graph = capture([self.restore] * 16)
         for g in self.step_graphs:
             g.replay()
+        self.loop_graph.replay()
         self.score_graph.replay()
         self.topk_graph.replay()
+        self.restore_graph.replay()
         torch.cuda.synchronize()
 
     def time_steps(self, steps):
+        """Exactly `steps` decode steps: whole loop graphs (one step per rotating
+        set each), then single-step graphs for the remainder."""
+        import torch
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps // self.n):
+            self.loop_graph.replay()
+        for i in range(steps % self.n):
+            self.step_graphs[i].replay()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    def time_steps_single(self, steps):
+        """The same steps, one graph launch per step."""
         import torch
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
@@ -261,9 +302,8 @@ class DecodeBench:
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / steps
 
-    def time_kernel(self, which, reps=3):
+    def _time_graph(self, g, n, reps):
         import torch
-        g, n = (self.score_graph, self.score_launches) if which == "score" else (self.topk_graph, self.topk_launches)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         for _ in range(reps):
@@ -271,6 +311,12 @@ class DecodeBench:
         e1.record()
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / (reps * n)
+
+    def time_kernel(self, which, reps=3):
+        if which == "score":
+            return self._time_graph(self.score_graph, self.score_launches, reps)
+        both = self._time_graph(self.topk_graph, self.topk_launches, reps)
+        return both - self._time_graph(self.restore_graph, self.topk_launches, reps)
 
     def time_direct(self, steps):
         import torch
@@ -310,7 +356,9 @@ def run_li(args, rank, world, local_rank):
     score_ms = bench.time_kernel("score")
     topk_ms = bench.time_kernel("topk")
     direct_ms = bench.time_direct(args.steps)
-    ms, score_ms, topk_ms, direct_ms = li_dist.max_over_ranks([ms, score_ms, topk_ms, direct_ms], device=dev)
+    single_ms = bench.time_steps_single(args.steps)
+    ms, score_ms, topk_ms, direct_ms, single_ms = li_dist.max_over_ranks(
+        [ms, score_ms, topk_ms, direct_ms, single_ms], device=dev)
     launches = 2 * args.steps
 
     # ---- end to end through the public API: each step copies the pinned host
@@ -375,16 +423,17 @@ def run_li(args, rank, world, local_rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
         "config": {"workload": WORKLOAD, "B": B, "L": L, "H": H, "d": D, "k": KTOP,
                    "l2": f"{bench.n} rotating key-cache copies, {bench.set_bytes / 1e6:.0f} MB > 126 MB L2",
-                   "launch": "CUDA graph per step (score + top-k)", "per_rank": "own batch of B requests"},
+                   "launch": "CUDA graphs of back-to-back steps (li_decode_select: score + top-k per step)",
+                   "per_rank": "own batch of B requests"},
         "roofline": {"bound": "hbm", "kernel": SCORER_KERNEL, "achieved": achieved, "peak": hbm,
                      "peak_source": which, "unit": "GB/s", "frac": achieved / hbm,
                      "traffic": traffic_for(SCORER_KERNEL, units), "algorithmic_bytes": algo_bytes,
                      "kernel_us": score_ms * 1e3},
         "topk": {"us": topk_ms * 1e3, "rows_per_s": B / (topk_ms * 1e-3), "row_len": L, "k": KTOP},
-        "direct_us_per_step": direct_ms * 1e3,
+        "direct_us_per_step": direct_ms * 1e3, "graph_per_step_us": single_ms * 1e3,
         "e2e": {"value": world * B * L / (e2e_ms * 1e-3), "unit": "keys/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-                "api": "DecodeIndexer.step (graph: H2D q,w -> score -> top-k -> D2H indices)"},
+                "api": "DecodeIndexer.step (graph: H2D q,w -> li_decode_select -> D2H indices)"},
         "gpu_launches": launches,
         "clocks": clk,
     }

@@ -142,6 +142,56 @@ li_status li_topk(const float* scores, int64_t scores_ld, const int32_t* len, in
                   int causal_offset, int k, int32_t* idx, float* vals, li_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Decode indexer step: score, then select                                   */
+/* ------------------------------------------------------------------------ */
+/* One decode step of the indexer: li_index_score in its decode form (causal
+ * 0) followed by li_topk(k_top) on the same scores, with identical results.
+ * The difference is internal.  The pages run the indexer as a full scan
+ * followed by top-k ("one score per visible position ... before top-k",
+ * IndexCache explainer, Symbol Map), and this call follows that order.  While
+ * writing each score, the scorer also counts it by the top 11 bits of the
+ * selection's order key.  The top-k takes its first radix digit from those
+ * counts instead of sweeping the row for it.
+ *   q, w, k, k_scale, cache_batch_rows, len, scores, scores_ld, desc
+ *           as li_index_score (desc->causal must be 0; tensor-core path only:
+ *           BF16 query, E4M3 keys, heads 64, dim 128).  scores_ld must be a
+ *           multiple of 4 and scores 16-byte aligned, as li_topk requires.
+ *   k_top, idx, vals   as li_topk's k, idx, vals.
+ *   workspace  li_decode_select_workspace(desc) bytes of device memory,
+ *           256-byte aligned, holding one 2048-bin histogram per row.  It must
+ *           be all zero before the first call (a cudaMemset after allocating
+ *           it).  Each call leaves it all zero again when its kernels
+ *           complete.  Calls that overlap in time must not share one.
+ * If the workspace was not zero, the result is still exact, but slower:
+ * the top-k checks the counts against the keys and runs its plain passes.
+ * The next li_get_last_error then reports LI_ERR_BOUNDS.  The histogram is
+ * zero again afterwards. */
+li_status li_decode_select(const void* q, const float* w, const void* k, const float* k_scale, int64_t cache_batch_rows,
+                           const int32_t* len, float* scores, int64_t scores_ld, const li_score_desc* desc, int k_top,
+                           int32_t* idx, float* vals, void* workspace, size_t workspace_bytes, li_stream_t stream);
+
+/* Bytes of zeroed device workspace li_decode_select needs (0 when desc->rows <= 0). */
+size_t li_decode_select_workspace(const li_score_desc* desc);
+
+/* The two halves of li_decode_select, for callers that place them
+ * separately; li_decode_select is exactly this pair on one stream.
+ * li_decode_score_hist: li_index_score in its decode form (same arguments and
+ *   restrictions as li_decode_select).  For every score it writes, it also
+ *   adds 1 to hist[r * 2048 + (key >> 21)], where key is the score's order key
+ *   (fp32 bits made monotonic: larger score, larger key; NaN lowest; -0.0
+ *   as +0.0).  hist: [rows, 2048] uint32, 16-byte aligned, zero before the
+ *   call; it is added to, not overwritten.
+ * li_topk_hist: li_topk (causal 0) that takes its first digit from hist and
+ *   leaves hist all zero.  The result equals li_topk's for any hist.  When hist
+ *   does not count exactly the row's scores, the call reports LI_ERR_BOUNDS
+ *   through li_get_last_error and selects without it. */
+li_status li_decode_score_hist(const void* q, const float* w, const void* k, const float* k_scale,
+                               int64_t cache_batch_rows, const int32_t* len, float* scores, int64_t scores_ld,
+                               const li_score_desc* desc, uint32_t* hist, li_stream_t stream);
+li_status li_topk_hist(const float* scores, int64_t scores_ld, const int32_t* len, int rows, int max_len, int k,
+                       int32_t* idx, float* vals, uint32_t* hist, li_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* LatentIndex: decoder absorption and latent-cache scoring                  */
 /* ------------------------------------------------------------------------ */
 /* Absorbs one layer's key decoder into its queries (LatentIndex abstract,
@@ -150,7 +200,7 @@ li_status li_topk(const float* scores, int64_t scores_ld, const int32_t* len, in
  *   q_bf16      [batch, heads, dim] bf16
  *   w_dec_bf16  [heads, dim, latent_dim] bf16 (maps a latent row to head j's key)
  *   q_tilde     [batch, heads, latent_dim] bf16 (out)
- * dim <= 256, latent_dim a multiple of 64. */
+ * dim <= 256, latent_dim a multiple of 64, w_dec 16-byte aligned. */
 li_status li_absorb_query(const void* q_bf16, const void* w_dec_bf16, void* q_tilde_bf16, int batch, int heads,
                           int dim, int latent_dim, li_stream_t stream);
 

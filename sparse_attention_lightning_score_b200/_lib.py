@@ -35,6 +35,11 @@ SIGNATURES = {
     "li_index_score": (i32, [vp, vp, vp, vp, i64, vp, vp, i64, ctypes.POINTER(ScoreDesc), vp, sz, vp]),
     "li_index_score_workspace": (sz, [ctypes.POINTER(ScoreDesc)]),
     "li_topk": (i32, [vp, i64, vp, i32, i32, i32, i32, i32, vp, vp, vp]),
+    "li_decode_select": (i32, [vp, vp, vp, vp, i64, vp, vp, i64, ctypes.POINTER(ScoreDesc), i32, vp, vp, vp, sz,
+                               vp]),
+    "li_decode_select_workspace": (sz, [ctypes.POINTER(ScoreDesc)]),
+    "li_decode_score_hist": (i32, [vp, vp, vp, vp, i64, vp, vp, i64, ctypes.POINTER(ScoreDesc), vp, vp]),
+    "li_topk_hist": (i32, [vp, i64, vp, i32, i32, i32, vp, vp, vp, vp]),
     "li_absorb_query": (i32, [vp, vp, vp, i32, i32, i32, i32, vp]),
     "li_latent_score": (i32, [vp, vp, vp, i64, vp, vp, i64, i32, i32, i32, i32, vp]),
     "li_hs_refine": (i32, [vp, i64, i64, vp, i32, i32, vp, vp, i32, i32, i32, i32, vp, vp, sz, vp]),

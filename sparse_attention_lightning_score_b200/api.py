@@ -122,6 +122,97 @@ def li_topk(scores: torch.Tensor, k: int, *, lens: Optional[torch.Tensor] = None
     return (idx, vals) if with_values else idx
 
 
+def li_decode_select_workspace(rows: int, device) -> torch.Tensor:
+    """A zeroed workspace for li_decode_select over `rows` requests (it stays zero between calls)."""
+    desc = score_desc(rows, 64, 128, 0)
+    need = _lib.load().li_decode_select_workspace(ctypes.byref(desc))
+    return torch.zeros(max(int(need), 256), dtype=torch.uint8, device=device)
+
+
+def li_decode_select(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, k_scale: torch.Tensor, k_top: int, *,
+                     lens: Optional[torch.Tensor] = None, scores: Optional[torch.Tensor] = None,
+                     workspace: Optional[torch.Tensor] = None, with_values: bool = False, idx=None, vals=None,
+                     stream=None):
+    """Decode score + top-k in one call -> (scores, idx[, vals]).
+
+    Same arguments as li_index_score's decode form (q bf16 [B,64,128], k e4m3 [B,L,128] or [L,128],
+    k_scale) and li_topk's k / outputs.  `workspace` is a zeroed buffer from li_decode_select_workspace
+    (made here when omitted); it is left zero again for the next call.
+    """
+    _need(q, "q", torch.bfloat16)
+    _need(w, "w", torch.float32)
+    _need(k, "k")
+    _need(k_scale, "k_scale", torch.float32)
+    if k.dtype == torch.float8_e4m3fn:
+        k = k.view(torch.uint8)
+    R, H, d = q.shape
+    L = k.shape[-2]
+    batch_rows = k.shape[1] if k.dim() == 3 else 0
+    if lens is not None:
+        _need(lens, "lens", torch.int32)
+    desc = score_desc(R, H, d, L)
+    lib = _lib.load()
+    if scores is None:
+        scores = torch.empty((R, _round4(L)), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = li_decode_select_workspace(R, q.device)
+    if idx is None:
+        idx = torch.empty((R, k_top), dtype=torch.int32, device=q.device)
+    if with_values and vals is None:
+        vals = torch.empty((R, k_top), dtype=torch.float32, device=q.device)
+    st = lib.li_decode_select(_ptr(q), _ptr(w), _ptr(k), _ptr(k_scale), batch_rows, _ptr(lens), _ptr(scores),
+                              scores.stride(0), ctypes.byref(desc), int(k_top), _ptr(idx),
+                              _ptr(vals) if with_values else None, _ptr(workspace), workspace.numel(),
+                              _stream(stream))
+    _lib.check("li_decode_select", st)
+    return (scores, idx, vals) if with_values else (scores, idx)
+
+
+def li_decode_score_hist(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, k_scale: torch.Tensor,
+                         hist: torch.Tensor, *, lens: Optional[torch.Tensor] = None,
+                         scores: Optional[torch.Tensor] = None, stream=None):
+    """First half of li_decode_select: decode scores, plus counts added to `hist` (a zeroed
+    li_decode_select_workspace buffer)."""
+    _need(q, "q", torch.bfloat16)
+    _need(w, "w", torch.float32)
+    _need(k, "k")
+    _need(k_scale, "k_scale", torch.float32)
+    if k.dtype == torch.float8_e4m3fn:
+        k = k.view(torch.uint8)
+    R, H, d = q.shape
+    L = k.shape[-2]
+    batch_rows = k.shape[1] if k.dim() == 3 else 0
+    if lens is not None:
+        _need(lens, "lens", torch.int32)
+    if scores is None:
+        scores = torch.empty((R, _round4(L)), dtype=torch.float32, device=q.device)
+    desc = score_desc(R, H, d, L)
+    st = _lib.load().li_decode_score_hist(_ptr(q), _ptr(w), _ptr(k), _ptr(k_scale), batch_rows, _ptr(lens),
+                                          _ptr(scores), scores.stride(0), ctypes.byref(desc), _ptr(hist),
+                                          _stream(stream))
+    _lib.check("li_decode_score_hist", st)
+    return scores
+
+
+def li_topk_hist(scores: torch.Tensor, k: int, hist: torch.Tensor, *, lens: Optional[torch.Tensor] = None,
+                 max_len: Optional[int] = None, with_values: bool = False, idx=None, vals=None, stream=None):
+    """Second half of li_decode_select: li_topk using (and clearing) the scorer's histogram."""
+    _need(scores, "scores", torch.float32)
+    rows, ld = scores.shape
+    if max_len is None:
+        max_len = ld
+    if lens is not None:
+        _need(lens, "lens", torch.int32)
+    if idx is None:
+        idx = torch.empty((rows, k), dtype=torch.int32, device=scores.device)
+    if with_values and vals is None:
+        vals = torch.empty((rows, k), dtype=torch.float32, device=scores.device)
+    st = _lib.load().li_topk_hist(_ptr(scores), ld, _ptr(lens), rows, int(max_len), int(k), _ptr(idx),
+                                  _ptr(vals) if with_values else None, _ptr(hist), _stream(stream))
+    _lib.check("li_topk_hist", st)
+    return (idx, vals) if with_values else idx
+
+
 def li_absorb_query(q: torch.Tensor, w_dec: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None):
     """q bf16 [B,H,d], W_dec bf16 [H,d,dc] -> q~ bf16 [B,H,dc]."""
     _need(q, "q", torch.bfloat16)

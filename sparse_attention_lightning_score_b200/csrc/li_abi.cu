@@ -221,8 +221,85 @@ li_status li_topk(const float* scores, int64_t scores_ld, const int32_t* len, in
     if (causal && len) return LI_ERR_INVALID_ARG;
     DevErr e;
     if (ready(&e) != LI_OK) return LI_ERR_CUDA;
-    TopkArgs a{scores, scores_ld, len, rows, max_len, causal ? 1 : 0, causal_offset, k, idx, vals, nullptr, 0, 1, e};
+    TopkArgs a{scores, scores_ld, len, rows, max_len, causal ? 1 : 0, causal_offset, k, idx, vals, nullptr, 0, 1,
+                nullptr, 0, e};
     return launch_topk(a, stream);
+}
+
+size_t li_decode_select_workspace(const li_score_desc* d) {
+    if (!d || d->rows <= 0) return 0;
+    return align_up((size_t)d->rows * LI_HIST_BINS * sizeof(uint32_t), 256);
+}
+
+li_status li_decode_score_hist(const void* q, const float* w, const void* k, const float* k_scale,
+                               int64_t cache_batch_rows, const int32_t* len, float* scores, int64_t scores_ld,
+                               const li_score_desc* desc, uint32_t* hist, li_stream_t stream) {
+    if (!desc) return LI_ERR_INVALID_ARG;
+    const li_score_desc d = *desc;
+    if (d.rows < 0 || d.heads <= 0 || d.dim <= 0 || d.max_len < 0 || cache_batch_rows < 0 || d.causal)
+        return LI_ERR_INVALID_ARG;
+    if (d.rows == 0 || d.max_len == 0) return LI_OK;
+    if (d.q_dtype != LI_DTYPE_BF16 || d.k_dtype != LI_DTYPE_E4M3) return LI_ERR_UNSUPPORTED;
+    if (d.heads != 64 || d.dim != 128) return LI_ERR_UNSUPPORTED;
+    if (!q || !w || !k || !k_scale || !scores || !hist || scores_ld < d.max_len) return LI_ERR_INVALID_ARG;
+    if (!aligned(k, 16) || !aligned(q, 16) || !aligned(hist, 16)) return LI_ERR_INVALID_ARG;
+    DevErr e;
+    if (ready(&e) != LI_OK) return LI_ERR_CUDA;
+    const uint64_t total_rows = cache_batch_rows > 0 ? (uint64_t)(d.rows - 1) * cache_batch_rows + d.max_len
+                                                     : (uint64_t)d.max_len;
+    if (total_rows >= (1ull << 31)) return LI_ERR_UNSUPPORTED;
+    CUtensorMap kmap;
+    if (!encode_map_2d(&kmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, k, 128, total_rows, 128, 128, 128)) return LI_ERR_CUDA;
+    StreamArgs a{};
+    a.q = q;
+    a.w = w;
+    a.kscale = k_scale;
+    a.len = len;
+    a.scores = scores;
+    a.scores_ld = scores_ld;
+    a.batch_rows = cache_batch_rows;
+    a.max_len = d.max_len;
+    a.hist = hist;
+    a.err = e;
+    return launch_stream_score_fp8_hist(kmap, a, d.rows, (d.max_len + 127) / 128, stream);
+}
+
+li_status li_topk_hist(const float* scores, int64_t scores_ld, const int32_t* len, int rows, int max_len, int k,
+                       int32_t* idx, float* vals, uint32_t* hist, li_stream_t stream) {
+    if (rows < 0 || max_len < 0 || k < 1 || k > LI_TOPK_MAX_LEN || max_len > LI_TOPK_MAX_LEN) return LI_ERR_INVALID_ARG;
+    if (rows == 0) return LI_OK;
+    if (!idx || !hist || (!scores && max_len > 0) || scores_ld < max_len || (scores_ld % 4) != 0)
+        return LI_ERR_INVALID_ARG;
+    if ((scores && !aligned(scores, 16)) || !aligned(hist, 16)) return LI_ERR_INVALID_ARG;
+    DevErr e;
+    if (ready(&e) != LI_OK) return LI_ERR_CUDA;
+    TopkArgs a{scores, scores_ld, len, rows, max_len, 0, 0, k, idx, vals, nullptr, 0, 1, hist, 0, e};
+    return launch_topk(a, stream);
+}
+
+li_status li_decode_select(const void* q, const float* w, const void* k, const float* k_scale, int64_t cache_batch_rows,
+                           const int32_t* len, float* scores, int64_t scores_ld, const li_score_desc* desc, int k_top,
+                           int32_t* idx, float* vals, void* workspace, size_t workspace_bytes, li_stream_t stream) {
+    if (!desc) return LI_ERR_INVALID_ARG;
+    const li_score_desc d = *desc;
+    if (d.rows < 0 || d.heads <= 0 || d.dim <= 0 || d.max_len < 0 || cache_batch_rows < 0 || d.causal)
+        return LI_ERR_INVALID_ARG;
+    if (k_top < 1 || k_top > LI_TOPK_MAX_LEN || d.max_len > LI_TOPK_MAX_LEN) return LI_ERR_INVALID_ARG;
+    if (d.rows == 0) return LI_OK;
+    if (d.q_dtype != LI_DTYPE_BF16 || d.k_dtype != LI_DTYPE_E4M3) return LI_ERR_UNSUPPORTED;
+    if (d.heads != 64 || d.dim != 128) return LI_ERR_UNSUPPORTED;
+    if (!idx || !workspace || workspace_bytes < li_decode_select_workspace(&d) || !aligned(workspace, 256))
+        return LI_ERR_INVALID_ARG;
+    if (d.max_len > 0) {
+        if (!q || !w || !k || !k_scale || !scores || scores_ld < d.max_len || (scores_ld % 4) != 0)
+            return LI_ERR_INVALID_ARG;
+        if (!aligned(k, 16) || !aligned(q, 16) || !aligned(scores, 16)) return LI_ERR_INVALID_ARG;
+    }
+    uint32_t* hist = static_cast<uint32_t*>(workspace);
+    const li_status s = li_decode_score_hist(q, w, k, k_scale, cache_batch_rows, len, scores, scores_ld, desc, hist,
+                                             stream);
+    if (s != LI_OK) return s;
+    return li_topk_hist(scores, d.max_len > 0 ? scores_ld : 4, len, d.rows, d.max_len, k_top, idx, vals, hist, stream);
 }
 
 li_status li_absorb_query(const void* q_bf16, const void* w_dec_bf16, void* q_tilde_bf16, int batch, int heads,
@@ -231,7 +308,7 @@ li_status li_absorb_query(const void* q_bf16, const void* w_dec_bf16, void* q_ti
         heads > 65535)
         return LI_ERR_INVALID_ARG;
     if (batch == 0) return LI_OK;
-    if (!q_bf16 || !w_dec_bf16 || !q_tilde_bf16 || !aligned(w_dec_bf16, 4) || !aligned(q_tilde_bf16, 4))
+    if (!q_bf16 || !w_dec_bf16 || !q_tilde_bf16 || !aligned(w_dec_bf16, 16) || !aligned(q_tilde_bf16, 2))
         return LI_ERR_INVALID_ARG;
     DevErr e;
     if (ready(&e) != LI_OK) return LI_ERR_CUDA;
@@ -285,7 +362,7 @@ li_status li_hs_refine(const void* c_bf16, int64_t cache_batch_rows, int64_t cac
     DevErr e;
     if (ready(&e) != LI_OK) return LI_ERR_CUDA;
     if (n_cand == 0) {
-        TopkArgs t{nullptr, 4, nullptr, followers * batch, 0, 0, 0, k, out_idx, nullptr, nullptr, 0, 1, e};
+        TopkArgs t{nullptr, 4, nullptr, followers * batch, 0, 0, 0, k, out_idx, nullptr, nullptr, 0, 1, nullptr, 0, e};
         return launch_topk(t, stream);
     }
     if (!c_bf16 || !cand || !q_tilde_bf16 || !w || !aligned(c_bf16, 16) || !aligned(q_tilde_bf16, 16))
@@ -297,7 +374,8 @@ li_status li_hs_refine(const void* c_bf16, int64_t cache_batch_rows, int64_t cac
     HsArgs h{c_bf16, cache_batch_rows, cache_rows, cand, batch, n_cand, followers, q_tilde_bf16, w, sc, e};
     li_status s = launch_hs_rescore(h, stream);
     if (s != LI_OK) return s;
-    TopkArgs t{sc, ldw, nullptr, followers * batch, n_cand, 0, 0, k, out_idx, nullptr, cand, n_cand, batch, e};
+    TopkArgs t{sc, ldw, nullptr, followers * batch, n_cand, 0, 0, k, out_idx, nullptr, cand, n_cand, batch,
+               nullptr, 0, e};
     return launch_topk(t, stream);
 }
 

@@ -275,6 +275,21 @@ __device__ __forceinline__ float relu_dot32(const uint32_t (&v)[32], const float
     return (a0 + a1) + (a2 + a3);
 }
 
+// Order-preserving uint32 image of an fp32 score for the top-k: larger score,
+// larger key; NaN maps to 0 (below -inf), -0.0 to the key of +0.0.
+__device__ __forceinline__ uint32_t order_key(float f) {
+    if (f != f) return 0u;
+    uint32_t u = __float_as_uint(f);
+    if (f == 0.f) u = 0u;
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// The decode scorer counts the top LI_HIST_BITS bits of every score's key
+// into a per-row histogram that the top-k then uses as its first radix digit.
+constexpr int LI_HIST_BITS = 11;
+constexpr int LI_HIST_BINS = 1 << LI_HIST_BITS;
+constexpr int LI_HIST_SHIFT = 32 - LI_HIST_BITS;
+
 // acc.{x,y} += a.{0,1} * b.{0,1} with one packed fp32x2 FMA (same rounding as two fmaf).
 __device__ __forceinline__ void ffma2(float2& acc, float a0, float a1, float b0, float b1) {
     asm("{\n\t.reg .b64 ra, rb, rc;\n\t"

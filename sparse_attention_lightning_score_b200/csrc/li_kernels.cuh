@@ -22,10 +22,14 @@ struct StreamArgs {
     long long batch_rows;   // cache rows between requests (0 = shared cache)
     int max_len;
     int tiles_per_cta;      // set by the launcher
+    uint32_t* hist;         // FP8 kind, optional: [B, LI_HIST_BINS] counts of order_key(score) >> LI_HIST_SHIFT are
+                            // added to it (the caller provides it zeroed)
     DevErr err;
 };
 li_status launch_stream_score_fp8(const CUtensorMap& map, const StreamArgs& args, int batch, int ntiles_max,
                                   cudaStream_t st);
+li_status launch_stream_score_fp8_hist(const CUtensorMap& map, const StreamArgs& args, int batch, int ntiles_max,
+                                       cudaStream_t st);
 li_status launch_stream_score_bf16(const CUtensorMap& map, const StreamArgs& args, int batch, int ntiles_max,
                                    cudaStream_t st);
 
@@ -74,6 +78,11 @@ struct TopkArgs {
     const int32_t* map;
     long long map_ld;
     int map_rows;
+    // optional [rows, LI_HIST_BINS] histogram of the rows' keys by their top
+    // LI_HIST_BITS bits (counted by the decode scorer); the top-k takes its first
+    // digit from it and leaves it all zero
+    uint32_t* hist;
+    int cand_cap;           // set by the launcher: candidate keys one CTA can hold
     DevErr err;
 };
 li_status launch_topk(const TopkArgs& a, cudaStream_t st);

@@ -19,7 +19,11 @@
 // warps per TMEM lane quarter, one per token).  The epilogue is exact fp32:
 // ReLU as FMNMX and the head-weighted sum as packed fp32x2 FMAs, 1.5
 // instructions per logit; sixteen warps keep enough of them in flight to
-// overlap the next tile's MMA.
+// overlap the next tile's MMA.  A warp holds its token's 64 head weights in
+// registers for the whole block: read from shared memory per tile, the
+// broadcast loads alone kept the load/store pipe busier than the tensor pipe.
+// The next block's weights are fetched from global memory while the current
+// block's tiles are processed.
 #include "li_common.cuh"
 #include "li_kernels.cuh"
 
@@ -42,6 +46,27 @@ constexpr int PF_OFF_TMEM = PF_OFF_BAR + PF_NBAR * 8;
 constexpr int PF_SMEM = PF_OFF_TMEM + 16 + 1024;
 constexpr int PF_THREADS = 576;
 constexpr int PF_EPI_THREADS = 512;
+
+// 16 consecutive TMEM columns of this thread's lane (32x32b shape, 16 repeats).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+// a0/a1 += w[j] * max(v[j - j0], 0) for the 16 heads j0 .. j0+15 (packed fp32x2 FMAs).
+template <int J0>
+__device__ __forceinline__ void relu_acc16(const uint32_t (&v)[16], const float (&w)[PF_H], float2& a0, float2& a1) {
+#pragma unroll
+    for (int j = 0; j < 16; j += 4) {
+        ffma2(a0, fmaxf(__uint_as_float(v[j]), 0.f), fmaxf(__uint_as_float(v[j + 1]), 0.f), w[J0 + j], w[J0 + j + 1]);
+        ffma2(a1, fmaxf(__uint_as_float(v[j + 2]), 0.f), fmaxf(__uint_as_float(v[j + 3]), 0.f), w[J0 + j + 2],
+              w[J0 + j + 3]);
+    }
+}
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -167,6 +192,12 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_score_kernel(const __gr
         const int g = warp & 3;         // TMEM lane quarter
         const int u = e >> 2;           // this warp's token within the block
         const int et = threadIdx.x - 64;
+        // w_eff of block bi is staged in wbuf[bi & 1]; thread et < PF_N owns entry et
+        auto w_of = [&](int qb) {
+            const int t = qb * PF_NT + et / PF_H;
+            return (qb >= 0 && et < PF_N && t < a.T) ? __ldg(a.w_eff + (size_t)qb * PF_N + et) : 0.f;
+        };
+        float wnext = w_of(pf_block_at(0, c, G, nqb));
         uint32_t tc = 0;
         bool ok = true;
         for (int bi = 0; ok; ++bi) {
@@ -174,11 +205,20 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_score_kernel(const __gr
             if (qb < 0) break;
             const int t0 = qb * PF_NT;
             float* wb = wbuf + (bi & 1) * PF_N;
-            if (et < PF_N) {
-                const int t = t0 + et / PF_H;
-                wb[et] = t < a.T ? __ldg(a.w_eff + (size_t)t0 * PF_H + et) : 0.f;
-            }
+            if (et < PF_N) wb[et] = wnext;
             asm volatile("bar.sync 1, 512;" ::: "memory");
+            wnext = w_of(pf_block_at(bi + 1, c, G, nqb));  // consumed at the next block
+            float wr[PF_H];
+#pragma unroll
+            for (int j = 0; j < PF_H; j += 4) {
+                const float4 w4 = *reinterpret_cast<const float4*>(wb + u * PF_H + j);
+                wr[j] = w4.x;
+                wr[j + 1] = w4.y;
+                wr[j + 2] = w4.z;
+                wr[j + 3] = w4.w;
+            }
+            const int t = t0 + u;
+            float* orow = a.scores + (size_t)t * a.scores_ld;
             const int nt = pf_ntiles(qb, a);
             for (int kt = 0; kt < nt; ++kt, ++tc) {
                 const uint32_t acc = tc & 1u;
@@ -187,15 +227,24 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_score_kernel(const __gr
                 if (!mbar_wait(&accf[acc], (tc >> 1) & 1u, a.err)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t tb = tmem_base + ((uint32_t)(g * 32) << 16) + acc * PF_N + u * PF_H;
-                uint32_t v0[32], v1[32];
-                tmem_ld32(tb, v0);
-                tmem_ld32(tb + 32, v1);
+                uint32_t v[16];
+                float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+                tmem_ld16(tb, v);
+                tmem_ld_wait();
+                relu_acc16<0>(v, wr, a0, a1);
+                tmem_ld16(tb + 16, v);
+                tmem_ld_wait();
+                relu_acc16<16>(v, wr, a0, a1);
+                tmem_ld16(tb + 32, v);
+                tmem_ld_wait();
+                relu_acc16<32>(v, wr, a0, a1);
+                tmem_ld16(tb + 48, v);
                 tmem_ld_wait();
                 tc_fence_before();
                 mbar_arrive(&acce[acc]);
-                const float sum = relu_dot32_x2(v0, wb + u * PF_H) + relu_dot32_x2(v1, wb + u * PF_H + 32);
-                const int t = t0 + u;
-                if (t < a.T && s <= t + a.causal_offset && s < a.L) a.scores[(size_t)t * a.scores_ld + s] = sum * sk;
+                relu_acc16<48>(v, wr, a0, a1);
+                const float sum = (a0.x + a0.y) + (a1.x + a1.y);
+                if (t < a.T && s <= t + a.causal_offset && s < a.L) orow[s] = sum * sk;
             }
         }
     }

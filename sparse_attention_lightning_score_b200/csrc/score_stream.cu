@@ -24,6 +24,11 @@
 //               weighted ReLU sum -> one score per key.
 // Grid: (CTAs per request, requests).  Each CTA streams a contiguous range of
 // key tiles of one request; sized for two CTAs per SM.
+//
+// HIST variant (decode score + top-k): every written score's order key is also
+// counted by its top LI_HIST_BITS bits in a shared-memory histogram, which the
+// epilogue adds to the request's global histogram at the end; the top-k then
+// starts from that digit instead of sweeping the row for it.
 #include "li_common.cuh"
 #include "li_kernels.cuh"
 
@@ -31,7 +36,7 @@ namespace li {
 
 namespace {
 
-template <bool FP8, int KBLK, int STAGES, int NACC>
+template <bool FP8, int KBLK, int STAGES, int NACC, bool HIST>
 struct StreamCfg {
     static constexpr int H = 64;                       // heads = MMA N
     static constexpr int M = 128;                      // keys per tile = MMA M = TMEM lanes
@@ -42,7 +47,8 @@ struct StreamCfg {
     static constexpr int OFF_BAR = OFF_W + H * 4;
     static constexpr int NBAR = 2 * STAGES + 2 * NACC + 1;
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
-    static constexpr int SMEM = OFF_TMEM + 16 + 1024;  // + slack to align the base to 1024
+    static constexpr int OFF_HIST = OFF_TMEM + 16;
+    static constexpr int SMEM = OFF_HIST + (HIST ? LI_HIST_BINS * 4 : 0) + 1024;  // + slack to align the base to 1024
     static constexpr int TMEM_COLS = NACC * H;
     // FP8: warps 6..9 only help quantise the query in the prologue
     static constexpr int PRO_WARPS = FP8 ? 8 : 4;
@@ -55,10 +61,11 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-template <bool FP8, int KBLK, int STAGES, int NACC>
-__global__ void __launch_bounds__(StreamCfg<FP8, KBLK, STAGES, NACC>::THREADS, 2) stream_score_kernel(const __grid_constant__ CUtensorMap kmap,
-                                                           const StreamArgs a) {
-    using C = StreamCfg<FP8, KBLK, STAGES, NACC>;
+template <bool FP8, int KBLK, int STAGES, int NACC, bool HIST>
+__global__ void __launch_bounds__(StreamCfg<FP8, KBLK, STAGES, NACC, HIST>::THREADS, 2)
+    stream_score_kernel(const __grid_constant__ CUtensorMap kmap, const StreamArgs a) {
+    using C = StreamCfg<FP8, KBLK, STAGES, NACC, HIST>;
+    static_assert(!HIST || C::PRO_WARPS == 8, "the histogram is cleared by the prologue helper warps");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
 
@@ -75,6 +82,7 @@ __global__ void __launch_bounds__(StreamCfg<FP8, KBLK, STAGES, NACC>::THREADS, 2
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
     float* wsm = reinterpret_cast<float*>(smem + C::OFF_W);
     uint8_t* qsm = smem + C::OFF_Q;
+    uint32_t* hs = reinterpret_cast<uint32_t*>(smem + C::OFF_HIST);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -212,6 +220,10 @@ __global__ void __launch_bounds__(StreamCfg<FP8, KBLK, STAGES, NACC>::THREADS, 2
             }
             if (et < C::H) wsm[et] = __ldg(a.w + (size_t)b * C::H + et);
         }
+        if constexpr (HIST) {
+            if (warp >= 6)
+                for (int i = threadIdx.x - 192; i < LI_HIST_BINS; i += 128) hs[i] = 0u;
+        }
         fence_proxy_async_smem();
         mbar_arrive(qready);
         // w_eff visible to every epilogue thread
@@ -238,7 +250,20 @@ __global__ void __launch_bounds__(StreamCfg<FP8, KBLK, STAGES, NACC>::THREADS, 2
             tc_fence_before();
             mbar_arrive(&acce[acc]);
             const float sum = relu_dot32(v0, wsm) + relu_dot32(v1, wsm + 32);
-            if (s < len_b) out[s] = FP8 ? sum * sk : sum;
+            if (s < len_b) {
+                const float sc = FP8 ? sum * sk : sum;
+                out[s] = sc;
+                if constexpr (HIST) atomicAdd(&hs[order_key(sc) >> LI_HIST_SHIFT], 1u);
+            }
+        }
+        if constexpr (HIST) {
+            // all epilogue counts are in; add the non-empty bins to the request's histogram
+            asm volatile("bar.sync 2, 128;" ::: "memory");
+            uint32_t* gh = a.hist + (size_t)b * LI_HIST_BINS;
+            for (int i = et; i < LI_HIST_BINS; i += 128) {
+                const uint32_t v = hs[i];
+                if (v) atomicAdd(gh + i, v);
+            }
         }
     }
 done:
@@ -250,10 +275,10 @@ done:
     }
 }
 
-template <bool FP8, int KBLK, int STAGES, int NACC>
+template <bool FP8, int KBLK, int STAGES, int NACC, bool HIST = false>
 li_status launch_impl(const CUtensorMap& map, const StreamArgs& args, int batch, int ntiles_max, cudaStream_t st) {
-    using C = StreamCfg<FP8, KBLK, STAGES, NACC>;
-    auto kern = stream_score_kernel<FP8, KBLK, STAGES, NACC>;
+    using C = StreamCfg<FP8, KBLK, STAGES, NACC, HIST>;
+    auto kern = stream_score_kernel<FP8, KBLK, STAGES, NACC, HIST>;
     static bool attr_done[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -280,6 +305,12 @@ li_status launch_impl(const CUtensorMap& map, const StreamArgs& args, int batch,
 li_status launch_stream_score_fp8(const CUtensorMap& map, const StreamArgs& args, int batch, int ntiles_max,
                                   cudaStream_t st) {
     return launch_impl<true, 1, 6, 4>(map, args, batch, ntiles_max, st);
+}
+
+li_status launch_stream_score_fp8_hist(const CUtensorMap& map, const StreamArgs& args, int batch, int ntiles_max,
+                                       cudaStream_t st) {
+    // five stages instead of six leave room for the histogram at two CTAs per SM
+    return launch_impl<true, 1, 5, 4, true>(map, args, batch, ntiles_max, st);
 }
 
 li_status launch_stream_score_bf16(const CUtensorMap& map, const StreamArgs& args, int batch, int ntiles_max,

@@ -87,57 +87,91 @@ __global__ void __launch_bounds__(128) simt_score_kernel(const SimtArgs a) {
 
 // ---------------------------------------------------------------------------
 // Decoder absorption: q~[b,j,c] = sum_e q[b,j,e] * W[j,e,c], fp32 accumulate,
-// one rounding to bf16.  Grid (heads, dc/64); the block's 256 threads cover
-// 64 columns as 32 bf16 pairs x 8 groups of e; W[j] is read once per block.
+// one rounding to bf16.  Grid (heads, dc/64): a block owns head j and 64
+// columns of W[j] (d rows x 128 bytes), read once for all requests.  Thread t
+// holds 8 columns (one 16-byte load) of rows e = t/8 + 32*i; every load of W is
+// issued before any arithmetic, so the block's slice of W is in flight at
+// once.  Partial sums over the 32 row groups are reduced with warp shuffles,
+// then across the 8 warps through shared memory.
 // ---------------------------------------------------------------------------
-constexpr int AB_BCH = 16;  // requests per pass over W
+constexpr int AB_BCH = 4;     // requests per pass over the registers of W
+constexpr int AB_MAXR = 8;    // rows per thread: d <= 256
 
 __global__ void __launch_bounds__(256) absorb_kernel(const __nv_bfloat16* __restrict__ q,
                                                      const __nv_bfloat16* __restrict__ W,
                                                      __nv_bfloat16* __restrict__ qt, int B, int H, int d, int dc) {
-    __shared__ __nv_bfloat16 qsh[AB_BCH][256];
-    __shared__ float2 red[8][AB_BCH][32];
+    __shared__ float qsh[AB_BCH][256];
+    __shared__ float red[8][AB_BCH][64];
     const int j = blockIdx.x;
     const int c0 = blockIdx.y * 64;
-    const int cp = threadIdx.x & 31;   // column pair
-    const int eg = threadIdx.x >> 5;   // e group
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int rg = t >> 3;   // row group 0..31
+    const int cg = t & 7;    // 8 columns c0+8cg .. c0+8cg+7
+    // the block's slice of W: all loads first
+    uint4 wv[AB_MAXR];
+#pragma unroll
+    for (int i = 0; i < AB_MAXR; ++i) {
+        const int e = rg + 32 * i;
+        wv[i] = e < d ? __ldg(reinterpret_cast<const uint4*>(W + ((size_t)j * d + e) * dc + c0) + cg)
+                      : make_uint4(0u, 0u, 0u, 0u);
+    }
     for (int b0 = 0; b0 < B; b0 += AB_BCH) {
         const int nb = min(AB_BCH, B - b0);
         __syncthreads();
-        for (int i = threadIdx.x; i < nb * d; i += blockDim.x) {
+        for (int i = t; i < AB_BCH * d; i += 256) {
             const int bb = i / d, e = i % d;
-            qsh[bb][e] = q[((size_t)(b0 + bb) * H + j) * d + e];
+            qsh[bb][e] = bb < nb ? __bfloat162float(q[((size_t)(b0 + bb) * H + j) * d + e]) : 0.f;
         }
         __syncthreads();
-        float2 acc[AB_BCH];
+        float acc[AB_BCH][8];
 #pragma unroll
-        for (int bb = 0; bb < AB_BCH; ++bb) acc[bb] = make_float2(0.f, 0.f);
-        for (int e = eg; e < d; e += 8) {
-            const __nv_bfloat162 wv =
-                *reinterpret_cast<const __nv_bfloat162*>(W + ((size_t)j * d + e) * dc + c0 + 2 * cp);
-            const float w0 = __low2float(wv), w1 = __high2float(wv);
+        for (int bb = 0; bb < AB_BCH; ++bb)
 #pragma unroll
-            for (int bb = 0; bb < AB_BCH; ++bb) {
-                if (bb < nb) {
-                    const float qv = __bfloat162float(qsh[bb][e]);
-                    acc[bb].x = fmaf(qv, w0, acc[bb].x);
-                    acc[bb].y = fmaf(qv, w1, acc[bb].y);
+            for (int x = 0; x < 8; ++x) acc[bb][x] = 0.f;
+#pragma unroll
+        for (int i = 0; i < AB_MAXR; ++i) {
+            const int e = rg + 32 * i;
+            if (e < d) {
+                const uint32_t wp[4] = {wv[i].x, wv[i].y, wv[i].z, wv[i].w};
+                float wf[8];
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    wf[2 * x] = __uint_as_float(wp[x] << 16);
+                    wf[2 * x + 1] = __uint_as_float(wp[x] & 0xffff0000u);
+                }
+#pragma unroll
+                for (int bb = 0; bb < AB_BCH; ++bb) {
+                    const float qv = qsh[bb][e];
+#pragma unroll
+                    for (int x = 0; x < 8; ++x) acc[bb][x] = fmaf(qv, wf[x], acc[bb][x]);
                 }
             }
         }
+        // reduce the 4 row groups of this warp (lanes that differ in bits 3, 4)
 #pragma unroll
-        for (int bb = 0; bb < AB_BCH; ++bb) red[eg][bb][cp] = acc[bb];
-        __syncthreads();
-        for (int i = threadIdx.x; i < nb * 32; i += blockDim.x) {
-            const int bb = i / 32, p = i % 32;
-            float2 s = red[0][bb][p];
+        for (int bb = 0; bb < AB_BCH; ++bb)
 #pragma unroll
-            for (int g = 1; g < 8; ++g) {
-                s.x += red[g][bb][p].x;
-                s.y += red[g][bb][p].y;
+            for (int x = 0; x < 8; ++x) {
+                float v = acc[bb][x];
+                v += __shfl_xor_sync(0xffffffffu, v, 8);
+                v += __shfl_xor_sync(0xffffffffu, v, 16);
+                acc[bb][x] = v;
             }
-            *reinterpret_cast<__nv_bfloat162*>(qt + ((size_t)(b0 + bb) * H + j) * dc + c0 + 2 * p) =
-                __floats2bfloat162_rn(s.x, s.y);
+        if (lane < 8) {
+#pragma unroll
+            for (int bb = 0; bb < AB_BCH; ++bb)
+#pragma unroll
+                for (int x = 0; x < 8; ++x) red[warp][bb][8 * cg + x] = acc[bb][x];
+        }
+        __syncthreads();
+        {
+            const int bb = t >> 6, c = t & 63;  // 256 threads = 4 requests x 64 columns
+            if (bb < nb) {
+                float sum = 0.f;
+#pragma unroll
+                for (int w = 0; w < 8; ++w) sum += red[w][bb][c];
+                qt[((size_t)(b0 + bb) * H + j) * dc + c0 + c] = __float2bfloat16_rn(sum);
+            }
         }
     }
 }

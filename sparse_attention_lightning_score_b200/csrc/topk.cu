@@ -31,6 +31,18 @@
 // the cluster once, then the slice is written in order, 4 keys per thread per
 // tile, positions from a block-wide scan.  No output depends on the order of
 // any atomic operation.
+//
+// With a histogram from the decode scorer (HIST): its LI_HIST_BITS-bit digit
+// is the first pass, found by one block-wide scan in every CTA with no cluster
+// merge.  The keys in the k-th key's bin (the candidates, about 3-5% of a row
+// of real scores) are appended to a list per CTA; one cluster exchange gives
+// every CTA the whole row's list, and the remaining 21 bits are selected from
+// it locally (two passes, no cluster barrier).  The exchange also checks the
+// histogram against the keys (the counts above and in the bin must agree);
+// if they do not, or the bin holds more candidates than a CTA can keep, the
+// plain passes run instead, so the result never depends on the histogram.
+// The histogram is left all zero for the next step.
+#include <algorithm>
 #include <cooperative_groups.h>
 
 #include "li_common.cuh"
@@ -45,13 +57,6 @@ namespace {
 constexpr int TK_SMEM_ROW = 40960;  // longest slice held by one CTA (160 KB of keys)
 constexpr int TK_MAX_CS = 8;        // largest cluster
 constexpr int TK_SLICE = 4096;      // target slice of a row per cluster CTA
-
-__device__ __forceinline__ uint32_t order_key(float f) {
-    if (f != f) return 0u;  // NaN: the only key mapped to 0, below -inf (0x007FFFFF)
-    uint32_t u = __float_as_uint(f);
-    if (f == 0.f) u = 0u;   // fold -0.0 onto +0.0
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
 
 __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v, int lane) {
 #pragma unroll
@@ -96,6 +101,42 @@ __device__ __forceinline__ const uint32_t* cl_peer(uint32_t* p, int rank) {
 // Kernel shape: NT threads, DBITS-bit digits (11 for a row held by one CTA:
 // three passes, no merge; 8 for a row split over a cluster: up to four
 // passes, but each cluster merge moves 256 bins instead of 2048).
+// Digit of the krem-th largest key from a histogram h[NB] indexed by digit:
+// bc[0] = digit, bc[1] = keys in higher digits, bc[2] = keys in that digit,
+// bc[3] = total count.  Ends with a block-wide barrier; every thread may read
+// bc afterwards.  (0, 0, 0) when the histogram holds fewer than krem keys.
+template <int NT, int NB>
+__device__ __forceinline__ void find_digit(const uint32_t* h, int krem, uint32_t* wsum, uint32_t* bc) {
+    constexpr int OW = NB < NT ? NB : NT;
+    constexpr int BPT = NB / OW;
+    uint32_t tot[BPT];
+    uint32_t s = 0u;
+    const bool own = threadIdx.x < OW;
+#pragma unroll
+    for (int i = 0; i < BPT; ++i) {
+        tot[i] = own ? h[NB - 1 - (BPT * threadIdx.x + i)] : 0u;
+        s += tot[i];
+    }
+    if (threadIdx.x == 0) bc[0] = bc[1] = bc[2] = 0u;
+    uint32_t total;
+    const uint32_t incl = block_scan1<NT / 32>(s, wsum, &total);
+    const uint32_t excl = incl - s;
+    if (own && excl < (uint32_t)krem && incl >= (uint32_t)krem) {
+        uint32_t run = excl;
+#pragma unroll
+        for (int i = 0; i < BPT; ++i) {
+            if (run < (uint32_t)krem && run + tot[i] >= (uint32_t)krem) {
+                bc[0] = (uint32_t)(NB - 1 - (BPT * threadIdx.x + i));
+                bc[1] = run;
+                bc[2] = tot[i];
+            }
+            run += tot[i];
+        }
+    }
+    if (threadIdx.x == 0) bc[3] = total;
+    __syncthreads();
+}
+
 template <int NT, bool CLUSTER>
 struct TopkShape {
     static constexpr int WARPS = NT / 32;
@@ -111,6 +152,9 @@ struct TopkShape {
     static size_t smem(int chunk) {
         return (size_t)((chunk + 3) & ~3) * 4 + (size_t)NCOPY * BINS * 4 + (CLUSTER ? 2 * BINS * 4 : 0);
     }
+    // with a histogram: this CTA's candidate list and (cluster) the row's gathered list
+    static size_t smem_hist(int chunk, int cap) { return smem(chunk) + (size_t)cap * 4 * (CLUSTER ? 2 : 1); }
+    static_assert(NCOPY * BINS >= LI_HIST_BINS, "the histogram copies hold the scorer's histogram");
     __device__ static int shift(int p) { return 32 - DBITS * (p + 1) > 0 ? 32 - DBITS * (p + 1) : 0; }
     __device__ static uint32_t digits(int p) {
         const int lo = shift(p), hi = 32 - DBITS * p;  // bits [lo, hi)
@@ -120,7 +164,7 @@ struct TopkShape {
 
 // Thread t < OWNERS owns the BPT contiguous bins BINS-BPT(t+1) .. BINS-BPT*t-1
 // (descending positions BPT*t .. BPT*t+BPT-1).
-template <int NT, bool CLUSTER>
+template <int NT, bool CLUSTER, bool HIST>
 __global__ void __launch_bounds__(NT) topk_kernel(const TopkArgs a, int row0, int chunk) {
     using S = TopkShape<NT, CLUSTER>;
     constexpr int BPT = S::BPT, NW = S::WARPS, NCOPY = S::NCOPY, BINS = S::BINS;
@@ -129,9 +173,13 @@ __global__ void __launch_bounds__(NT) topk_kernel(const TopkArgs a, int row0, in
     uint32_t* keys = reinterpret_cast<uint32_t*>(tk_dyn);
     uint32_t* hcopy = keys + ((chunk + 3) & ~3);     // [NCOPY][BINS]
     uint32_t* pub = hcopy + NCOPY * BINS;            // [2][BINS], cluster only
+    uint32_t* cand = pub + (CLUSTER ? 2 * BINS : 0); // HIST: this CTA's candidate keys [cand_cap]
+    uint32_t* gath = CLUSTER ? cand + a.cand_cap : cand;  // HIST: the row's candidate keys [cand_cap]
     __shared__ uint32_t wsum[2][32];
     __shared__ uint32_t bc[4];
     __shared__ uint32_t xch[2];
+    __shared__ uint32_t xcand[2];                    // HIST: candidates and keys above the bin, this CTA
+    __shared__ uint32_t coff[TK_MAX_CS + 1];         // HIST: candidate list offsets by cluster rank
 
     pdl_trigger();
     pdl_wait();  // the scores come from the previous kernel of the stream
@@ -151,8 +199,13 @@ __global__ void __launch_bounds__(NT) topk_kernel(const TopkArgs a, int row0, in
     float* oval = a.vals ? a.vals + (size_t)r * k : nullptr;
     const float* srow = a.scores + (size_t)r * a.ld;
     const int32_t* mrow = a.map ? a.map + (size_t)(r % a.map_rows) * a.map_ld : nullptr;
+    uint32_t* hrow = HIST ? a.hist + (size_t)r * LI_HIST_BINS : nullptr;
 
     if (n <= k) {  // every score is selected; the branch is uniform over the cluster
+        if constexpr (HIST) {
+            if (c == 0)
+                for (int i = threadIdx.x; i < LI_HIST_BINS; i += NT) hrow[i] = 0u;
+        }
         for (int i = threadIdx.x; i < cnt; i += NT) {
             const int p = base + i;
             oidx[p] = mrow ? __ldg(mrow + p) : p;
@@ -172,17 +225,123 @@ __global__ void __launch_bounds__(NT) topk_kernel(const TopkArgs a, int row0, in
         const float4 v = __ldg(s4 + i);
         tk_dyn[i] = make_uint4(order_key(v.x), order_key(v.y), order_key(v.z), order_key(v.w));
     }
-    for (int i = threadIdx.x; i < NCOPY * BINS; i += NT) hcopy[i] = 0u;
+    if constexpr (HIST) {
+        const uint4* h4 = reinterpret_cast<const uint4*>(hrow);
+        for (int i = threadIdx.x; i < LI_HIST_BINS / 4; i += NT) reinterpret_cast<uint4*>(hcopy)[i] = __ldcg(h4 + i);
+        if (threadIdx.x == 0) xcand[0] = xcand[1] = 0u;
+    } else {
+        for (int i = threadIdx.x; i < NCOPY * BINS; i += NT) hcopy[i] = 0u;
+    }
     __syncthreads();
 
-    // ---- radix select, most significant digit first
     uint32_t prefix = 0u, mask = 0u;
     int krem = k;
     bool ties = true;
+    bool selected = false;
+    if constexpr (HIST) {
+        // ---- first digit from the scorer's histogram (the same in every CTA of the cluster)
+        find_digit<NT, LI_HIST_BINS>(hcopy, krem, wsum[0], bc);
+        const uint32_t b1 = bc[0], above_h = bc[1], inbin_h = bc[2], total_h = bc[3];
+        if (total_h != (uint32_t)n && c == 0 && threadIdx.x == 0) record_error(a.err, ERRBIT_BOUNDS);
+        if (total_h == (uint32_t)n && inbin_h <= (uint32_t)a.cand_cap) {
+            // ---- this slice's candidates (keys in bin b1) and its count of keys above the bin
+            uint32_t my_above = 0u;
+            for (int i = threadIdx.x; i < ((cnt + 31) & ~31); i += NT) {
+                const uint32_t kk = i < cnt ? keys[i] : 0u;
+                const uint32_t d = kk >> LI_HIST_SHIFT;
+                const bool is_c = i < cnt && d == b1;
+                my_above += (i < cnt && d > b1) ? 1u : 0u;
+                const uint32_t bal = __ballot_sync(0xffffffffu, is_c);
+                if (bal == 0u) continue;
+                uint32_t slot = 0u;
+                if (lane == 0) slot = atomicAdd(&xcand[0], (uint32_t)__popc(bal));
+                slot = __shfl_sync(0xffffffffu, slot, 0) + (uint32_t)__popc(bal & ((1u << lane) - 1u));
+                if (is_c && slot < (uint32_t)a.cand_cap) cand[slot] = kk;
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) my_above += __shfl_xor_sync(0xffffffffu, my_above, o);
+            if (lane == 0 && my_above) atomicAdd(&xcand[1], my_above);
+            uint32_t ntot, above_sum;
+            if constexpr (CLUSTER) {
+                cl_sync<true>();
+                // gather every CTA's candidates, in rank order, into gath
+                if (warp == 0) {
+                    uint32_t cq = 0u, aq = 0u;
+                    if (lane < CS) {
+                        const uint32_t* px = cl_peer<true>(xcand, lane);
+                        cq = px[0];
+                        aq = px[1];
+                    }
+                    const bool over = __ballot_sync(0xffffffffu, cq > (uint32_t)a.cand_cap) != 0u;
+                    cq = min(cq, (uint32_t)a.cand_cap);
+                    const uint32_t incl = warp_incl_scan(cq, lane);
+                    const uint32_t sum = __shfl_sync(0xffffffffu, incl, 31);
+                    uint32_t as = aq;
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) as += __shfl_xor_sync(0xffffffffu, as, o);
+                    if (lane < CS) coff[lane + 1] = incl;
+                    if (lane == 0) {
+                        coff[0] = 0u;
+                        bc[0] = over ? (uint32_t)a.cand_cap + 1u : sum;  // bc is free again: broadcast through it
+                        bc[1] = as;
+                    }
+                }
+                __syncthreads();
+                ntot = bc[0];
+                above_sum = bc[1];
+                if (ntot <= (uint32_t)a.cand_cap) {
+#pragma unroll 4
+                    for (int j = threadIdx.x; j < (int)ntot; j += NT) {
+                        int q = 0;
+#pragma unroll
+                        for (int t = 1; t < TK_MAX_CS; ++t) q += (t < CS && (uint32_t)j >= coff[t]) ? 1 : 0;
+                        gath[j] = cl_peer<true>(cand, q)[j - (int)coff[q]];
+                    }
+                }
+            } else {
+                __syncthreads();
+                ntot = xcand[0];
+                above_sum = xcand[1];
+            }
+            __syncthreads();
+            if (ntot == inbin_h && above_sum == above_h) {
+                // ---- the remaining 21 bits, from the candidates alone: 11 then 10 bits
+                krem -= (int)above_h;
+                prefix = b1 << LI_HIST_SHIFT;
+                mask = ~0u << LI_HIST_SHIFT;
+                ties = (int)inbin_h != krem;
+                for (int lp = 0; ties && lp < 2; ++lp) {
+                    const int sh = lp == 0 ? 10 : 0;
+                    const uint32_t dm = lp == 0 ? 0x7ffu : 0x3ffu;
+                    for (int i = threadIdx.x; i < LI_HIST_BINS; i += NT) hcopy[i] = 0u;
+                    __syncthreads();
+                    for (int i = threadIdx.x; i < (int)ntot; i += NT) {
+                        const uint32_t kk = gath[i];
+                        if ((kk & mask) == prefix) atomicAdd(&hcopy[(kk >> sh) & dm], 1u);
+                    }
+                    __syncthreads();
+                    find_digit<NT, LI_HIST_BINS>(hcopy, krem, wsum[lp & 1], bc);
+                    krem -= (int)bc[1];
+                    prefix |= bc[0] << sh;
+                    mask |= dm << sh;
+                    if ((int)bc[2] == krem) ties = false;
+                }
+                selected = true;
+            } else if (c == 0 && threadIdx.x == 0) {
+                record_error(a.err, ERRBIT_BOUNDS);  // the histogram does not describe these keys
+            }
+        }
+        if (!selected) {
+            for (int i = threadIdx.x; i < NCOPY * BINS; i += NT) hcopy[i] = 0u;
+            __syncthreads();
+        }
+    }
+
+    // ---- radix select, most significant digit first
     const bool owner = threadIdx.x < S::OWNERS;
     const int b0 = BINS - BPT * (threadIdx.x + 1);  // an owner's bins b0 .. b0+BPT-1
     uint32_t* hmine = hcopy + (warp % NCOPY) * BINS;
-    for (int pass = 0; pass < S::PASSES; ++pass) {
+    for (int pass = 0; !selected && pass < S::PASSES; ++pass) {
         const int shift = S::shift(pass);
         const uint32_t dm = S::digits(pass);
         for (int i = threadIdx.x; i < ((cnt + 31) & ~31); i += NT) {
@@ -339,21 +498,40 @@ __global__ void __launch_bounds__(NT) topk_kernel(const TopkArgs a, int row0, in
         carry_eq += (int)(ttot & 0xffffu);
     }
     if constexpr (CLUSTER) asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+    if constexpr (HIST) {
+        // every CTA of the cluster has read the histogram (before the first cluster barrier)
+        if (c == 0) {
+            uint4* h4 = reinterpret_cast<uint4*>(hrow);
+            for (int i = threadIdx.x; i < LI_HIST_BINS / 4; i += NT) h4[i] = make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
 }
 
-template <int NT, bool CLUSTER>
+constexpr int TK_SMEM_BUDGET = 220 * 1024;  // dynamic shared memory a top-k CTA may take
+constexpr int TK_CAND_MAX = 8192;            // candidate keys per list (HIST)
+
+template <int NT, bool CLUSTER, bool HIST>
 cudaError_t launch_one(const TopkArgs& a, int row0, int nr, int cs, int chunk, cudaStream_t st) {
     using S = TopkShape<NT, CLUSTER>;
+    auto kern = topk_kernel<NT, CLUSTER, HIST>;
     static bool attr_done[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && !attr_done[dev]) {
-        cudaFuncSetAttribute(topk_kernel<NT, CLUSTER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)S::smem(TK_SMEM_ROW));
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TK_SMEM_BUDGET);
         attr_done[dev] = true;
     }
-    return launch_pdl(topk_kernel<NT, CLUSTER>, dim3(CLUSTER ? cs : 1, nr), dim3(NT), S::smem(chunk), st,
-                      CLUSTER ? cs : 1, a, row0, chunk);
+    TopkArgs b = a;
+    size_t smem = S::smem(chunk);
+    if constexpr (HIST) {
+        // candidate lists take what the slice leaves; below 256 keys the plain passes always run
+        const long long room = ((long long)TK_SMEM_BUDGET - (long long)smem) / (CLUSTER ? 8 : 4);
+        int cap = (int)std::min<long long>(TK_CAND_MAX, std::max<long long>(room, 0)) & ~3;
+        if (cap < 256) cap = 0;
+        b.cand_cap = cap;
+        smem = S::smem_hist(chunk, cap);
+    }
+    return launch_pdl(kern, dim3(CLUSTER ? cs : 1, nr), dim3(NT), smem, st, CLUSTER ? cs : 1, b, row0, chunk);
 }
 
 }  // namespace
@@ -375,9 +553,15 @@ li_status launch_topk(const TopkArgs& a, cudaStream_t st) {
     for (int row0 = 0; row0 < a.rows; row0 += 65535) {
         const int nr = min(65535, a.rows - row0);
         cudaError_t e;
-        if (cs == 1) e = small ? launch_one<256, false>(a, row0, nr, cs, chunk, st)
-                               : launch_one<1024, false>(a, row0, nr, cs, chunk, st);
-        else e = launch_one<512, true>(a, row0, nr, cs, chunk, st);
+        if (a.hist) {
+            if (cs == 1) e = small ? launch_one<256, false, true>(a, row0, nr, cs, chunk, st)
+                                   : launch_one<1024, false, true>(a, row0, nr, cs, chunk, st);
+            else e = launch_one<512, true, true>(a, row0, nr, cs, chunk, st);
+        } else {
+            if (cs == 1) e = small ? launch_one<256, false, false>(a, row0, nr, cs, chunk, st)
+                                   : launch_one<1024, false, false>(a, row0, nr, cs, chunk, st);
+            else e = launch_one<512, true, false>(a, row0, nr, cs, chunk, st);
+        }
         if (e != cudaSuccess) return host_check_launch();
         const li_status s = host_check_launch();
         if (s != LI_OK) return s;

@@ -7,7 +7,7 @@ decode step in SGLang's decode graph).  ``DecodeIndexer`` does the same with
 the li kernels: at construction it allocates device buffers and pinned host
 buffers once and captures
 
-    H2D copy of (q, w)  ->  li_index_score  ->  li_topk  ->  D2H copy of the indices
+    H2D copy of (q, w)  ->  li_decode_select (score + top-k)  ->  D2H copy of the indices
 
 as one CUDA graph; each ``step()`` writes the host inputs and replays it.
 Every kernel in the graph is an li kernel; torch only provides the buffers,
@@ -49,6 +49,7 @@ class DecodeIndexer:
         self.w_host = self.in_host[qbytes:].view(torch.float32).view(B, heads)
         self.scores = torch.empty((B, (L + 3) // 4 * 4), dtype=torch.float32, device=dev)
         self.idx_dev = torch.empty((B, k), dtype=torch.int32, device=dev)
+        self.ws = api.li_decode_select_workspace(B, dev)
         self.idx_host = torch.empty((B, k), dtype=torch.int32).pin_memory()
         self._launch()  # warm-up: loads the module, sets kernel attributes, checks arguments
         torch.cuda.synchronize(dev)
@@ -58,8 +59,8 @@ class DecodeIndexer:
 
     def _launch(self):
         self.in_dev.copy_(self.in_host, non_blocking=True)
-        api.li_index_score(self.q_dev, self.w_dev, self.k8, self.ks, lens=self.lens, scores=self.scores)
-        api.li_topk(self.scores, self.k, lens=self.lens, max_len=self.L, idx=self.idx_dev)
+        api.li_decode_select(self.q_dev, self.w_dev, self.k8, self.ks, self.k, lens=self.lens, scores=self.scores,
+                             workspace=self.ws, idx=self.idx_dev)
         self.idx_host.copy_(self.idx_dev, non_blocking=True)
 
     def step(self, q: Optional[torch.Tensor] = None, w: Optional[torch.Tensor] = None, sync: bool = True):

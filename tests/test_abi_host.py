@@ -21,7 +21,7 @@ def declared_symbols():
 def test_header_declares_the_boundary():
     syms = declared_symbols()
     for name in ["li_absorb_query", "li_index_score", "li_topk", "li_latent_score", "li_hs_refine",
-                 "li_get_last_error", "li_quantize_query"]:
+                 "li_get_last_error", "li_quantize_query", "li_decode_select", "li_decode_select_workspace"]:
         assert name in syms
 
 
@@ -52,6 +52,35 @@ def test_invalid_arguments_rejected_on_host():
     assert lib.li_index_score(p, p, p, p, 100, None, p, 100, ctypes.byref(d), None, 0, None) == _lib.LI_ERR_INVALID_ARG
     assert lib.li_absorb_query(p, p, p, 1, 64, 128, 100, None) == _lib.LI_ERR_INVALID_ARG
     assert lib.li_hs_refine(p, 0, 10, p, 1, 8, p, p, 0, 64, 256, 4, p, p, 0, None) == _lib.LI_ERR_INVALID_ARG
+
+
+def test_decode_select_rejects_bad_arguments_on_host():
+    lib = _lib.load()
+    p = ctypes.c_void_p(256)
+    d = _lib.ScoreDesc(2, 64, 128, 100, 0, 0, _lib.LI_DTYPE_BF16, _lib.LI_DTYPE_E4M3)
+    ws = lib.li_decode_select_workspace(ctypes.byref(d))
+    assert ws == 2 * 2048 * 4
+
+    def call(desc, k_top=8, ld=100, wsb=ws, wsp=p, scores=p):
+        return lib.li_decode_select(p, p, p, p, 0, None, scores, ld, ctypes.byref(desc), k_top, p, None, wsp, wsb,
+                                    None)
+
+    assert call(d, k_top=0) == _lib.LI_ERR_INVALID_ARG                      # k out of range
+    assert call(d, k_top=_lib.LI_TOPK_MAX_LEN + 1) == _lib.LI_ERR_INVALID_ARG
+    assert call(d, wsb=ws - 4) == _lib.LI_ERR_INVALID_ARG                   # workspace too small
+    assert call(d, wsp=ctypes.c_void_p(272)) == _lib.LI_ERR_INVALID_ARG     # workspace not 256-byte aligned
+    assert call(d, wsp=None) == _lib.LI_ERR_INVALID_ARG
+    assert call(d, ld=102) == _lib.LI_ERR_INVALID_ARG                       # ld not a multiple of 4
+    assert call(d, ld=96) == _lib.LI_ERR_INVALID_ARG                        # ld below max_len
+    assert call(d, scores=ctypes.c_void_p(264)) == _lib.LI_ERR_INVALID_ARG  # scores not 16-byte aligned
+    c = _lib.ScoreDesc(2, 64, 128, 100, 1, 0, _lib.LI_DTYPE_BF16, _lib.LI_DTYPE_E4M3)
+    assert call(c) == _lib.LI_ERR_INVALID_ARG                               # causal is not a decode step
+    u = _lib.ScoreDesc(2, 32, 128, 100, 0, 0, _lib.LI_DTYPE_BF16, _lib.LI_DTYPE_E4M3)
+    assert call(u) == _lib.LI_ERR_UNSUPPORTED                               # only the tensor-core shape
+    f = _lib.ScoreDesc(2, 64, 128, 100, 0, 0, _lib.LI_DTYPE_F32, _lib.LI_DTYPE_F32)
+    assert call(f) == _lib.LI_ERR_UNSUPPORTED
+    z = _lib.ScoreDesc(0, 64, 128, 100, 0, 0, _lib.LI_DTYPE_BF16, _lib.LI_DTYPE_E4M3)
+    assert call(z) == _lib.LI_OK                                            # no rows: nothing to do
 
 
 def test_zero_sized_calls_are_no_ops():

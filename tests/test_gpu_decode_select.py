@@ -1,0 +1,127 @@
+"""GPU parity of the one-call decode step (li_decode_select).
+
+The call must return exactly what li_index_score followed by li_topk returns
+on the same inputs: scores bit for bit, selections and their values bit for
+bit.  Those two calls are pinned to the oracle elsewhere; one case here also
+goes to the oracle directly.  The histogram workspace must be all zero again
+after every call, and a workspace that was not zero must still give the exact
+result and raise LI_ERR_BOUNDS.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_attention_lightning_score_b200 import api, synth
+from sparse_attention_lightning_score_b200._lib import LI_ERR_BOUNDS, LI_OK
+from tests._checks import assert_scores_close, assert_topk_equivalent
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _np(t):
+    return t.detach().cpu().numpy()
+
+
+def _dev(case):
+    return case.q.to(DEV), case.w.to(DEV), case.k8.to(DEV), case.ks.to(DEV), case.lens.to(DEV)
+
+
+def _two_calls(q, w, k8, ks, lens, k_top):
+    L = k8.shape[-2]
+    sc = api.li_index_score(q, w, k8, ks, lens=lens)
+    idx, vals = api.li_topk(sc, k_top, lens=lens, max_len=L, with_values=True)
+    return sc, idx, vals
+
+
+def _assert_same(got, want, lens):
+    sc, idx, vals = got
+    sc_r, idx_r, vals_r = want
+    for b, n in enumerate(_np(lens).tolist()):
+        assert np.array_equal(_np(sc[b, :n]).view(np.uint32), _np(sc_r[b, :n]).view(np.uint32)), b
+    assert np.array_equal(_np(idx), _np(idx_r))
+    assert np.array_equal(_np(vals).view(np.uint32), _np(vals_r).view(np.uint32))
+
+
+@pytest.mark.parametrize("B,L,lens,k_top", [
+    (3, 1000, [1000, 517, 129], 64),
+    (5, 300, [0, 1, 127, 128, 300], 100),       # empty, single and ragged rows
+    (4, 5000, [5000, 2048, 2049, 0], 2048),     # rows at and just above k
+    (8, 32768, None, 2048),                     # the benchmarked decode step
+    (2, 131072, None, 2048),
+    (1, 262144, None, 2048),                    # longest row: more candidates than a CTA keeps
+    (3, 20000, None, 1),
+])
+def test_decode_select_matches_score_then_topk(B, L, lens, k_top):
+    case = synth.dsa_decode(B=B, L=L, seed=40 + B, lens=lens)
+    q, w, k8, ks, ln = _dev(case)
+    ws = api.li_decode_select_workspace(B, DEV)
+    got = api.li_decode_select(q, w, k8, ks, k_top, lens=ln, workspace=ws, with_values=True)
+    _assert_same(got, _two_calls(q, w, k8, ks, ln, k_top), ln)
+    assert api.li_get_last_error() == LI_OK
+    assert int(ws.count_nonzero()) == 0
+
+
+def test_decode_select_against_oracle():
+    case = synth.dsa_decode(B=4, L=3000, seed=23, lens=[3000, 2500, 100, 2049])
+    q8, sq, _ = oracle.quantize_query(case.q, case.w.numpy())
+    L = 3000
+    ref, mag = oracle.index_score(q8, oracle.E4M3, case.w, case.k8, oracle.E4M3, q_scale=sq, k_scale=case.ks,
+                                  k_batch_rows=L, L=L, lens=case.lens.numpy(), with_mag=True)
+    q, w, k8, ks, ln = _dev(case)
+    sc, idx = api.li_decode_select(q, w, k8, ks, 512, lens=ln)
+    assert_scores_close(_np(sc)[:, :L], ref, mag, 1e-2)
+    ridx, _ = oracle.topk(ref, 512, lens=case.lens.numpy())
+    assert_topk_equivalent(_np(idx), ridx, ref, 1e-2, n_valid=case.lens.numpy())
+    assert api.li_get_last_error() == LI_OK
+
+
+def test_decode_select_workspace_reused_across_steps():
+    ws = api.li_decode_select_workspace(4, DEV)
+    for seed in (1, 2, 3):
+        case = synth.dsa_decode(B=4, L=9000, seed=seed, lens=[9000, 7000, 3000, 2100])
+        q, w, k8, ks, ln = _dev(case)
+        got = api.li_decode_select(q, w, k8, ks, 2048, lens=ln, workspace=ws, with_values=True)
+        _assert_same(got, _two_calls(q, w, k8, ks, ln, 2048), ln)
+    assert api.li_get_last_error() == LI_OK
+    assert int(ws.count_nonzero()) == 0
+
+
+def test_decode_select_shared_cache_and_many_rows():
+    # 160 rows (more rows than SMs: one CTA per row) over one shared cache
+    case = synth.dsa_decode(B=1, L=6000, seed=9)
+    g = torch.Generator().manual_seed(9)
+    q = torch.randn(160, 64, 128, generator=g).to(torch.bfloat16).to(DEV)
+    w = (torch.randn(160, 64, generator=g) * 0.1).to(DEV)
+    k8, ks = case.k8[0].to(DEV), case.ks[0].to(DEV)
+    lens = torch.randint(0, 6001, (160,), generator=g, dtype=torch.int32).to(DEV)
+    got = api.li_decode_select(q, w, k8, ks, 1024, lens=lens, with_values=True)
+    _assert_same(got, _two_calls(q, w, k8, ks, lens, 1024), lens)
+    assert api.li_get_last_error() == LI_OK
+
+
+def test_decode_select_all_scores_equal():
+    # zero weights: every score is 0, one bin holds the whole row, ties go to the lowest positions
+    case = synth.dsa_decode(B=2, L=40000, seed=5)
+    q, _, k8, ks, ln = _dev(case)
+    w = torch.zeros(2, 64, device=DEV)
+    ws = api.li_decode_select_workspace(2, DEV)
+    sc, idx = api.li_decode_select(q, w, k8, ks, 2048, lens=ln, workspace=ws)
+    assert np.array_equal(_np(idx), np.tile(np.arange(2048, dtype=np.int32), (2, 1)))
+    assert api.li_get_last_error() == LI_OK
+    assert int(ws.count_nonzero()) == 0
+
+
+def test_decode_select_dirty_workspace_is_reported_and_healed():
+    case = synth.dsa_decode(B=3, L=12000, seed=6)
+    q, w, k8, ks, ln = _dev(case)
+    ws = api.li_decode_select_workspace(3, DEV)
+    ws.view(torch.int32)[::7] = 3  # counts that describe no row
+    got = api.li_decode_select(q, w, k8, ks, 2048, lens=ln, workspace=ws, with_values=True)
+    _assert_same(got, _two_calls(q, w, k8, ks, ln, 2048), ln)
+    assert api.li_get_last_error() == LI_ERR_BOUNDS
+    assert int(ws.count_nonzero()) == 0
+    got = api.li_decode_select(q, w, k8, ks, 2048, lens=ln, workspace=ws, with_values=True)
+    _assert_same(got, _two_calls(q, w, k8, ks, ln, 2048), ln)
+    assert api.li_get_last_error() == LI_OK
