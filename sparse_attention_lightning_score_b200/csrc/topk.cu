@@ -146,7 +146,6 @@ struct TopkShape {
     static constexpr int OWNERS = BINS < NT ? BINS : NT;  // threads that own bins
     static constexpr int BPT = BINS / OWNERS;              // bins per owner
     static constexpr int NCOPY = CLUSTER ? 8 : (NT >= 1024 ? 4 : 2);  // private histogram copies
-    static constexpr int TILE = NT * 4;                    // compaction tile (4 keys per thread)
     // dynamic shared memory: keys, NCOPY histogram copies, then (cluster) the
     // double-buffered merged histogram the peers read
     static size_t smem(int chunk) {
@@ -238,30 +237,49 @@ __global__ void __launch_bounds__(NT) topk_kernel(const TopkArgs a, int row0, in
     int krem = k;
     bool ties = true;
     bool selected = false;
+    uint32_t gt_before = 0u, eq_before = 0u;  // selected keys in lower-ranked CTAs: above T, at T
+    bool have_offsets = false;
     if constexpr (HIST) {
         // ---- first digit from the scorer's histogram (the same in every CTA of the cluster)
         find_digit<NT, LI_HIST_BINS>(hcopy, krem, wsum[0], bc);
         const uint32_t b1 = bc[0], above_h = bc[1], inbin_h = bc[2], total_h = bc[3];
         if (total_h != (uint32_t)n && c == 0 && threadIdx.x == 0) record_error(a.err, ERRBIT_BOUNDS);
         if (total_h == (uint32_t)n && inbin_h <= (uint32_t)a.cand_cap) {
-            // ---- this slice's candidates (keys in bin b1) and its count of keys above the bin
-            uint32_t my_above = 0u;
-            for (int i = threadIdx.x; i < ((cnt + 31) & ~31); i += NT) {
-                const uint32_t kk = i < cnt ? keys[i] : 0u;
-                const uint32_t d = kk >> LI_HIST_SHIFT;
-                const bool is_c = i < cnt && d == b1;
-                my_above += (i < cnt && d > b1) ? 1u : 0u;
-                const uint32_t bal = __ballot_sync(0xffffffffu, is_c);
-                if (bal == 0u) continue;
-                uint32_t slot = 0u;
-                if (lane == 0) slot = atomicAdd(&xcand[0], (uint32_t)__popc(bal));
-                slot = __shfl_sync(0xffffffffu, slot, 0) + (uint32_t)__popc(bal & ((1u << lane) - 1u));
-                if (is_c && slot < (uint32_t)a.cand_cap) cand[slot] = kk;
-            }
+            // ---- this slice's candidates (keys in bin b1, in position order) and its count of keys
+            // above the bin: eight consecutive keys per thread, offsets from one block-wide scan
+            uint32_t ncand = 0u, nabove = 0u;
+            for (int tb = 0, flip = 0; tb < cnt; tb += NT * 8, flip ^= 1) {
+                const int i0 = tb + threadIdx.x * 8;
+                uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
+                if (i0 < cnt) v0 = tk_dyn[i0 >> 2];
+                if (i0 + 4 < cnt) v1 = tk_dyn[(i0 >> 2) + 1];
+                const uint32_t kk[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                uint32_t cm = 0u, na = 0u;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) my_above += __shfl_xor_sync(0xffffffffu, my_above, o);
-            if (lane == 0 && my_above) atomicAdd(&xcand[1], my_above);
-            uint32_t ntot, above_sum;
+                for (int e = 0; e < 8; ++e) {
+                    const uint32_t d = kk[e] >> LI_HIST_SHIFT;
+                    const bool valid = i0 + e < cnt;
+                    cm |= (valid && d == b1) ? 1u << e : 0u;
+                    na += (valid && d > b1) ? 1u : 0u;
+                }
+                const uint32_t packed = (na << 16) | (uint32_t)__popc(cm);
+                uint32_t tot;
+                const uint32_t excl = block_scan1<NW>(packed, wsum[flip], &tot) - packed;
+                uint32_t slot = ncand + (excl & 0xffffu);
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    if (cm & (1u << e)) {
+                        if (slot < (uint32_t)a.cand_cap) cand[slot] = kk[e];
+                        ++slot;
+                    }
+                ncand += tot & 0xffffu;
+                nabove += tot >> 16;
+            }
+            if (threadIdx.x == 0) {
+                xcand[0] = ncand;
+                xcand[1] = nabove;
+            }
+            uint32_t ntot, above_sum, above_before = 0u, cand_before = 0u;
             if constexpr (CLUSTER) {
                 cl_sync<true>();
                 // gather every CTA's candidates, in rank order, into gath
@@ -279,16 +297,22 @@ __global__ void __launch_bounds__(NT) topk_kernel(const TopkArgs a, int row0, in
                     uint32_t as = aq;
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) as += __shfl_xor_sync(0xffffffffu, as, o);
+                    uint32_t ab = lane < c ? aq : 0u;  // keys above the bin in lower-ranked CTAs
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) ab += __shfl_xor_sync(0xffffffffu, ab, o);
                     if (lane < CS) coff[lane + 1] = incl;
                     if (lane == 0) {
                         coff[0] = 0u;
                         bc[0] = over ? (uint32_t)a.cand_cap + 1u : sum;  // bc is free again: broadcast through it
                         bc[1] = as;
+                        bc[2] = ab;
                     }
                 }
                 __syncthreads();
                 ntot = bc[0];
                 above_sum = bc[1];
+                above_before = bc[2];
+                cand_before = coff[c];
                 if (ntot <= (uint32_t)a.cand_cap) {
 #pragma unroll 4
                     for (int j = threadIdx.x; j < (int)ntot; j += NT) {
@@ -298,6 +322,9 @@ __global__ void __launch_bounds__(NT) topk_kernel(const TopkArgs a, int row0, in
                         gath[j] = cl_peer<true>(cand, q)[j - (int)coff[q]];
                     }
                 }
+                __syncthreads();
+                // this CTA reads no peer's shared memory from here on; peers may leave after the final wait
+                asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
             } else {
                 __syncthreads();
                 ntot = xcand[0];
@@ -327,8 +354,23 @@ __global__ void __launch_bounds__(NT) topk_kernel(const TopkArgs a, int row0, in
                     if ((int)bc[2] == krem) ties = false;
                 }
                 selected = true;
-            } else if (c == 0 && threadIdx.x == 0) {
-                record_error(a.err, ERRBIT_BOUNDS);  // the histogram does not describe these keys
+                // output offset: keys above the bin in lower ranks, plus their candidates above / at T
+                uint32_t my = 0u;
+                for (int j = threadIdx.x; j < (int)cand_before; j += NT) {
+                    const uint32_t kk = gath[j];
+                    if (ties ? kk > prefix : kk >= prefix) my += 1u << 16;
+                    else if (ties && kk == prefix) my += 1u;
+                }
+                uint32_t tot;
+                (void)block_scan1<NW>(my, wsum[0], &tot);
+                gt_before = above_before + (tot >> 16);
+                eq_before = tot & 0xffffu;
+                have_offsets = true;
+            } else {
+                if (c == 0 && threadIdx.x == 0) record_error(a.err, ERRBIT_BOUNDS);  // the histogram does not
+                                                                                       // describe these keys
+                // close the phase opened by the arrive above before the plain passes' own cluster barriers
+                if constexpr (CLUSTER) asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
             }
         }
         if (!selected) {
@@ -428,70 +470,90 @@ __global__ void __launch_bounds__(NT) topk_kernel(const TopkArgs a, int row0, in
     const uint32_t T = prefix;
 
     // ---- counts of this slice; with a cluster, exchanged for the CTA's output offset
-    uint32_t my = 0u;
-    for (int i = threadIdx.x; i < cnt; i += NT) {
-        const uint32_t kk = keys[i];
-        if (ties ? kk > T : kk >= T) my += 1u << 16;
-        else if (ties && kk == T) my += 1u;
-    }
-    uint32_t ctot;
-    (void)block_scan1<NW>(my, wsum[0], &ctot);  // per-thread counts < 2^16: slices <= 40960 keys
-    uint32_t gt_before = 0u, eq_before = 0u;
-    if constexpr (CLUSTER) {
-        if (threadIdx.x == 0) {
-            xch[0] = ctot >> 16;
-            xch[1] = ctot & 0xffffu;
+    // (the histogram path has its offsets already)
+    if (!have_offsets) {
+        uint32_t my = 0u;
+        for (int i = threadIdx.x; i < cnt; i += NT) {
+            const uint32_t kk = keys[i];
+            if (ties ? kk > T : kk >= T) my += 1u << 16;
+            else if (ties && kk == T) my += 1u;
         }
-        cl_sync<true>();
-        for (int q = 0; q < c; ++q) {
-            const uint32_t* px = cl_peer<true>(xch, q);
-            gt_before += px[0];
-            eq_before += px[1];
+        uint32_t ctot;
+        (void)block_scan1<NW>(my, wsum[0], &ctot);  // per-thread counts < 2^16: slices <= 40960 keys
+        if constexpr (CLUSTER) {
+            if (threadIdx.x == 0) {
+                xch[0] = ctot >> 16;
+                xch[1] = ctot & 0xffffu;
+            }
+            cl_sync<true>();
+            if (warp == 0) {  // lane q < c reads CTA q's counts; all peers at once
+                uint32_t g = 0u, q = 0u;
+                if (lane < c) {
+                    const uint32_t* px = cl_peer<true>(xch, lane);
+                    g = px[0];
+                    q = px[1];
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    g += __shfl_xor_sync(0xffffffffu, g, o);
+                    q += __shfl_xor_sync(0xffffffffu, q, o);
+                }
+                if (lane == 0) {
+                    bc[0] = g;
+                    bc[1] = q;
+                }
+            }
+            __syncthreads();
+            gt_before = bc[0];
+            eq_before = bc[1];
+            // peers read this CTA's shared memory no more; they may leave after the wait below
+            asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
         }
-        // peers read this CTA's shared memory no more; they may leave after the wait below
-        asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
     }
     const int quota = ties ? max(0, krem - (int)eq_before) : 0;
     const int out_base = (int)gt_before + (ties ? min((int)eq_before, krem) : 0);
 
-    // ---- ordered compaction of the slice in tiles of 4 keys per thread
+    // ---- ordered compaction of the slice: eight consecutive keys per thread, positions from a
+    // block-wide scan per NT * 8 keys
     int carry_gt = 0, carry_eq = 0;
-    int tile = 1;  // wsum[1] is free from here on; tiles alternate 1, 0, 1, ...
-    for (int tb = 0; tb < cnt; tb += S::TILE, tile ^= 1) {
-        const int i0 = tb + threadIdx.x * 4;
-        uint4 kv = make_uint4(0u, 0u, 0u, 0u);
-        if (i0 < cnt) kv = tk_dyn[i0 >> 2];
-        const uint32_t kk[4] = {kv.x, kv.y, kv.z, kv.w};
+    for (int tb = 0, flip = 1; tb < cnt; tb += NT * 8, flip ^= 1) {
+        const int i0 = tb + threadIdx.x * 8;
+        uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
+        if (i0 < cnt) v0 = tk_dyn[i0 >> 2];
+        if (i0 + 4 < cnt) v1 = tk_dyn[(i0 >> 2) + 1];
+        const uint32_t kk[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
         uint32_t gm = 0u, em = 0u;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
+        for (int e = 0; e < 8; ++e) {
             const bool valid = i0 + e < cnt;
             if (valid && (ties ? kk[e] > T : kk[e] >= T)) gm |= 1u << e;
             else if (valid && ties && kk[e] == T) em |= 1u << e;
         }
         const uint32_t packed = ((uint32_t)__popc(gm) << 16) | (uint32_t)__popc(em);
         uint32_t ttot;
-        const uint32_t excl = block_scan1<NW>(packed, wsum[tile], &ttot) - packed;
+        const uint32_t excl = block_scan1<NW>(packed, wsum[flip], &ttot) - packed;
         int gb = carry_gt + (int)(excl >> 16);
         int eb = carry_eq + (int)(excl & 0xffffu);
+        if (gm | em) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            int pos = -1;
-            if (gm & (1u << e)) {
-                pos = out_base + gb + min(eb, quota);
-                ++gb;
-            } else if (em & (1u << e)) {
-                if (eb < quota) pos = out_base + gb + eb;
-                ++eb;
-            }
-            if (pos >= k) {  // cannot happen when the counts agree; never write past the row
-                record_error(a.err, ERRBIT_BOUNDS);
-                pos = -1;
-            }
-            if (pos >= 0) {
-                const int p = base + i0 + e;
-                oidx[pos] = mrow ? __ldg(mrow + p) : p;
-                if (oval) oval[pos] = __ldg(srow + p);
+            for (int e = 0; e < 8; ++e) {
+                int pos = -1;
+                if (gm & (1u << e)) {
+                    pos = out_base + gb + min(eb, quota);
+                    ++gb;
+                } else if (em & (1u << e)) {
+                    if (eb < quota) pos = out_base + gb + eb;
+                    ++eb;
+                }
+                if (pos >= k) {  // cannot happen when the counts agree; never write past the row
+                    record_error(a.err, ERRBIT_BOUNDS);
+                    pos = -1;
+                }
+                if (pos >= 0) {
+                    const int p = base + i0 + e;
+                    oidx[pos] = mrow ? __ldg(mrow + p) : p;
+                    if (oval) oval[pos] = __ldg(srow + p);
+                }
             }
         }
         carry_gt += (int)(ttot >> 16);
