@@ -315,6 +315,24 @@ __device__ __forceinline__ float relu_dot32_x2(const uint32_t (&v)[32], const fl
     return (a0.x + a0.y) + (a1.x + a1.y);
 }
 
+// e4m3(x / sq) (round to nearest even, saturating) with the quotient rounded as
+// IEEE fp32 division rounds it, at the cost of one multiply in almost every
+// case.  With r the correctly rounded reciprocal of sq, y = x * r lies within
+// 2.5 ulp of the correctly rounded quotient q (each of the two roundings is a
+// relative error of at most 2^-24).  y and q then round to the same e4m3 value
+// unless an e4m3 rounding midpoint lies between them.  For |y| in e4m3's
+// normal range, those midpoints are the values whose 20 low mantissa bits are
+// 0x80000.  So only a product within 8 ulp of such a point, or outside
+// [2^-6, 512] (e4m3 subnormals, zero, an overflowed reciprocal, NaN), is
+// recomputed with the division.
+__device__ __forceinline__ uint32_t e4m3_quotient(float x, float sq, float r) {
+    float y = x * r;
+    const float ay = fabsf(y);
+    const uint32_t m = __float_as_uint(y) & 0xfffffu;
+    if (!(ay >= 0x1p-6f && ay <= 512.f) || (m - 0x7fff8u) <= 16u) y = __fdiv_rn(x, sq);
+    return __nv_cvt_float_to_fp8(y, __NV_SATFINITE, __NV_E4M3);
+}
+
 // Per-(row, head) e4m3 quantisation of one 128-element bf16 head vector held
 // as 4 consecutive elements per lane of a warp.  Returns the packed 4 bytes
 // of this lane and writes the head scale to *sq (all lanes).
@@ -327,10 +345,11 @@ __device__ __forceinline__ uint32_t quantize_head128(uint2 raw, float* sq_out) {
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     const float sq = m > 0.f ? __fdiv_rn(m, 448.f) : 1.f;
     *sq_out = sq;
-    const uint32_t b0 = __nv_cvt_float_to_fp8(__fdiv_rn(x0, sq), __NV_SATFINITE, __NV_E4M3);
-    const uint32_t b1 = __nv_cvt_float_to_fp8(__fdiv_rn(x1, sq), __NV_SATFINITE, __NV_E4M3);
-    const uint32_t b2 = __nv_cvt_float_to_fp8(__fdiv_rn(x2, sq), __NV_SATFINITE, __NV_E4M3);
-    const uint32_t b3 = __nv_cvt_float_to_fp8(__fdiv_rn(x3, sq), __NV_SATFINITE, __NV_E4M3);
+    const float r = __frcp_rn(sq);
+    const uint32_t b0 = e4m3_quotient(x0, sq, r);
+    const uint32_t b1 = e4m3_quotient(x1, sq, r);
+    const uint32_t b2 = e4m3_quotient(x2, sq, r);
+    const uint32_t b3 = e4m3_quotient(x3, sq, r);
     return b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
 }
 
@@ -353,13 +372,14 @@ __device__ __forceinline__ uint4 quantize_head128_g8(uint4 lo, uint4 hi, float* 
     for (int o = 4; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     const float sq = m > 0.f ? __fdiv_rn(m, 448.f) : 1.f;
     *sq_out = sq;
+    const float r = __frcp_rn(sq);
     uint32_t b[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const uint32_t b0 = __nv_cvt_float_to_fp8(__fdiv_rn(x[4 * i + 0], sq), __NV_SATFINITE, __NV_E4M3);
-        const uint32_t b1 = __nv_cvt_float_to_fp8(__fdiv_rn(x[4 * i + 1], sq), __NV_SATFINITE, __NV_E4M3);
-        const uint32_t b2 = __nv_cvt_float_to_fp8(__fdiv_rn(x[4 * i + 2], sq), __NV_SATFINITE, __NV_E4M3);
-        const uint32_t b3 = __nv_cvt_float_to_fp8(__fdiv_rn(x[4 * i + 3], sq), __NV_SATFINITE, __NV_E4M3);
+        const uint32_t b0 = e4m3_quotient(x[4 * i + 0], sq, r);
+        const uint32_t b1 = e4m3_quotient(x[4 * i + 1], sq, r);
+        const uint32_t b2 = e4m3_quotient(x[4 * i + 2], sq, r);
+        const uint32_t b3 = e4m3_quotient(x[4 * i + 3], sq, r);
         b[i] = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
     }
     return make_uint4(b[0], b[1], b[2], b[3]);

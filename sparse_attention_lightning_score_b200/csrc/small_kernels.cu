@@ -9,8 +9,8 @@ namespace {
 
 // ---------------------------------------------------------------------------
 // Query quantisation: one warp per (row, head).  Same per-(row, head) recipe
-// as the prologue of the FP8 scorer (absmax / 448 scale, IEEE division,
-// nearest-even saturating e4m3 conversion).
+// as the prologue of the FP8 scorer (absmax / 448 scale, the quotient rounded
+// as IEEE division rounds it, nearest-even saturating e4m3 conversion).
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) quantize_query_kernel(const __nv_bfloat16* __restrict__ q,
                                                              const float* __restrict__ w, long long nheads, int dim,
@@ -49,8 +49,8 @@ __global__ void __launch_bounds__(256) quantize_query_kernel(const __nv_bfloat16
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         s = m > 0.f ? __fdiv_rn(m, 448.f) : 1.f;
-        for (int e = lane; e < dim; e += 32)
-            q8[gw * dim + e] = __nv_cvt_float_to_fp8(__fdiv_rn(__bfloat162float(src[e]), s), __NV_SATFINITE, __NV_E4M3);
+        const float r = __frcp_rn(s);
+        for (int e = lane; e < dim; e += 32) q8[gw * dim + e] = (uint8_t)e4m3_quotient(__bfloat162float(src[e]), s, r);
     }
     if (lane == 0) {
         sq[gw] = s;

@@ -39,6 +39,51 @@ def test_quantize_query_bit_exact(R, H, d):
     assert np.array_equal(_np(we).view(np.uint32), we_o.view(np.uint32))
 
 
+def _near_midpoint_heads(n_heads, seed):
+    """bf16 heads [n_heads, 128] whose quotients x / (absmax / 448) land within 8 fp32 ulps of an e4m3
+    rounding midpoint (exact ties included): the hard cases of the quantiser's rounding.  Found by
+    brute force over bf16 pairs with numpy's IEEE fp32 division."""
+    A = ((np.arange(0x3d80, 0x4180, dtype=np.uint32) << 16).view(np.float32))
+    X = ((np.arange(0x3980, 0x4180, dtype=np.uint32) << 16).view(np.float32))
+    pairs = {}
+    for a in A:
+        sq = np.float32(a) / np.float32(448.0)
+        xs = X[X <= a]
+        qv = xs / sq
+        m = qv.view(np.uint32) & 0xFFFFF
+        near = (np.abs(m.astype(np.int64) - 0x80000) <= 8) & (qv >= 2.0 ** -6) & (qv <= 448)
+        if near.any():
+            pairs[float(a)] = xs[near]
+    rng = np.random.default_rng(seed)
+    keys = sorted(pairs)
+    heads = np.empty((n_heads, 128), np.float32)
+    for h in range(n_heads):
+        a = keys[rng.integers(len(keys))]
+        xs = pairs[a]
+        row = rng.choice(xs, 127) * rng.choice([-1.0, 1.0], 127).astype(np.float32)
+        heads[h, 0] = a * rng.choice([-1.0, 1.0])
+        heads[h, 1:] = row
+        rng.shuffle(heads[h])
+    return torch.from_numpy(heads).to(torch.bfloat16)
+
+
+def test_quantize_query_near_rounding_midpoints():
+    q = _near_midpoint_heads(4 * 64, seed=3).view(4, 64, 128)
+    w = torch.randn(4, 64, generator=torch.Generator().manual_seed(3))
+    q8_o, sq_o, we_o = oracle.quantize_query(q, w.numpy())
+    q8, sq, we = api.li_quantize_query(q.to(DEV), w.to(DEV))
+    assert np.array_equal(_np(q8), q8_o)
+    assert np.array_equal(_np(sq).view(np.uint32), sq_o.view(np.uint32))
+    # the decode scorer quantises in its prologue: same bytes, so the same scores as the
+    # oracle's quantised query within the FP8 tolerance
+    k = torch.randn(4, 300, 128, generator=torch.Generator().manual_seed(4))
+    k8, ks = synth.encode_e4m3_cache(k)
+    ref, mag = oracle.index_score(q8_o, oracle.E4M3, w, k8, oracle.E4M3, q_scale=sq_o, k_scale=ks,
+                                  k_batch_rows=300, L=300, with_mag=True)
+    sc = api.li_index_score(q.to(DEV), w.to(DEV), k8.to(DEV), ks.to(DEV))
+    assert_scores_close(_np(sc)[:, :300], ref, mag, 1e-2)
+
+
 # ---------------------------------------------------------------------------
 # tiny fp32 case: exact scalar path, tolerance 1e-4
 # ---------------------------------------------------------------------------
