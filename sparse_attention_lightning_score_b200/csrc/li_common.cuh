@@ -325,12 +325,23 @@ __device__ __forceinline__ float relu_dot32_x2(const uint32_t (&v)[32], const fl
 // 0x80000.  So only a product within 8 ulp of such a point, or outside
 // [2^-6, 512] (e4m3 subnormals, zero, an overflowed reciprocal, NaN), is
 // recomputed with the division.
-__device__ __forceinline__ uint32_t e4m3_quotient(float x, float sq, float r) {
+__device__ __forceinline__ float quotient_for_e4m3(float x, float sq, float r) {
     float y = x * r;
     const float ay = fabsf(y);
     const uint32_t m = __float_as_uint(y) & 0xfffffu;
     if (!(ay >= 0x1p-6f && ay <= 512.f) || (m - 0x7fff8u) <= 16u) y = __fdiv_rn(x, sq);
-    return __nv_cvt_float_to_fp8(y, __NV_SATFINITE, __NV_E4M3);
+    return y;
+}
+
+// Two fp32 values to e4m3 (nearest even, saturating to +-448): lo in the low byte, hi in the high byte.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+    uint16_t d;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t e4m3_quotient(float x, float sq, float r) {
+    return e4m3x2(quotient_for_e4m3(x, sq, r), 0.f) & 0xffu;
 }
 
 // Per-(row, head) e4m3 quantisation of one 128-element bf16 head vector held
@@ -346,11 +357,8 @@ __device__ __forceinline__ uint32_t quantize_head128(uint2 raw, float* sq_out) {
     const float sq = m > 0.f ? __fdiv_rn(m, 448.f) : 1.f;
     *sq_out = sq;
     const float r = __frcp_rn(sq);
-    const uint32_t b0 = e4m3_quotient(x0, sq, r);
-    const uint32_t b1 = e4m3_quotient(x1, sq, r);
-    const uint32_t b2 = e4m3_quotient(x2, sq, r);
-    const uint32_t b3 = e4m3_quotient(x3, sq, r);
-    return b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+    return e4m3x2(quotient_for_e4m3(x0, sq, r), quotient_for_e4m3(x1, sq, r)) |
+           (e4m3x2(quotient_for_e4m3(x2, sq, r), quotient_for_e4m3(x3, sq, r)) << 16);
 }
 
 // Same quantisation with 8 lanes per head: the lane holds 16 consecutive bf16
@@ -375,13 +383,9 @@ __device__ __forceinline__ uint4 quantize_head128_g8(uint4 lo, uint4 hi, float* 
     const float r = __frcp_rn(sq);
     uint32_t b[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t b0 = e4m3_quotient(x[4 * i + 0], sq, r);
-        const uint32_t b1 = e4m3_quotient(x[4 * i + 1], sq, r);
-        const uint32_t b2 = e4m3_quotient(x[4 * i + 2], sq, r);
-        const uint32_t b3 = e4m3_quotient(x[4 * i + 3], sq, r);
-        b[i] = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
-    }
+    for (int i = 0; i < 4; ++i)
+        b[i] = e4m3x2(quotient_for_e4m3(x[4 * i + 0], sq, r), quotient_for_e4m3(x[4 * i + 1], sq, r)) |
+               (e4m3x2(quotient_for_e4m3(x[4 * i + 2], sq, r), quotient_for_e4m3(x[4 * i + 3], sq, r)) << 16);
     return make_uint4(b[0], b[1], b[2], b[3]);
 }
 

@@ -107,6 +107,27 @@ __global__ void __launch_bounds__(StreamCfg<FP8, KBLK, STAGES, NACC, HIST>::THRE
 
     // everything above overlaps the previous kernel; inputs are read only after it completed
     pdl_wait();
+    // FP8: the prologue warps issue their query loads before the length is known, so that the two
+    // round trips overlap (the length decides only whether this CTA has any tile)
+    constexpr int QHPW = C::H / C::PRO_WARPS;  // heads per prologue warp
+    constexpr int QIT = QHPW / 4;              // four heads at a time, eight lanes per head
+    uint4 qraw[FP8 ? QIT : 1][2];
+    float qw[FP8 ? QIT : 1];
+    if constexpr (FP8) {
+        if (warp >= 2) {
+            const int ew = (threadIdx.x - 64) >> 5;
+            const int g8 = lane >> 3, l8 = lane & 7;
+            const __nv_bfloat16* q = reinterpret_cast<const __nv_bfloat16*>(a.q) + (size_t)b * C::H * 128;
+#pragma unroll
+            for (int i = 0; i < QIT; ++i) {
+                const int j = QHPW * ew + 4 * i + g8;
+                const uint4* src = reinterpret_cast<const uint4*>(q + (size_t)j * 128) + 2 * l8;
+                qraw[i][0] = __ldg(src);
+                qraw[i][1] = __ldg(src + 1);
+                qw[i] = __ldg(a.w + (size_t)b * C::H + j);
+            }
+        }
+    }
     int len_b = a.len ? __ldg(a.len + b) : a.max_len;
     if (len_b < 0 || len_b > a.max_len) {
         if (threadIdx.x == 0 && blockIdx.x == 0) record_error(a.err, ERRBIT_BOUNDS);
@@ -177,28 +198,15 @@ __global__ void __launch_bounds__(StreamCfg<FP8, KBLK, STAGES, NACC, HIST>::THRE
         const int ew = et >> 5;
         if constexpr (FP8) {
             // 8 heads per warp, four at a time (8 lanes per head, 16 elements per
-            // lane); all loads are issued before any is consumed
-            constexpr int HPW = C::H / C::PRO_WARPS;
-            constexpr int IT = HPW / 4;
+            // lane), from the loads issued above
             const int g8 = lane >> 3, l8 = lane & 7;
-            const __nv_bfloat16* q = reinterpret_cast<const __nv_bfloat16*>(a.q) + (size_t)b * C::H * 128;
-            uint4 raw[IT][2];
-            float wv[IT];
 #pragma unroll
-            for (int i = 0; i < IT; ++i) {
-                const int j = HPW * ew + 4 * i + g8;
-                const uint4* src = reinterpret_cast<const uint4*>(q + (size_t)j * 128) + 2 * l8;
-                raw[i][0] = __ldg(src);
-                raw[i][1] = __ldg(src + 1);
-                wv[i] = __ldg(a.w + (size_t)b * C::H + j);
-            }
-#pragma unroll
-            for (int i = 0; i < IT; ++i) {
-                const int j = HPW * ew + 4 * i + g8;
+            for (int i = 0; i < QIT; ++i) {
+                const int j = QHPW * ew + 4 * i + g8;
                 float sq;
-                const uint4 packed = quantize_head128_g8(raw[i][0], raw[i][1], &sq);
+                const uint4 packed = quantize_head128_g8(qraw[i][0], qraw[i][1], &sq);
                 *reinterpret_cast<uint4*>(qsm + sw128_offset(j, l8)) = packed;
-                if (l8 == 0) wsm[j] = wv[i] * sq;
+                if (l8 == 0) wsm[j] = qw[i] * sq;
             }
         } else {
             constexpr int CH = KBLK * 8;                // 16-byte chunks per query row

@@ -67,23 +67,26 @@ __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v, int lane) {
     return v;
 }
 
-// Block-wide inclusive scan with one __syncthreads.  wsum must not be reused
-// before every thread has passed the next block-wide barrier.
+// Block-wide inclusive scan with one __syncthreads: each warp scans its lanes,
+// then every warp scans the NW warp totals in parallel (lane l holds warp l's).
+// wsum must not be reused before every thread has passed the next block-wide
+// barrier.
 template <int NW>
 __device__ __forceinline__ uint32_t block_scan1(uint32_t v, uint32_t* wsum, uint32_t* total) {
+    static_assert(NW >= 1 && NW <= 32, "warps per block");
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const uint32_t incl = warp_incl_scan(v, lane);
     if (lane == 31) wsum[warp] = incl;
     __syncthreads();
-    uint32_t off = 0u, tot = 0u;
+    uint32_t x = lane < NW ? wsum[lane] : 0u;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) {
-        const uint32_t x = wsum[w];
-        off += w < warp ? x : 0u;
-        tot += x;
+    for (int o = 1; o < NW; o <<= 1) {
+        const uint32_t t = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += t;
     }
-    *total = tot;
-    return incl + off;
+    *total = __shfl_sync(0xffffffffu, x, NW - 1);
+    const uint32_t before = __shfl_sync(0xffffffffu, x, (warp + 31) & 31);  // warps 0 .. warp-1
+    return incl + (warp > 0 ? before : 0u);
 }
 
 template <bool CLUSTER>
@@ -217,19 +220,32 @@ __global__ void __launch_bounds__(NT) topk_kernel(const TopkArgs a, int row0, in
         return;
     }
 
-    // ---- load this CTA's slice (row start and slice start are 16-byte aligned)
-    const float4* s4 = reinterpret_cast<const float4*>(srow + base);
-    const int nvec = (cnt + 3) >> 2;
-    for (int i = threadIdx.x; i < nvec; i += NT) {
-        const float4 v = __ldg(s4 + i);
-        tk_dyn[i] = make_uint4(order_key(v.x), order_key(v.y), order_key(v.z), order_key(v.w));
-    }
+    // ---- load this CTA's slice (row start and slice start are 16-byte aligned), LU loads in
+    // flight per thread; the histogram's loads go out first
     if constexpr (HIST) {
         const uint4* h4 = reinterpret_cast<const uint4*>(hrow);
         for (int i = threadIdx.x; i < LI_HIST_BINS / 4; i += NT) reinterpret_cast<uint4*>(hcopy)[i] = __ldcg(h4 + i);
-        if (threadIdx.x == 0) xcand[0] = xcand[1] = 0u;
     } else {
         for (int i = threadIdx.x; i < NCOPY * BINS; i += NT) hcopy[i] = 0u;
+    }
+    {
+        constexpr int LU = 4;
+        const float4* s4 = reinterpret_cast<const float4*>(srow + base);
+        const int nvec = (cnt + 3) >> 2;
+        for (int i0 = threadIdx.x; i0 < nvec; i0 += NT * LU) {
+            float4 v[LU];
+#pragma unroll
+            for (int u = 0; u < LU; ++u) {
+                const int i = i0 + u * NT;
+                v[u] = i < nvec ? __ldg(s4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < LU; ++u) {
+                const int i = i0 + u * NT;
+                if (i < nvec)
+                    tk_dyn[i] = make_uint4(order_key(v[u].x), order_key(v[u].y), order_key(v[u].z), order_key(v[u].w));
+            }
+        }
     }
     __syncthreads();
 
