@@ -3,10 +3,10 @@
  *
  * The lightning indexer of DeepSeek Sparse Attention gives every visible cache
  * position s of a query token t one score and keeps the k highest-scoring
- * positions for that layer's sparse attention ("scores the whole cache and
- * keeps the k=2048 highest-scoring tokens", Multi-layer Indexer abstract;
- * "one score per visible position ... before top-k", IndexCache explainer,
- * Symbol Map).  The score computed here is
+ * positions for that layer's sparse attention (Multi-layer Indexer abstract:
+ * a scan over the whole cache, then the k = 2048 best tokens; IndexCache
+ * explainer, Symbol Map: each visible position gets one score, and top-k
+ * follows).  The score computed here is
  *
  *     I[t,s] = sum_j w[t,j] * ReLU(q[t,j,:] . k[s,:])        (j < H heads)
  *
@@ -106,9 +106,9 @@ typedef struct {
 /* Scores every visible cache position of every row:
  *     scores[r * scores_ld + s] = sk[s] * sum_j w_eff[r,j] * ReLU(q8[r,j,:] . k8[s,:])
  * which is I[r,s] of the header comment with q = q8*sq and k = k8*sk.
- * The scan runs over "the whole cache" of each row (Multi-layer Indexer
- * abstract); in prefill each token sees its prefix including its own position
- * ("scans the prefix", IndexCache explainer, Why This Exists).
+ * Each row's scan covers its entire cache (Multi-layer Indexer abstract).  In
+ * prefill each token sees its prefix, its own position included (IndexCache
+ * explainer, Why This Exists: the indexer runs over the prefix).
  *   q        [rows, heads, dim] (q_dtype)     w [rows, heads] fp32
  *   k        key rows of `dim` elements (k_dtype); request r's cache begins at row
  *            r * cache_batch_rows (0 = every row reads the same cache)
@@ -146,9 +146,9 @@ li_status li_topk(const float* scores, int64_t scores_ld, const int32_t* len, in
 /* ------------------------------------------------------------------------ */
 /* One decode step of the indexer: li_index_score in its decode form (causal
  * 0) followed by li_topk(k_top) on the same scores, with identical results.
- * The difference is internal.  The pages run the indexer as a full scan
- * followed by top-k ("one score per visible position ... before top-k",
- * IndexCache explainer, Symbol Map), and this call follows that order.  While
+ * The difference is internal.  The pages run the indexer as a full scan that
+ * scores every visible position, with top-k after it (IndexCache explainer,
+ * Symbol Map), and this call keeps that order.  While
  * writing each score, the scorer also counts it by the top 11 bits of the
  * selection's order key.  The top-k takes its first radix digit from those
  * counts instead of sweeping the row for it.
@@ -204,6 +204,13 @@ li_status li_topk_hist(const float* scores, int64_t scores_ld, const int32_t* le
 li_status li_absorb_query(const void* q_bf16, const void* w_dec_bf16, void* q_tilde_bf16, int batch, int heads,
                           int dim, int latent_dim, li_stream_t stream);
 
+/* li_absorb_query for `layers` layers of a group in one launch: layer l's query
+ * is at q_bf16 + l*batch*heads*dim, its decoder at w_dec_bf16 +
+ * l*heads*dim*latent_dim and its output at q_tilde_bf16 + l*batch*heads*latent_dim
+ * (elements).  Same arithmetic per layer; 0 <= layers <= 65535. */
+li_status li_absorb_query_layers(const void* q_bf16, const void* w_dec_bf16, void* q_tilde_bf16, int layers,
+                                 int batch, int heads, int dim, int latent_dim, li_stream_t stream);
+
 /* Scores the shared latent cache with absorbed queries:
  *     scores[b * scores_ld + s] = sum_j w[b,j] * ReLU(q~[b,j,:] . c[b,s,:])   for s < len[b]
  *   q_tilde [batch, heads, latent_dim] bf16     w [batch, heads] fp32
@@ -214,11 +221,20 @@ li_status li_latent_score(const void* q_tilde_bf16, const float* w, const void* 
                           const int32_t* len, float* scores, int64_t scores_ld, int batch, int heads, int latent_dim,
                           int max_len, li_stream_t stream);
 
+/* li_latent_score that also counts every score it writes into
+ * hist[b * 2048 + (key >> 21)], key being the score's order key as for
+ * li_decode_score_hist.  hist: [batch, 2048] uint32, 16-byte aligned and zero
+ * before the call.  li_topk_hist then selects from the same scores, for
+ * example the anchor's candidate set of hierarchical selection. */
+li_status li_latent_score_hist(const void* q_tilde_bf16, const float* w, const void* c_bf16,
+                               int64_t cache_batch_rows, const int32_t* len, float* scores, int64_t scores_ld,
+                               int batch, int heads, int latent_dim, int max_len, uint32_t* hist, li_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Hierarchical selection: followers refine the anchor's candidates         */
 /* ------------------------------------------------------------------------ */
-/* LatentIndex abstract: "followers independently refine a shared candidate
- * set proposed by the anchor".  For every follower f and request b, each
+/* LatentIndex abstract: the anchor proposes one candidate set, shared by its
+ * followers, and each follower refines it on its own.  For every follower f and request b, each
  * candidate latent row c[b, cand[b,i]] is gathered once and scored against all
  * followers' absorbed queries,
  *     I_f[b,i] = sum_j w[f,b,j] * ReLU(q~[f,b,j,:] . c[b, cand[b,i], :]),

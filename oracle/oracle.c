@@ -11,11 +11,11 @@
  *
  *     I[t,s] = sum_j w[t,j] * ReLU(q[t,j,:] . k[s,:])
  *
- * which the pages describe as "one score per visible position ... before
- * top-k" (IndexCache explainer, "Symbol Map") computed by an indexer that
- * "scores the whole cache and keeps the k=2048 highest-scoring tokens"
- * (Multi-layer Indexer abstract), a "low-rank bilinear interaction" like an
- * attention logit (Multi-layer Indexer podcast page, deep dive).
+ * In the pages each visible position receives one such score and top-k
+ * follows (IndexCache explainer, Symbol Map); the indexer scans the whole
+ * cache and keeps the 2048 best tokens (Multi-layer Indexer abstract); and
+ * the score is a low-rank bilinear form of query and key, of the same kind
+ * as an attention logit (Multi-layer Indexer podcast page, deep dive).
  *
  * Arithmetic: every score is accumulated in double.  The one place where the
  * oracle works in fp32 is the query quantiser, whose output is an integer code
@@ -53,7 +53,7 @@ double orc_e4m3_decode(uint8_t b)
 }
 
 /* Round an fp32 value to the nearest e4m3 value, ties to even mantissa, and
- * clamp finite values beyond 448 to +-448 ("saturate to finite").  Written
+ * clamp finite values beyond 448 to +-448 (saturation to the largest finite).  Written
  * from the format definition above: find the binade, divide by the grid step
  * of that binade (a power of two, so exact), round with nearbyint (the default
  * rounding mode is round-to-nearest-even), then re-assemble the fields. */
@@ -149,11 +149,11 @@ typedef struct {
 } orc_score_args;
 
 /* Number of cache positions row r may see.  Decode: the whole cache of that
- * request, i.e. its first len[r] positions ("scores the whole cache",
- * Multi-layer Indexer abstract).  Causal prefill: query token t sees the
- * prefix up to and including its own position ("scans the prefix",
- * IndexCache explainer, "Why This Exists"; inclusive is this oracle's
- * reading). */
+ * request, i.e. its first len[r] positions (Multi-layer Indexer abstract:
+ * the scan covers the entire cache).  Causal prefill: query token t sees the
+ * prefix up to and including its own position (IndexCache explainer, Why This
+ * Exists: in prefill the indexer runs over the prefix; inclusive is this
+ * oracle's reading). */
 static int visible_len(const orc_score_args* a, int r)
 {
     long long n;
@@ -281,9 +281,9 @@ static int cmp_pos(const void* pa, const void* pb)
     return a < b ? -1 : (a > b ? 1 : 0);
 }
 
-/* Keep the k highest-scoring of the n values (IndexCache explainer, "Symbol
- * Map": the selected set T_t holds k token positions; Multi-layer Indexer
- * abstract: "keeps the k=2048 highest-scoring tokens").  Full sort by rank,
+/* Keep the k highest-scoring of the n values (IndexCache explainer, Symbol
+ * Map: the selected set T_t holds k token positions; Multi-layer Indexer
+ * abstract: the 2048 best-scoring tokens are kept).  Full sort by rank,
  * take min(k, n), report them in ascending position order, pad with -1.
  * ``pos`` (optional) maps slot i to the reported position. */
 static void topk_one(const double* v, int n, const int* pos, int k, int* idx, double* vals)
@@ -380,7 +380,7 @@ void orc_latent_score_rebuilt(const uint16_t* q, const float* w, const uint16_t*
 /* ------------------------------------------------------------------------ */
 
 /* LatentIndex abstract: the anchor proposes a shared candidate set and each
- * follower "independently refines" it.  Reading: a follower re-scores only
+ * follower refines it on its own.  Reading: a follower re-scores only
  * the candidate latent rows (cand[b, i] >= 0; negative entries are padding)
  * with its own absorbed query and keeps its k best by (score desc, cache
  * position asc); it never adds a position outside the candidates.  Output:

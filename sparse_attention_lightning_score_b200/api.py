@@ -226,6 +226,39 @@ def li_absorb_query(q: torch.Tensor, w_dec: torch.Tensor, out: Optional[torch.Te
     return out
 
 
+def li_absorb_query_layers(q: torch.Tensor, w_dec: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None):
+    """q bf16 [G,B,H,d], W_dec bf16 [G,H,d,dc] -> q~ bf16 [G,B,H,dc], all G layers in one launch."""
+    _need(q, "q", torch.bfloat16)
+    _need(w_dec, "w_dec", torch.bfloat16)
+    G, B, H, d = q.shape
+    dc = w_dec.shape[3]
+    if out is None:
+        out = torch.empty((G, B, H, dc), dtype=torch.bfloat16, device=q.device)
+    st = _lib.load().li_absorb_query_layers(_ptr(q), _ptr(w_dec), _ptr(out), G, B, H, d, dc, _stream(stream))
+    _lib.check("li_absorb_query_layers", st)
+    return out
+
+
+def li_latent_score_hist(q_tilde: torch.Tensor, w: torch.Tensor, c: torch.Tensor, hist: torch.Tensor, *,
+                         lens: Optional[torch.Tensor] = None, scores: Optional[torch.Tensor] = None, stream=None):
+    """li_latent_score that also adds its scores' first-digit counts to `hist` (zeroed [B, 2048] uint32
+    buffer, e.g. from li_decode_select_workspace) for li_topk_hist."""
+    _need(q_tilde, "q_tilde", torch.bfloat16)
+    _need(w, "w", torch.float32)
+    _need(c, "c", torch.bfloat16)
+    B, H, dc = q_tilde.shape
+    L = c.shape[-2]
+    batch_rows = c.shape[1] if c.dim() == 3 else 0
+    if lens is not None:
+        _need(lens, "lens", torch.int32)
+    if scores is None:
+        scores = torch.empty((B, _round4(L)), dtype=torch.float32, device=c.device)
+    st = _lib.load().li_latent_score_hist(_ptr(q_tilde), _ptr(w), _ptr(c), batch_rows, _ptr(lens), _ptr(scores),
+                                          scores.stride(0), B, H, dc, L, _ptr(hist), _stream(stream))
+    _lib.check("li_latent_score_hist", st)
+    return scores
+
+
 def li_latent_score(q_tilde: torch.Tensor, w: torch.Tensor, c: torch.Tensor, *, lens: Optional[torch.Tensor] = None,
                     scores: Optional[torch.Tensor] = None, stream=None):
     """q~ bf16 [B,H,dc], w fp32 [B,H], c bf16 [B,L,dc] (or shared [L,dc]) -> scores fp32 [B, round4(L)]."""

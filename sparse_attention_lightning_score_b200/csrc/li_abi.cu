@@ -302,27 +302,33 @@ li_status li_decode_select(const void* q, const float* w, const void* k, const f
     return li_topk_hist(scores, d.max_len > 0 ? scores_ld : 4, len, d.rows, d.max_len, k_top, idx, vals, hist, stream);
 }
 
-li_status li_absorb_query(const void* q_bf16, const void* w_dec_bf16, void* q_tilde_bf16, int batch, int heads,
-                          int dim, int latent_dim, li_stream_t stream) {
-    if (batch < 0 || heads <= 0 || dim <= 0 || dim > 256 || latent_dim <= 0 || (latent_dim % 64) != 0 ||
-        heads > 65535)
+li_status li_absorb_query_layers(const void* q_bf16, const void* w_dec_bf16, void* q_tilde_bf16, int layers,
+                                 int batch, int heads, int dim, int latent_dim, li_stream_t stream) {
+    if (layers < 0 || layers > 65535 || batch < 0 || heads <= 0 || dim <= 0 || dim > 256 || latent_dim <= 0 ||
+        (latent_dim % 64) != 0 || heads > 65535)
         return LI_ERR_INVALID_ARG;
-    if (batch == 0) return LI_OK;
+    if (batch == 0 || layers == 0) return LI_OK;
     if (!q_bf16 || !w_dec_bf16 || !q_tilde_bf16 || !aligned(w_dec_bf16, 16) || !aligned(q_tilde_bf16, 2))
         return LI_ERR_INVALID_ARG;
     DevErr e;
     if (ready(&e) != LI_OK) return LI_ERR_CUDA;
-    return launch_absorb(q_bf16, w_dec_bf16, q_tilde_bf16, batch, heads, dim, latent_dim, stream);
+    return launch_absorb(q_bf16, w_dec_bf16, q_tilde_bf16, layers, batch, heads, dim, latent_dim, stream);
 }
 
-li_status li_latent_score(const void* q_tilde_bf16, const float* w, const void* c_bf16, int64_t cache_batch_rows,
-                          const int32_t* len, float* scores, int64_t scores_ld, int batch, int heads, int latent_dim,
-                          int max_len, li_stream_t stream) {
+li_status li_absorb_query(const void* q_bf16, const void* w_dec_bf16, void* q_tilde_bf16, int batch, int heads,
+                          int dim, int latent_dim, li_stream_t stream) {
+    return li_absorb_query_layers(q_bf16, w_dec_bf16, q_tilde_bf16, 1, batch, heads, dim, latent_dim, stream);
+}
+
+static li_status latent_score_impl(const void* q_tilde_bf16, const float* w, const void* c_bf16,
+                                   int64_t cache_batch_rows, const int32_t* len, float* scores, int64_t scores_ld,
+                                   int batch, int heads, int latent_dim, int max_len, uint32_t* hist,
+                                   li_stream_t stream) {
     if (batch < 0 || heads <= 0 || latent_dim <= 0 || max_len < 0 || cache_batch_rows < 0) return LI_ERR_INVALID_ARG;
     if (batch == 0 || max_len == 0) return LI_OK;
     if (!q_tilde_bf16 || !w || !c_bf16 || !scores || scores_ld < max_len) return LI_ERR_INVALID_ARG;
     if (heads != 64 || latent_dim != 256) return LI_ERR_UNSUPPORTED;
-    if (!aligned(c_bf16, 16) || !aligned(q_tilde_bf16, 16)) return LI_ERR_INVALID_ARG;
+    if (!aligned(c_bf16, 16) || !aligned(q_tilde_bf16, 16) || (hist && !aligned(hist, 16))) return LI_ERR_INVALID_ARG;
     DevErr e;
     if (ready(&e) != LI_OK) return LI_ERR_CUDA;
     const uint64_t total_rows = cache_batch_rows > 0 ? (uint64_t)(batch - 1) * cache_batch_rows + max_len
@@ -340,8 +346,26 @@ li_status li_latent_score(const void* q_tilde_bf16, const float* w, const void* 
     a.scores_ld = scores_ld;
     a.batch_rows = cache_batch_rows;
     a.max_len = max_len;
+    a.hist = hist;
     a.err = e;
-    return launch_stream_score_bf16(cmap, a, batch, (max_len + 127) / 128, stream);
+    const int ntiles = (max_len + 127) / 128;
+    return hist ? launch_stream_score_bf16_hist(cmap, a, batch, ntiles, stream)
+                : launch_stream_score_bf16(cmap, a, batch, ntiles, stream);
+}
+
+li_status li_latent_score(const void* q_tilde_bf16, const float* w, const void* c_bf16, int64_t cache_batch_rows,
+                          const int32_t* len, float* scores, int64_t scores_ld, int batch, int heads, int latent_dim,
+                          int max_len, li_stream_t stream) {
+    return latent_score_impl(q_tilde_bf16, w, c_bf16, cache_batch_rows, len, scores, scores_ld, batch, heads,
+                             latent_dim, max_len, nullptr, stream);
+}
+
+li_status li_latent_score_hist(const void* q_tilde_bf16, const float* w, const void* c_bf16,
+                               int64_t cache_batch_rows, const int32_t* len, float* scores, int64_t scores_ld,
+                               int batch, int heads, int latent_dim, int max_len, uint32_t* hist, li_stream_t stream) {
+    if (!hist && batch > 0 && max_len > 0) return LI_ERR_INVALID_ARG;
+    return latent_score_impl(q_tilde_bf16, w, c_bf16, cache_batch_rows, len, scores, scores_ld, batch, heads,
+                             latent_dim, max_len, hist, stream);
 }
 
 size_t li_hs_refine_workspace(int batch, int n_cand, int followers) {

@@ -22,7 +22,7 @@ struct StreamArgs {
     long long batch_rows;   // cache rows between requests (0 = shared cache)
     int max_len;
     int tiles_per_cta;      // set by the launcher
-    uint32_t* hist;         // FP8 kind, optional: [B, LI_HIST_BINS] counts of order_key(score) >> LI_HIST_SHIFT are
+    uint32_t* hist;         // optional: [B, LI_HIST_BINS] counts of order_key(score) >> LI_HIST_SHIFT are
                             // added to it (the caller provides it zeroed)
     DevErr err;
 };
@@ -32,6 +32,8 @@ li_status launch_stream_score_fp8_hist(const CUtensorMap& map, const StreamArgs&
                                        cudaStream_t st);
 li_status launch_stream_score_bf16(const CUtensorMap& map, const StreamArgs& args, int batch, int ntiles_max,
                                    cudaStream_t st);
+li_status launch_stream_score_bf16_hist(const CUtensorMap& map, const StreamArgs& args, int batch, int ntiles_max,
+                                        cudaStream_t st);
 
 // ---------------------------------------------------------------- causal prefill scorer
 struct PrefillArgs {
@@ -88,7 +90,8 @@ struct TopkArgs {
 li_status launch_topk(const TopkArgs& a, cudaStream_t st);
 
 // ---------------------------------------------------------------- absorption
-li_status launch_absorb(const void* q, const void* wdec, void* qt, int B, int H, int d, int dc, cudaStream_t st);
+li_status launch_absorb(const void* q, const void* wdec, void* qt, int G, int B, int H, int d, int dc,
+                        cudaStream_t st);
 
 // ---------------------------------------------------------------- HS gather + rescore
 struct HsArgs {

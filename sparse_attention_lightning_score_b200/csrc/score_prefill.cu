@@ -1,6 +1,6 @@
 // Causal prefill scorer: every query token t scans its own prefix, positions
-// s <= t + causal_offset ("scans the prefix", IndexCache explainer, Why This
-// Exists), I[t,s] = sk[s] * sum_j w_eff[t,j] * ReLU(q8[t,j,:] . k8[s,:]).
+// s <= t + causal_offset (IndexCache explainer, Why This Exists: in prefill the
+// indexer runs over each token's prefix), I[t,s] = sk[s] * sum_j w_eff[t,j] * ReLU(q8[t,j,:] . k8[s,:]).
 //
 // This is the compute-bound form of the indexer (the indexer is 81% of prefill
 // at 200K context on the IndexCache explainer's 30B model).  One MMA tile is

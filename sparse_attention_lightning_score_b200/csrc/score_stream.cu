@@ -1,5 +1,6 @@
 // Streaming indexer scorer for decode: one query token per request scans its
-// whole cache ("scores the whole cache", Multi-layer Indexer abstract).
+// entire cache (Multi-layer Indexer abstract: the indexer scores every cached
+// token).
 //
 //   FP8 kind (DSA decode):   I[b,s] = sk[s] * sum_j w_eff[b,j] * ReLU(q8[b,j,:] . k8[s,:])
 //                            q8/w_eff come from the bf16 query, quantised per
@@ -25,7 +26,7 @@
 // Grid: (CTAs per request, requests).  Each CTA streams a contiguous range of
 // key tiles of one request; sized for two CTAs per SM.
 //
-// HIST variant (decode score + top-k): every written score's order key is also
+// HIST variants (score + top-k): every written score's order key is also
 // counted by its top LI_HIST_BITS bits in a shared-memory histogram, which the
 // epilogue adds to the request's global histogram at the end; the top-k then
 // starts from that digit instead of sweeping the row for it.
@@ -65,7 +66,6 @@ template <bool FP8, int KBLK, int STAGES, int NACC, bool HIST>
 __global__ void __launch_bounds__(StreamCfg<FP8, KBLK, STAGES, NACC, HIST>::THREADS, 2)
     stream_score_kernel(const __grid_constant__ CUtensorMap kmap, const StreamArgs a) {
     using C = StreamCfg<FP8, KBLK, STAGES, NACC, HIST>;
-    static_assert(!HIST || C::PRO_WARPS == 8, "the histogram is cleared by the prologue helper warps");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
 
@@ -229,8 +229,7 @@ __global__ void __launch_bounds__(StreamCfg<FP8, KBLK, STAGES, NACC, HIST>::THRE
             if (et < C::H) wsm[et] = __ldg(a.w + (size_t)b * C::H + et);
         }
         if constexpr (HIST) {
-            if (warp >= 6)
-                for (int i = threadIdx.x - 192; i < LI_HIST_BINS; i += 128) hs[i] = 0u;
+            for (int i = et; i < LI_HIST_BINS; i += 32 * C::PRO_WARPS) hs[i] = 0u;
         }
         fence_proxy_async_smem();
         mbar_arrive(qready);
@@ -324,6 +323,11 @@ li_status launch_stream_score_fp8_hist(const CUtensorMap& map, const StreamArgs&
 li_status launch_stream_score_bf16(const CUtensorMap& map, const StreamArgs& args, int batch, int ntiles_max,
                                    cudaStream_t st) {
     return launch_impl<false, 4, 4, 4>(map, args, batch, ntiles_max, st);
+}
+
+li_status launch_stream_score_bf16_hist(const CUtensorMap& map, const StreamArgs& args, int batch, int ntiles_max,
+                                        cudaStream_t st) {
+    return launch_impl<false, 4, 4, 4, true>(map, args, batch, ntiles_max, st);
 }
 
 }  // namespace li

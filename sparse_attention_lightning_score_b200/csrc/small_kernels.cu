@@ -104,6 +104,10 @@ __global__ void __launch_bounds__(256) absorb_kernel(const __nv_bfloat16* __rest
     __shared__ float red[8][AB_BCH][64];
     const int j = blockIdx.x;
     const int c0 = blockIdx.y * 64;
+    // layer blockIdx.z: its queries, decoder and output follow the previous layer's
+    q += (size_t)blockIdx.z * B * H * d;
+    W += (size_t)blockIdx.z * H * d * dc;
+    qt += (size_t)blockIdx.z * B * H * dc;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int rg = t >> 3;   // row group 0..31
     const int cg = t & 7;    // 8 columns c0+8cg .. c0+8cg+7
@@ -223,9 +227,10 @@ li_status launch_simt_score(const SimtArgs& a, cudaStream_t st) {
     return LI_OK;
 }
 
-li_status launch_absorb(const void* q, const void* wdec, void* qt, int B, int H, int d, int dc, cudaStream_t st) {
-    if (B == 0) return LI_OK;
-    absorb_kernel<<<dim3(H, dc / 64), 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(q),
+li_status launch_absorb(const void* q, const void* wdec, void* qt, int G, int B, int H, int d, int dc,
+                        cudaStream_t st) {
+    if (B == 0 || G == 0) return LI_OK;
+    absorb_kernel<<<dim3(H, dc / 64, G), 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(q),
                                                      reinterpret_cast<const __nv_bfloat16*>(wdec),
                                                      reinterpret_cast<__nv_bfloat16*>(qt), B, H, d, dc);
     return host_check_launch();

@@ -145,3 +145,40 @@ def test_hs_full_size(B):
             ri = np.array([[pos[int(p)] for p in ro[f, i]]])
             assert_topk_equivalent(gi, ri, cs[f, i:i + 1], 1e-2)
     assert api.li_get_last_error() == LI_OK
+
+
+# ---------------------------------------------------------------------------
+# one-launch absorption of a layer group; latent scan with the first-digit histogram
+# ---------------------------------------------------------------------------
+def test_absorb_layers_matches_per_layer_calls():
+    case = synth.latent_hs(B=5, L=64, seed=81)
+    q = case.q.to(DEV).contiguous()          # [4, B, H, d]
+    wd = case.w_dec.to(DEV).contiguous()     # [4, H, d, dc]
+    got = api.li_absorb_query_layers(q, wd)
+    for l in range(4):
+        one = api.li_absorb_query(q[l], wd[l])
+        assert torch.equal(got[l].view(torch.int16), one.view(torch.int16)), l
+    assert api.li_get_last_error() == LI_OK
+
+
+@pytest.mark.parametrize("B,L,k,lens", [(1, 131072, 8192, None), (16, 32768, 8192, None),
+                                        (3, 20000, 2048, [20000, 2048, 0]), (2, 5000, 100, [4999, 1])])
+def test_latent_score_hist_then_topk_hist(B, L, k, lens):
+    """The anchor's scan with the histogram, then li_topk_hist: bit for bit what li_latent_score
+    followed by li_topk gives, and the histogram left zero."""
+    case = synth.latent_hs(B=B, L=L, seed=82 + B, lens=lens)
+    c = case.c.to(DEV)
+    qt = api.li_absorb_query(case.q[0].to(DEV), case.w_dec[0].to(DEV))
+    w = case.w[0].to(DEV)
+    ln = case.lens.to(DEV)
+    hist = api.li_decode_select_workspace(B, DEV).view(torch.int32)[:B * 2048]
+    sc = api.li_latent_score_hist(qt, w, c, hist, lens=ln)
+    idx, vals = api.li_topk_hist(sc, k, hist, lens=ln, max_len=L, with_values=True)
+    sc_r = api.li_latent_score(qt, w, c, lens=ln)
+    idx_r, vals_r = api.li_topk(sc_r, k, lens=ln, max_len=L, with_values=True)
+    for b, n in enumerate(case.lens.tolist()):
+        assert np.array_equal(_np(sc[b, :n]).view(np.uint32), _np(sc_r[b, :n]).view(np.uint32)), b
+    assert np.array_equal(_np(idx), _np(idx_r))
+    assert np.array_equal(_np(vals).view(np.uint32), _np(vals_r).view(np.uint32))
+    assert api.li_get_last_error() == LI_OK
+    assert int(hist.count_nonzero()) == 0
