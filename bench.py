@@ -505,33 +505,48 @@ class PrefillBench:
 
 
 class LatentBench:
-    """LatentIndex G=4 group decode: 4 x (absorb + latent score + top-2048), B=4, L=65536."""
+    """LatentIndex G=4 group decode: 4 x (absorb + latent score + top-2048), B=4, L=65536; each
+    layer's scan counts its first radix digit for the top-k.  kind "bf16": the d_c = 256 bf16
+    latent cache; kind "fp8_192": DeepSeek-V3.2's 64 RoPE + 128 NoPE latent as an e4m3 cache
+    with per-row scales."""
 
-    def __init__(self, dev, B=4, Lx=65536):
+    def __init__(self, dev, B=4, Lx=65536, kind="bf16"):
         import torch
         from sparse_attention_lightning_score_b200 import api, synth
         self.api = api
-        self.B, self.L = B, Lx
-        case = synth.latent_group(B=B, L=Lx)
-        self.c = [case.c.to(dev)]
-        per = case.c.numel() * 2
+        self.B, self.L, self.kind = B, Lx, kind
+        if kind == "bf16":
+            case = synth.latent_group(B=B, L=Lx)
+            self.c = [(case.c.to(dev), None)]
+            per = case.c.numel() * 2
+            self.dc, self.key_bytes = 256, 512
+        else:
+            case = synth.latent_rope_nope(B=B, L=Lx)
+            self.c = [(case.c8.to(dev), case.cs.to(dev))]
+            per = case.c8.numel() + case.cs.numel() * 4
+            self.dc, self.key_bytes = 192, 196
         while len(self.c) * per < 1.5 * L2_BYTES:
-            self.c.append(self.c[0].clone())
+            self.c.append(tuple(t.clone() if t is not None else None for t in self.c[0]))
         self.q = [case.q[l].to(dev) for l in range(4)]
         self.wd = [case.w_dec[l].to(dev) for l in range(4)]
-        self.qf = case.q[1:].contiguous().to(dev)
-        self.wdf = case.w_dec[1:].contiguous().to(dev)
         self.hist = api.li_decode_select_workspace(B, dev).view(torch.int32)[:B * 2048]
-        self.side = torch.cuda.Stream(device=dev)
+        self.hist_scratch = api.li_decode_select_workspace(B, dev).view(torch.int32)[:B * 2048]
         self.w = [case.w[l].to(dev) for l in range(4)]
-        self.qt = torch.empty((B, H, 256), dtype=torch.bfloat16, device=dev)
+        self.qt = torch.empty((B, H, self.dc), dtype=torch.bfloat16, device=dev)
         self.sc = torch.empty((B, Lx), dtype=torch.float32, device=dev)
         self.idx = torch.empty((4, B, KTOP), dtype=torch.int32, device=dev)
 
+    def score(self, i, l, hist):
+        c, cs = self.c[i % len(self.c)]
+        if cs is None:
+            self.api.li_latent_score_hist(self.qt, self.w[l], c, hist, scores=self.sc)
+        else:
+            self.api.li_latent_score_fp8(self.qt, self.w[l], c, cs, hist=hist, scores=self.sc)
+
     def layer(self, i, l):
         self.api.li_absorb_query(self.q[l], self.wd[l], out=self.qt)
-        self.api.li_latent_score(self.qt, self.w[l], self.c[i % len(self.c)], scores=self.sc)
-        self.api.li_topk(self.sc, KTOP, idx=self.idx[l])
+        self.score(i, l, self.hist)
+        self.api.li_topk_hist(self.sc, KTOP, self.hist, idx=self.idx[l])
 
     def run(self, steps, warmup):
         import torch
@@ -540,8 +555,8 @@ class LatentBench:
                 self.layer(i, l)
         torch.cuda.synchronize()
         graphs = [capture([lambda i=i, l=l: self.layer(i, l) for l in range(4)]) for i in range(len(self.c))]
-        g_sc = capture([lambda i=i: self.api.li_latent_score(self.qt, self.w[0], self.c[i % len(self.c)], scores=self.sc)
-                        for i in range(8)])
+        # the scan alone (its counts go to a scratch histogram nobody reads)
+        g_sc = capture([lambda i=i: self.score(i, 0, self.hist_scratch) for i in range(8)])
         for g in graphs:
             g.replay()
         torch.cuda.synchronize()
@@ -645,20 +660,22 @@ def run_other(args, rank, world, local_rank):
                             "frac": achieved / fp8_burst, "frac_of_sustained": achieved / fp8_sust,
                             "score_ms": r["score"]},
                "topk": {"ms": r["topk"], "rows_per_s": bx.T / (r["topk"] * 1e-3)}, "clocks": clk}
-    elif args.workload == "latent":
-        bx = LatentBench(dev)
+    elif args.workload in ("latent", "latent192"):
+        bx = LatentBench(dev, kind="bf16" if args.workload == "latent" else "fp8_192")
         clocks.start()
         r = bx.run(args.steps, args.warmup)
         clk = clocks.stop()
-        per_layer_bytes = bx.B * bx.L * (512 + 4)
+        per_layer_bytes = bx.B * bx.L * (bx.key_bytes + 4)
         achieved = per_layer_bytes / (r["score"] * 1e-3) / 1e9
+        fp8 = bx.kind != "bf16"
         out = {"metric": METRIC, "value": 4 * bx.B * bx.L / (r["step"] * 1e-3), "unit": "keys/s",
                "ms_per_step": r["step"], "us_per_layer": r["step"] * 1e3 / 4, "higher_is_better": True,
-               "dtype": "bf16", "config": {"workload": "latent_g4_b4_l64k", "B": bx.B, "L": bx.L, "G": 4,
-                                           "d_c": 256, "k": KTOP, "l2": f"{len(bx.c)} rotating cache copies"},
-               "roofline": {"bound": "hbm", "kernel": "stream_score_kernel<bf16>", "achieved": achieved,
-                            "peak": hbm, "peak_source": which, "unit": "GB/s", "frac": achieved / hbm,
-                            "kernel_us": r["score"] * 1e3}, "clocks": clk}
+               "dtype": "e4m3" if fp8 else "bf16",
+               "config": {"workload": "latent_fp8_dc192_g4_b4_l64k" if fp8 else "latent_g4_b4_l64k", "B": bx.B,
+                          "L": bx.L, "G": 4, "d_c": bx.dc, "k": KTOP, "l2": f"{len(bx.c)} rotating cache copies"},
+               "roofline": {"bound": "hbm", "kernel": "latent8_score_kernel" if fp8 else "stream_score_kernel<bf16>",
+                            "achieved": achieved, "peak": hbm, "peak_source": which, "unit": "GB/s",
+                            "frac": achieved / hbm, "kernel_us": r["score"] * 1e3}, "clocks": clk}
     else:
         Bx = 1 if args.workload == "hs_b1" else 16
         bx = HsBench(dev, Bx)
@@ -688,7 +705,7 @@ def main():
     ap.add_argument("--impl", default="li", choices=["li", "reference"])
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "latent", "hs_b1", "hs_b16"],
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "latent", "latent192", "hs_b1", "hs_b16"],
                     help="decode (default) is the benchmarked configuration; the others time the other "
                          "configurations of the parity tests")
     args = ap.parse_args()

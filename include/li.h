@@ -230,6 +230,25 @@ li_status li_latent_score_hist(const void* q_tilde_bf16, const float* w, const v
                                int64_t cache_batch_rows, const int32_t* len, float* scores, int64_t scores_ld,
                                int batch, int heads, int latent_dim, int max_len, uint32_t* hist, li_stream_t stream);
 
+/* The LatentIndex scan over an FP8 latent cache: latent rows stored in e4m3
+ * with one fp32 scale per row, c = c8 * cs (per-row absmax / 448, as the DSA
+ * key cache).  The latent width is 192, DeepSeek-V3.2's shared latent of 64
+ * RoPE and 128 NoPE dimensions (LatentIndex appendix, Table 5).  The absorbed
+ * bf16 query is quantised per (request, head) inside the call exactly as
+ * li_quantize_query does, and the score is
+ *     scores[b * scores_ld + s] = cs[s] * sum_j w_eff[b,j] * ReLU(q8[b,j,:] . c8[s,:])
+ * for s < len[b], with w_eff = w * sq.
+ *   q_tilde [batch, 64, 192] bf16 (16-byte aligned)   w [batch, 64] fp32
+ *   c_e4m3  latent rows of 192 bytes (16-byte aligned); request b's rows begin
+ *           at row b * cache_batch_rows (0 = one cache shared by all requests)
+ *   c_scale one fp32 per latent row, same numbering
+ *   hist    NULL, or [batch, 2048] uint32 first-digit counts added to as
+ *           li_latent_score_hist does (zero before the call), for li_topk_hist
+ * heads must be 64 and latent_dim 192 (LI_ERR_UNSUPPORTED otherwise). */
+li_status li_latent_score_fp8(const void* q_tilde_bf16, const float* w, const void* c_e4m3, const float* c_scale,
+                              int64_t cache_batch_rows, const int32_t* len, float* scores, int64_t scores_ld,
+                              int batch, int heads, int latent_dim, int max_len, uint32_t* hist, li_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Hierarchical selection: followers refine the anchor's candidates         */
 /* ------------------------------------------------------------------------ */

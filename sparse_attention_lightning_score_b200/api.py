@@ -259,6 +259,31 @@ def li_latent_score_hist(q_tilde: torch.Tensor, w: torch.Tensor, c: torch.Tensor
     return scores
 
 
+def li_latent_score_fp8(q_tilde: torch.Tensor, w: torch.Tensor, c8: torch.Tensor, c_scale: torch.Tensor, *,
+                        lens: Optional[torch.Tensor] = None, scores: Optional[torch.Tensor] = None,
+                        hist: Optional[torch.Tensor] = None, stream=None):
+    """Latent scan over an FP8 latent cache: q~ bf16 [B,64,192], w fp32 [B,64], c8 e4m3/uint8
+    [B,L,192] (or shared [L,192]) with fp32 per-row scales -> scores fp32 [B, round4(L)].
+    With `hist` (zeroed [B, 2048] buffer) the first-digit counts for li_topk_hist are added."""
+    _need(q_tilde, "q_tilde", torch.bfloat16)
+    _need(w, "w", torch.float32)
+    _need(c8, "c8")
+    _need(c_scale, "c_scale", torch.float32)
+    if c8.dtype == torch.float8_e4m3fn:
+        c8 = c8.view(torch.uint8)
+    B, H, dc = q_tilde.shape
+    L = c8.shape[-2]
+    batch_rows = c8.shape[1] if c8.dim() == 3 else 0
+    if lens is not None:
+        _need(lens, "lens", torch.int32)
+    if scores is None:
+        scores = torch.empty((B, _round4(L)), dtype=torch.float32, device=c8.device)
+    st = _lib.load().li_latent_score_fp8(_ptr(q_tilde), _ptr(w), _ptr(c8), _ptr(c_scale), batch_rows, _ptr(lens),
+                                         _ptr(scores), scores.stride(0), B, H, dc, L, _ptr(hist), _stream(stream))
+    _lib.check("li_latent_score_fp8", st)
+    return scores
+
+
 def li_latent_score(q_tilde: torch.Tensor, w: torch.Tensor, c: torch.Tensor, *, lens: Optional[torch.Tensor] = None,
                     scores: Optional[torch.Tensor] = None, stream=None):
     """q~ bf16 [B,H,dc], w fp32 [B,H], c bf16 [B,L,dc] (or shared [L,dc]) -> scores fp32 [B, round4(L)]."""

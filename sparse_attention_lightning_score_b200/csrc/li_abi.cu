@@ -40,16 +40,16 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // 2-D tensor map over `rows` rows of `row_elems` elements (row pitch
 // `row_bytes`), box = [box_inner elements, box_rows rows], 128-byte swizzle.
 bool encode_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t row_elems, uint64_t rows,
-                   uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows) {
+                   uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows,
+                   CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
     auto fn = tensor_map_encoder();
     if (!fn) return false;
     cuuint64_t dims[2] = {row_elems, rows};
     cuuint64_t strides[1] = {row_bytes};
     cuuint32_t box[2] = {box_inner, box_rows};
     cuuint32_t estr[2] = {1, 1};
-    return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -366,6 +366,37 @@ li_status li_latent_score_hist(const void* q_tilde_bf16, const float* w, const v
     if (!hist && batch > 0 && max_len > 0) return LI_ERR_INVALID_ARG;
     return latent_score_impl(q_tilde_bf16, w, c_bf16, cache_batch_rows, len, scores, scores_ld, batch, heads,
                              latent_dim, max_len, hist, stream);
+}
+
+li_status li_latent_score_fp8(const void* q_tilde_bf16, const float* w, const void* c_e4m3, const float* c_scale,
+                              int64_t cache_batch_rows, const int32_t* len, float* scores, int64_t scores_ld,
+                              int batch, int heads, int latent_dim, int max_len, uint32_t* hist, li_stream_t stream) {
+    if (batch < 0 || heads <= 0 || latent_dim <= 0 || max_len < 0 || cache_batch_rows < 0) return LI_ERR_INVALID_ARG;
+    if (batch == 0 || max_len == 0) return LI_OK;
+    if (!q_tilde_bf16 || !w || !c_e4m3 || !c_scale || !scores || scores_ld < max_len) return LI_ERR_INVALID_ARG;
+    if (heads != 64 || latent_dim != 192) return LI_ERR_UNSUPPORTED;
+    if (!aligned(c_e4m3, 16) || !aligned(q_tilde_bf16, 16) || (hist && !aligned(hist, 16))) return LI_ERR_INVALID_ARG;
+    DevErr e;
+    if (ready(&e) != LI_OK) return LI_ERR_CUDA;
+    const uint64_t total_rows = cache_batch_rows > 0 ? (uint64_t)(batch - 1) * cache_batch_rows + max_len
+                                                     : (uint64_t)max_len;
+    if (total_rows >= (1ull << 31)) return LI_ERR_UNSUPPORTED;
+    CUtensorMap cmap;  // 192-byte rows, boxes of 64 bytes x 128 rows, 64-byte swizzle
+    if (!encode_map_2d(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, c_e4m3, 192, total_rows, 192, 64, 128,
+                       CU_TENSOR_MAP_SWIZZLE_64B))
+        return LI_ERR_CUDA;
+    Latent8Args a{};
+    a.q = q_tilde_bf16;
+    a.w = w;
+    a.cscale = c_scale;
+    a.len = len;
+    a.scores = scores;
+    a.scores_ld = scores_ld;
+    a.batch_rows = cache_batch_rows;
+    a.max_len = max_len;
+    a.hist = hist;
+    a.err = e;
+    return launch_latent8_score(cmap, a, batch, (max_len + 127) / 128, stream);
 }
 
 size_t li_hs_refine_workspace(int batch, int n_cand, int followers) {

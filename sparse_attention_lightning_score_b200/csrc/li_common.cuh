@@ -167,6 +167,15 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* map, int x, i
         : "memory");
 }
 
+// Contiguous global -> shared copy by the TMA engine, completing on `bar`.
+// dst and src 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // tcgen05: TMEM allocation, MMA issue, completion, loads
 // ---------------------------------------------------------------------------
@@ -237,6 +246,26 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr) {
     d |= uint64_t(1u) << 46;
     d |= uint64_t(2u) << 61;
     return d;
+}
+
+// The same for a K-major operand stored with the 64-byte swizzle: rows of 64
+// bytes, 8-row (512-byte) swizzle atoms 512 bytes apart, layout type
+// SWIZZLE_64B (4).
+__device__ __forceinline__ uint64_t sw64_kmajor_desc(uint32_t smem_addr) {
+    uint64_t d = 0;
+    d |= uint64_t((smem_addr >> 4) & 0x3FFFu);
+    d |= uint64_t(1u) << 16;
+    d |= uint64_t(512u >> 4) << 32;
+    d |= uint64_t(1u) << 46;
+    d |= uint64_t(4u) << 61;
+    return d;
+}
+
+// Byte offset of 16-byte chunk `chunk` (0..3) of row `row` inside a
+// 64-byte-swizzled tile whose base is 512-byte aligned: the chunk index is
+// XORed with address bits 7-8, i.e. (row / 2) mod 4.
+__device__ __forceinline__ uint32_t sw64_offset(uint32_t row, uint32_t chunk) {
+    return row * 64u + (((chunk ^ (row >> 1)) & 3u) << 4);
 }
 
 // Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside a

@@ -35,6 +35,23 @@ li_status launch_stream_score_bf16(const CUtensorMap& map, const StreamArgs& arg
 li_status launch_stream_score_bf16_hist(const CUtensorMap& map, const StreamArgs& args, int batch, int ntiles_max,
                                         cudaStream_t st);
 
+// ---------------------------------------------------------------- FP8 latent scorer (d_c = 192)
+struct Latent8Args {
+    const void* q;          // absorbed query q~, bf16 [B,64,192]
+    const float* w;         // [B,64]
+    const float* cscale;    // one fp32 per latent row
+    const int32_t* len;     // [B] or nullptr
+    float* scores;
+    long long scores_ld;
+    long long batch_rows;   // latent rows between requests (0 = shared cache)
+    int max_len;
+    int tiles_per_cta;      // set by the launcher
+    uint32_t* hist;         // optional [B, LI_HIST_BINS] first-digit counts, added to
+    DevErr err;
+};
+li_status launch_latent8_score(const CUtensorMap& map, const Latent8Args& args, int batch, int ntiles_max,
+                               cudaStream_t st);
+
 // ---------------------------------------------------------------- causal prefill scorer
 struct PrefillArgs {
     const float* w_eff;     // [T,64] (w * per-(token, head) query scale)

@@ -46,7 +46,7 @@ struct StreamCfg {
     static constexpr int OFF_Q = STAGES * STAGE_BYTES;
     static constexpr int OFF_W = OFF_Q + Q_BYTES;
     static constexpr int OFF_BAR = OFF_W + H * 4;
-    static constexpr int NBAR = 2 * STAGES + 2 * NACC + 1;
+    static constexpr int NBAR = 2 * STAGES + 2 * NACC + 2;  // ... qready, qload
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
     static constexpr int OFF_HIST = OFF_TMEM + 16;
     static constexpr int SMEM = OFF_HIST + (HIST ? LI_HIST_BINS * 4 : 0) + 1024;  // + slack to align the base to 1024
@@ -79,6 +79,7 @@ __global__ void __launch_bounds__(StreamCfg<FP8, KBLK, STAGES, NACC, HIST>::THRE
     uint64_t* accf = empty + STAGES;
     uint64_t* acce = accf + NACC;
     uint64_t* qready = acce + NACC;
+    uint64_t* qload = qready + 1;  // FP8: the query row's bulk copy into the last stage's buffer
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
     float* wsm = reinterpret_cast<float*>(smem + C::OFF_W);
     uint8_t* qsm = smem + C::OFF_Q;
@@ -94,6 +95,7 @@ __global__ void __launch_bounds__(StreamCfg<FP8, KBLK, STAGES, NACC, HIST>::THRE
             mbar_init(&acce[i], 128);
         }
         mbar_init(qready, 32 * C::PRO_WARPS);
+        mbar_init(qload, 1);
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -107,25 +109,25 @@ __global__ void __launch_bounds__(StreamCfg<FP8, KBLK, STAGES, NACC, HIST>::THRE
 
     // everything above overlaps the previous kernel; inputs are read only after it completed
     pdl_wait();
-    // FP8: the prologue warps issue their query loads before the length is known, so that the two
-    // round trips overlap (the length decides only whether this CTA has any tile)
+    // FP8: the request's bf16 query row (16 KB) comes in by one bulk copy into the last stage's
+    // buffer, issued before any key tile so that it is not queued behind them; the head weights
+    // are loaded by the prologue warps.  Both are issued before the length is known.
     constexpr int QHPW = C::H / C::PRO_WARPS;  // heads per prologue warp
     constexpr int QIT = QHPW / 4;              // four heads at a time, eight lanes per head
-    uint4 qraw[FP8 ? QIT : 1][2];
+    constexpr uint32_t QROW_BYTES = C::H * 128 * 2;
+    static_assert(!FP8 || QROW_BYTES <= C::STAGE_BYTES, "the query row fits one stage buffer");
+    uint8_t* qstage = smem + (STAGES - 1) * C::STAGE_BYTES;
     float qw[FP8 ? QIT : 1];
     if constexpr (FP8) {
+        if (threadIdx.x == 0) {
+            mbar_arrive_expect_tx(qload, QROW_BYTES);
+            bulk_load(qstage, reinterpret_cast<const uint8_t*>(a.q) + (size_t)b * QROW_BYTES, QROW_BYTES, qload);
+        }
         if (warp >= 2) {
             const int ew = (threadIdx.x - 64) >> 5;
-            const int g8 = lane >> 3, l8 = lane & 7;
-            const __nv_bfloat16* q = reinterpret_cast<const __nv_bfloat16*>(a.q) + (size_t)b * C::H * 128;
+            const int g8 = lane >> 3;
 #pragma unroll
-            for (int i = 0; i < QIT; ++i) {
-                const int j = QHPW * ew + 4 * i + g8;
-                const uint4* src = reinterpret_cast<const uint4*>(q + (size_t)j * 128) + 2 * l8;
-                qraw[i][0] = __ldg(src);
-                qraw[i][1] = __ldg(src + 1);
-                qw[i] = __ldg(a.w + (size_t)b * C::H + j);
-            }
+            for (int i = 0; i < QIT; ++i) qw[i] = __ldg(a.w + (size_t)b * C::H + QHPW * ew + 4 * i + g8);
         }
     }
     int len_b = a.len ? __ldg(a.len + b) : a.max_len;
@@ -150,6 +152,8 @@ __global__ void __launch_bounds__(StreamCfg<FP8, KBLK, STAGES, NACC, HIST>::THRE
             for (int it = 0; ok && it < nt; ++it) {
                 const int y = (int)(rowbase + (long long)(t0 + it) * C::M);
                 for (int kb = 0; kb < KBLK; ++kb) {
+                    // FP8: the last stage's buffer first holds the query row, until it is quantised
+                    if (FP8 && stage == STAGES - 1 && ph == 0u && !mbar_wait(qready, 0, a.err)) { ok = false; break; }
                     if (!mbar_wait(&empty[stage], ph ^ 1u, a.err)) { ok = false; break; }
                     mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
                     tma_load_2d(smem + stage * C::STAGE_BYTES, &kmap, kb * C::ELEMS_PER_KBLOCK, y, &full[stage],
@@ -198,8 +202,17 @@ __global__ void __launch_bounds__(StreamCfg<FP8, KBLK, STAGES, NACC, HIST>::THRE
         const int ew = et >> 5;
         if constexpr (FP8) {
             // 8 heads per warp, four at a time (8 lanes per head, 16 elements per
-            // lane), from the loads issued above
+            // lane), from the query row in shared memory
             const int g8 = lane >> 3, l8 = lane & 7;
+            const bool qin = mbar_wait(qload, 0, a.err);
+            uint4 qraw[QIT][2];
+#pragma unroll
+            for (int i = 0; i < QIT; ++i) {
+                const int j = QHPW * ew + 4 * i + g8;
+                const uint4* src = reinterpret_cast<const uint4*>(qstage + j * 256) + 2 * l8;
+                qraw[i][0] = qin ? src[0] : make_uint4(0u, 0u, 0u, 0u);
+                qraw[i][1] = qin ? src[1] : make_uint4(0u, 0u, 0u, 0u);
+            }
 #pragma unroll
             for (int i = 0; i < QIT; ++i) {
                 const int j = QHPW * ew + 4 * i + g8;
@@ -274,6 +287,9 @@ __global__ void __launch_bounds__(StreamCfg<FP8, KBLK, STAGES, NACC, HIST>::THRE
         }
     }
 done:
+    // the query row's bulk copy must have landed before the CTA may leave (a CTA without a
+    // tile never waited for it)
+    if (FP8 && threadIdx.x == 0) (void)mbar_wait(qload, 0, a.err);
     __syncwarp();
     __syncthreads();
     if (warp == 1) {

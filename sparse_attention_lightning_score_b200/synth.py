@@ -219,6 +219,51 @@ def latent_hs(B: int = 1, L: int = 131072, H: int = 64, d: int = 128, dc: int = 
 
 
 # --------------------------------------------------------------------------
+# LatentIndex with DeepSeek-V3.2's latent layout and an FP8 latent cache
+# --------------------------------------------------------------------------
+@dataclass
+class LatentFp8:
+    c: torch.Tensor        # bf16 [B, L, 192]    latent rows before FP8 storage
+    c8: torch.Tensor       # uint8 [B, L, 192]   e4m3 bytes of the cache
+    cs: torch.Tensor       # fp32 [B, L]         per-row scales
+    w_dec: torch.Tensor    # bf16 [G, H, 128, 192] per-layer key decoders
+    q: torch.Tensor        # bf16 [G, B, H, 128] per-layer indexer queries
+    w: torch.Tensor        # fp32 [G, B, H]
+    lens: torch.Tensor     # int32 [B]
+    k_top: int = 2048
+
+
+def latent_rope_nope(B: int = 4, L: int = 65536, H: int = 64, G: int = 4, k_top: int = 2048, seed: int = 5,
+                     lens: Optional[list] = None, device: str = "cpu") -> LatentFp8:
+    """Shared latent of 64 RoPE + 128 NoPE dimensions for 128-wide indexer keys of
+    64 RoPE + 64 NoPE dimensions (DeepSeek-V3.2's sizes, LatentIndex appendix,
+    Table 5), stored as an e4m3 cache with per-row scales.
+
+    Draw order: c (request by request), the NoPE decoders, q, w.  c ~ N(0,1) and
+    q ~ N(0,1) rounded to bf16; w ~ N(0, 0.1^2).  Each layer's decoder copies
+    the 64 RoPE latent dimensions to the key's 64 RoPE dimensions unchanged and
+    maps the 128 NoPE latent dimensions to the key's 64 NoPE dimensions with a
+    random matrix ~ N(0, (1/sqrt(128))^2) rounded to bf16.
+    """
+    g = _gen(seed, device)
+    c = torch.empty(B, L, 192, dtype=torch.bfloat16, device=device)
+    for b in range(B):
+        c[b] = _randn(g, L, 192, device=device).to(torch.bfloat16)
+    nope = (_randn(g, G, H, 64, 128, device=device) / math.sqrt(128)).to(torch.bfloat16)
+    w_dec = torch.zeros(G, H, 128, 192, dtype=torch.bfloat16, device=device)
+    w_dec[:, :, torch.arange(64), torch.arange(64)] = 1.0
+    w_dec[:, :, 64:, 64:] = nope
+    q = _randn(g, G, B, H, 128, device=device).to(torch.bfloat16)
+    w = _randn(g, G, B, H, device=device) * 0.1
+    c8, cs = encode_e4m3_cache(c.float())
+    if lens is None:
+        lens_t = torch.full((B,), L, dtype=torch.int32, device=device)
+    else:
+        lens_t = torch.tensor(lens, dtype=torch.int32, device=device)
+    return LatentFp8(c=c, c8=c8, cs=cs, w_dec=w_dec, q=q, w=w, lens=lens_t, k_top=k_top)
+
+
+# --------------------------------------------------------------------------
 # Plain score rows for the top-k select alone
 # --------------------------------------------------------------------------
 def score_rows(rows: int, L: int, seed: int = 5, ties: int = 0, device: str = "cpu") -> torch.Tensor:

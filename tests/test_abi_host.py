@@ -98,3 +98,24 @@ def test_workspace_sizes():
     d.causal = 0
     assert lib.li_index_score_workspace(ctypes.byref(d)) == 0
     assert lib.li_hs_refine_workspace(16, 8192, 3) == 3 * 16 * 8192 * 4
+
+
+def test_latent_fp8_and_layers_reject_bad_arguments_on_host():
+    lib = _lib.load()
+    p = ctypes.c_void_p(256)
+    # (q~, w, c8, cs, cache_batch_rows, len, scores, ld, batch, heads, latent_dim, max_len, hist, stream)
+    assert lib.li_latent_score_fp8(p, p, p, p, 0, None, p, 100, 2, 32, 192, 100, None, None) == _lib.LI_ERR_UNSUPPORTED
+    assert lib.li_latent_score_fp8(p, p, p, p, 0, None, p, 100, 2, 64, 256, 100, None, None) == _lib.LI_ERR_UNSUPPORTED
+    assert lib.li_latent_score_fp8(p, p, ctypes.c_void_p(264), p, 0, None, p, 100, 2, 64, 192, 100, None,
+                                   None) == _lib.LI_ERR_INVALID_ARG          # cache not 16-byte aligned
+    assert lib.li_latent_score_fp8(p, p, p, None, 0, None, p, 100, 2, 64, 192, 100, None,
+                                   None) == _lib.LI_ERR_INVALID_ARG          # no scales
+    assert lib.li_latent_score_fp8(p, p, p, p, 0, None, p, 50, 2, 64, 192, 100, None,
+                                   None) == _lib.LI_ERR_INVALID_ARG          # ld below max_len
+    assert lib.li_latent_score_fp8(p, p, p, p, 0, None, p, 100, 0, 64, 192, 100, None, None) == _lib.LI_OK
+    assert lib.li_latent_score_hist(p, p, p, 0, None, p, 100, 2, 64, 256, 100, None,
+                                    None) == _lib.LI_ERR_INVALID_ARG         # hist required
+    # (q, w_dec, q~, layers, batch, heads, dim, latent_dim, stream)
+    assert lib.li_absorb_query_layers(p, p, p, -1, 1, 64, 128, 256, None) == _lib.LI_ERR_INVALID_ARG
+    assert lib.li_absorb_query_layers(p, p, p, 2, 1, 64, 128, 100, None) == _lib.LI_ERR_INVALID_ARG
+    assert lib.li_absorb_query_layers(p, p, p, 0, 1, 64, 128, 256, None) == _lib.LI_OK
