@@ -193,6 +193,7 @@ li_status li_index_score(const void* q, const float* w, const void* k, const flo
         a.scores_ld = scores_ld;
         a.batch_rows = cache_batch_rows;
         a.max_len = d.max_len;
+        a.w_bulk = aligned(w, 16) ? 1 : 0;
         a.err = e;
         const int ntiles = (d.max_len + 127) / 128;
         return launch_stream_score_fp8(kmap, a, d.rows, ntiles, stream);
@@ -260,6 +261,7 @@ li_status li_decode_score_hist(const void* q, const float* w, const void* k, con
     a.batch_rows = cache_batch_rows;
     a.max_len = d.max_len;
     a.hist = hist;
+    a.w_bulk = aligned(w, 16) ? 1 : 0;
     a.err = e;
     return launch_stream_score_fp8_hist(kmap, a, d.rows, (d.max_len + 127) / 128, stream);
 }

@@ -352,14 +352,30 @@ __device__ __forceinline__ float relu_dot32_x2(const uint32_t (&v)[32], const fl
 // unless an e4m3 rounding midpoint lies between them.  For |y| in e4m3's
 // normal range, those midpoints are the values whose 20 low mantissa bits are
 // 0x80000.  So only a product within 8 ulp of such a point, or outside
-// [2^-6, 512] (e4m3 subnormals, zero, an overflowed reciprocal, NaN), is
-// recomputed with the division.
-__device__ __forceinline__ float quotient_for_e4m3(float x, float sq, float r) {
-    float y = x * r;
+// [2^-6, 512] (e4m3 subnormals, zero, an overflowed reciprocal, NaN), needs
+// the division.
+__device__ __forceinline__ bool quotient_needs_division(float y) {
     const float ay = fabsf(y);
     const uint32_t m = __float_as_uint(y) & 0xfffffu;
-    if (!(ay >= 0x1p-6f && ay <= 512.f) || (m - 0x7fff8u) <= 16u) y = __fdiv_rn(x, sq);
-    return y;
+    return !(ay >= 0x1p-6f && ay <= 512.f) || (m - 0x7fff8u) <= 16u;
+}
+
+// y[i] = x[i] / sq rounded as IEEE division for N elements of every lane.  The
+// products are taken first; when any lane of the warp has an element that needs
+// it, the whole warp divides instead (warp-uniform, so the rare path costs no
+// divergent branch per element).  All 32 lanes must call this together.
+template <int N>
+__device__ __forceinline__ void quotients_for_e4m3(const float (&x)[N], float sq, float r, float (&y)[N]) {
+    bool need = false;
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+        y[i] = x[i] * r;
+        need |= quotient_needs_division(y[i]);
+    }
+    if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+        for (int i = 0; i < N; ++i) y[i] = __fdiv_rn(x[i], sq);
+    }
 }
 
 // Two fp32 values to e4m3 (nearest even, saturating to +-448): lo in the low byte, hi in the high byte.
@@ -369,8 +385,12 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
     return d;
 }
 
+// One element (all 32 lanes call together).
 __device__ __forceinline__ uint32_t e4m3_quotient(float x, float sq, float r) {
-    return e4m3x2(quotient_for_e4m3(x, sq, r), 0.f) & 0xffu;
+    const float xs[1] = {x};
+    float y[1];
+    quotients_for_e4m3<1>(xs, sq, r, y);
+    return e4m3x2(y[0], 0.f) & 0xffu;
 }
 
 // Per-(row, head) e4m3 quantisation of one 128-element bf16 head vector held
@@ -386,8 +406,10 @@ __device__ __forceinline__ uint32_t quantize_head128(uint2 raw, float* sq_out) {
     const float sq = m > 0.f ? __fdiv_rn(m, 448.f) : 1.f;
     *sq_out = sq;
     const float r = __frcp_rn(sq);
-    return e4m3x2(quotient_for_e4m3(x0, sq, r), quotient_for_e4m3(x1, sq, r)) |
-           (e4m3x2(quotient_for_e4m3(x2, sq, r), quotient_for_e4m3(x3, sq, r)) << 16);
+    const float xs[4] = {x0, x1, x2, x3};
+    float y[4];
+    quotients_for_e4m3<4>(xs, sq, r, y);
+    return e4m3x2(y[0], y[1]) | (e4m3x2(y[2], y[3]) << 16);
 }
 
 // Same quantisation with 8 lanes per head: the lane holds 16 consecutive bf16
@@ -410,11 +432,11 @@ __device__ __forceinline__ uint4 quantize_head128_g8(uint4 lo, uint4 hi, float* 
     const float sq = m > 0.f ? __fdiv_rn(m, 448.f) : 1.f;
     *sq_out = sq;
     const float r = __frcp_rn(sq);
+    float y[16];
+    quotients_for_e4m3<16>(x, sq, r, y);
     uint32_t b[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-        b[i] = e4m3x2(quotient_for_e4m3(x[4 * i + 0], sq, r), quotient_for_e4m3(x[4 * i + 1], sq, r)) |
-               (e4m3x2(quotient_for_e4m3(x[4 * i + 2], sq, r), quotient_for_e4m3(x[4 * i + 3], sq, r)) << 16);
+    for (int i = 0; i < 4; ++i) b[i] = e4m3x2(y[4 * i], y[4 * i + 1]) | (e4m3x2(y[4 * i + 2], y[4 * i + 3]) << 16);
     return make_uint4(b[0], b[1], b[2], b[3]);
 }
 

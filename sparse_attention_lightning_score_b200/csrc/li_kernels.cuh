@@ -24,6 +24,7 @@ struct StreamArgs {
     int tiles_per_cta;      // set by the launcher
     uint32_t* hist;         // optional: [B, LI_HIST_BINS] counts of order_key(score) >> LI_HIST_SHIFT are
                             // added to it (the caller provides it zeroed)
+    int w_bulk;             // FP8: w is 16-byte aligned, so its rows can come in by bulk copy
     DevErr err;
 };
 li_status launch_stream_score_fp8(const CUtensorMap& map, const StreamArgs& args, int batch, int ntiles_max,

@@ -187,14 +187,17 @@ __global__ void __launch_bounds__(L8_THREADS, 2) latent8_score_kernel(const __gr
         for (int u = 0; u < 3; ++u) {  // 16 elements (two raw vectors) -> one 16-byte chunk of e4m3
             const uint32_t wv[8] = {raw[2 * u].x, raw[2 * u].y, raw[2 * u].z, raw[2 * u].w,
                                     raw[2 * u + 1].x, raw[2 * u + 1].y, raw[2 * u + 1].z, raw[2 * u + 1].w};
+            float xe[16], ye[16];
+#pragma unroll
+            for (int x = 0; x < 8; ++x) {
+                xe[2 * x] = __uint_as_float(wv[x] << 16);
+                xe[2 * x + 1] = __uint_as_float(wv[x] & 0xffff0000u);
+            }
+            quotients_for_e4m3<16>(xe, sq, r, ye);
             uint32_t pk[4];
 #pragma unroll
-            for (int x = 0; x < 4; ++x) {
-                const float e0 = __uint_as_float(wv[2 * x] << 16), e1 = __uint_as_float(wv[2 * x] & 0xffff0000u);
-                const float e2 = __uint_as_float(wv[2 * x + 1] << 16), e3 = __uint_as_float(wv[2 * x + 1] & 0xffff0000u);
-                pk[x] = e4m3x2(quotient_for_e4m3(e0, sq, r), quotient_for_e4m3(e1, sq, r)) |
-                        (e4m3x2(quotient_for_e4m3(e2, sq, r), quotient_for_e4m3(e3, sq, r)) << 16);
-            }
+            for (int x = 0; x < 4; ++x)
+                pk[x] = e4m3x2(ye[4 * x], ye[4 * x + 1]) | (e4m3x2(ye[4 * x + 2], ye[4 * x + 3]) << 16);
             const int gch = 3 * l4 + u;  // 16-byte chunk of the 192-byte row
             *reinterpret_cast<uint4*>(qsm + (gch >> 2) * L8_QBLK_BYTES + sw64_offset(j, gch & 3)) =
                 make_uint4(pk[0], pk[1], pk[2], pk[3]);

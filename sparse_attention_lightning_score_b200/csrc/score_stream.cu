@@ -120,10 +120,11 @@ __global__ void __launch_bounds__(StreamCfg<FP8, KBLK, STAGES, NACC, HIST>::THRE
     float qw[FP8 ? QIT : 1];
     if constexpr (FP8) {
         if (threadIdx.x == 0) {
-            mbar_arrive_expect_tx(qload, QROW_BYTES);
+            mbar_arrive_expect_tx(qload, QROW_BYTES + (a.w_bulk ? C::H * 4 : 0));
             bulk_load(qstage, reinterpret_cast<const uint8_t*>(a.q) + (size_t)b * QROW_BYTES, QROW_BYTES, qload);
+            if (a.w_bulk) bulk_load(wsm, a.w + (size_t)b * C::H, C::H * 4, qload);  // head weights into wsm
         }
-        if (warp >= 2) {
+        if (warp >= 2 && !a.w_bulk) {
             const int ew = (threadIdx.x - 64) >> 5;
             const int g8 = lane >> 3;
 #pragma unroll
@@ -219,7 +220,7 @@ __global__ void __launch_bounds__(StreamCfg<FP8, KBLK, STAGES, NACC, HIST>::THRE
                 float sq;
                 const uint4 packed = quantize_head128_g8(qraw[i][0], qraw[i][1], &sq);
                 *reinterpret_cast<uint4*>(qsm + sw128_offset(j, l8)) = packed;
-                if (l8 == 0) wsm[j] = qw[i] * sq;
+                if (l8 == 0) wsm[j] = (a.w_bulk ? wsm[j] : qw[i]) * sq;
             }
         } else {
             constexpr int CH = KBLK * 8;                // 16-byte chunks per query row

@@ -50,7 +50,11 @@ __global__ void __launch_bounds__(256) quantize_query_kernel(const __nv_bfloat16
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         s = m > 0.f ? __fdiv_rn(m, 448.f) : 1.f;
         const float r = __frcp_rn(s);
-        for (int e = lane; e < dim; e += 32) q8[gw * dim + e] = (uint8_t)e4m3_quotient(__bfloat162float(src[e]), s, r);
+        for (int e0 = 0; e0 < dim; e0 += 32) {  // uniform trip count: the quotient votes across the warp
+            const int e = e0 + lane;
+            const uint32_t b = e4m3_quotient(e < dim ? __bfloat162float(src[e]) : 0.f, s, r);
+            if (e < dim) q8[gw * dim + e] = (uint8_t)b;
+        }
     }
     if (lane == 0) {
         sq[gw] = s;
