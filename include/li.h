@@ -101,6 +101,11 @@ typedef struct {
     li_dtype q_dtype;  /* LI_DTYPE_BF16: quantised per (row, head) as li_quantize_query, FP8 tensor cores.
                           LI_DTYPE_F32 : exact fp32 scalar path (k_dtype must be LI_DTYPE_F32). */
     li_dtype k_dtype;  /* LI_DTYPE_E4M3 (k_scale required) or LI_DTYPE_F32 (k_scale NULL) */
+    int tokens_per_request; /* decode with T query tokens per request (multi-token prediction), 0 or 1 = one.
+                          Rows = requests * T; row r is token r % T of request r / T, reads that
+                          request's cache (cache_batch_rows, len[] and the histogram's row count are
+                          per request) and sees positions s < len[r / T] - (T - 1 - r % T): the
+                          request's newest T tokens are its last T cache positions.  FP8 decode only. */
 } li_score_desc;
 
 /* Scores every visible cache position of every row:
@@ -182,14 +187,15 @@ size_t li_decode_select_workspace(const li_score_desc* desc);
  *   as +0.0).  hist: [rows, 2048] uint32, 16-byte aligned, zero before the
  *   call; it is added to, not overwritten.
  * li_topk_hist: li_topk (causal 0) that takes its first digit from hist and
- *   leaves hist all zero.  The result equals li_topk's for any hist.  When hist
+ *   leaves hist all zero.  tokens_per_request as in li_score_desc (len per
+ *   request, rows = requests * T).  The result equals li_topk's for any hist.  When hist
  *   does not count exactly the row's scores, the call reports LI_ERR_BOUNDS
  *   through li_get_last_error and selects without it. */
 li_status li_decode_score_hist(const void* q, const float* w, const void* k, const float* k_scale,
                                int64_t cache_batch_rows, const int32_t* len, float* scores, int64_t scores_ld,
                                const li_score_desc* desc, uint32_t* hist, li_stream_t stream);
 li_status li_topk_hist(const float* scores, int64_t scores_ld, const int32_t* len, int rows, int max_len, int k,
-                       int32_t* idx, float* vals, uint32_t* hist, li_stream_t stream);
+                       int32_t* idx, float* vals, uint32_t* hist, int tokens_per_request, li_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* LatentIndex: decoder absorption and latent-cache scoring                  */

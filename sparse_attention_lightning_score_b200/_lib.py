@@ -24,7 +24,7 @@ sz = ctypes.c_size_t
 
 class ScoreDesc(ctypes.Structure):
     _fields_ = [("rows", i32), ("heads", i32), ("dim", i32), ("max_len", i32), ("causal", i32),
-                ("causal_offset", i32), ("q_dtype", i32), ("k_dtype", i32)]
+                ("causal_offset", i32), ("q_dtype", i32), ("k_dtype", i32), ("tokens_per_request", i32)]
 
 
 # name -> (restype, argtypes); every symbol declared in include/li.h
@@ -39,7 +39,7 @@ SIGNATURES = {
                                vp]),
     "li_decode_select_workspace": (sz, [ctypes.POINTER(ScoreDesc)]),
     "li_decode_score_hist": (i32, [vp, vp, vp, vp, i64, vp, vp, i64, ctypes.POINTER(ScoreDesc), vp, vp]),
-    "li_topk_hist": (i32, [vp, i64, vp, i32, i32, i32, vp, vp, vp, vp]),
+    "li_topk_hist": (i32, [vp, i64, vp, i32, i32, i32, vp, vp, vp, i32, vp]),
     "li_absorb_query": (i32, [vp, vp, vp, i32, i32, i32, i32, vp]),
     "li_latent_score": (i32, [vp, vp, vp, i64, vp, vp, i64, i32, i32, i32, i32, vp]),
     "li_latent_score_hist": (i32, [vp, vp, vp, i64, vp, vp, i64, i32, i32, i32, i32, vp, vp]),

@@ -59,14 +59,15 @@ def li_quantize_query(q: torch.Tensor, w: Optional[torch.Tensor] = None, stream=
 
 
 def score_desc(rows, heads, dim, max_len, causal=False, causal_offset=0, q_dtype=_lib.LI_DTYPE_BF16,
-               k_dtype=_lib.LI_DTYPE_E4M3) -> ScoreDesc:
+               k_dtype=_lib.LI_DTYPE_E4M3, tokens_per_request=1) -> ScoreDesc:
     return ScoreDesc(int(rows), int(heads), int(dim), int(max_len), int(bool(causal)), int(causal_offset),
-                     int(q_dtype), int(k_dtype))
+                     int(q_dtype), int(k_dtype), int(tokens_per_request))
 
 
 def li_index_score(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, k_scale: Optional[torch.Tensor] = None, *,
                    lens: Optional[torch.Tensor] = None, causal: bool = False, causal_offset: int = 0,
-                   scores: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None, stream=None):
+                   scores: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                   tokens_per_request: int = 1, stream=None):
     """DSA lightning-indexer scores.
 
     q: [R,H,d] bf16 (FP8 tensor-core path, k uint8/float8_e4m3fn + k_scale) or fp32
@@ -88,7 +89,7 @@ def li_index_score(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, k_scale: O
         _need(k_scale, "k_scale", torch.float32)
     if lens is not None:
         _need(lens, "lens", torch.int32)
-    desc = score_desc(R, H, d, L, causal, causal_offset, qd, kd)
+    desc = score_desc(R, H, d, L, causal, causal_offset, qd, kd, tokens_per_request)
     lib = _lib.load()
     if scores is None:
         scores = torch.empty((R, _round4(L)), dtype=torch.float32, device=q.device)
@@ -132,7 +133,7 @@ def li_decode_select_workspace(rows: int, device) -> torch.Tensor:
 def li_decode_select(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, k_scale: torch.Tensor, k_top: int, *,
                      lens: Optional[torch.Tensor] = None, scores: Optional[torch.Tensor] = None,
                      workspace: Optional[torch.Tensor] = None, with_values: bool = False, idx=None, vals=None,
-                     stream=None):
+                     tokens_per_request: int = 1, stream=None):
     """Decode score + top-k in one call -> (scores, idx[, vals]).
 
     Same arguments as li_index_score's decode form (q bf16 [B,64,128], k e4m3 [B,L,128] or [L,128],
@@ -150,7 +151,7 @@ def li_decode_select(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, k_scale:
     batch_rows = k.shape[1] if k.dim() == 3 else 0
     if lens is not None:
         _need(lens, "lens", torch.int32)
-    desc = score_desc(R, H, d, L)
+    desc = score_desc(R, H, d, L, tokens_per_request=tokens_per_request)
     lib = _lib.load()
     if scores is None:
         scores = torch.empty((R, _round4(L)), dtype=torch.float32, device=q.device)
@@ -170,7 +171,7 @@ def li_decode_select(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, k_scale:
 
 def li_decode_score_hist(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, k_scale: torch.Tensor,
                          hist: torch.Tensor, *, lens: Optional[torch.Tensor] = None,
-                         scores: Optional[torch.Tensor] = None, stream=None):
+                         scores: Optional[torch.Tensor] = None, tokens_per_request: int = 1, stream=None):
     """First half of li_decode_select: decode scores, plus counts added to `hist` (a zeroed
     li_decode_select_workspace buffer)."""
     _need(q, "q", torch.bfloat16)
@@ -186,7 +187,7 @@ def li_decode_score_hist(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, k_sc
         _need(lens, "lens", torch.int32)
     if scores is None:
         scores = torch.empty((R, _round4(L)), dtype=torch.float32, device=q.device)
-    desc = score_desc(R, H, d, L)
+    desc = score_desc(R, H, d, L, tokens_per_request=tokens_per_request)
     st = _lib.load().li_decode_score_hist(_ptr(q), _ptr(w), _ptr(k), _ptr(k_scale), batch_rows, _ptr(lens),
                                           _ptr(scores), scores.stride(0), ctypes.byref(desc), _ptr(hist),
                                           _stream(stream))
@@ -195,7 +196,8 @@ def li_decode_score_hist(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, k_sc
 
 
 def li_topk_hist(scores: torch.Tensor, k: int, hist: torch.Tensor, *, lens: Optional[torch.Tensor] = None,
-                 max_len: Optional[int] = None, with_values: bool = False, idx=None, vals=None, stream=None):
+                 max_len: Optional[int] = None, with_values: bool = False, idx=None, vals=None,
+                 tokens_per_request: int = 1, stream=None):
     """Second half of li_decode_select: li_topk using (and clearing) the scorer's histogram."""
     _need(scores, "scores", torch.float32)
     rows, ld = scores.shape
@@ -208,7 +210,8 @@ def li_topk_hist(scores: torch.Tensor, k: int, hist: torch.Tensor, *, lens: Opti
     if with_values and vals is None:
         vals = torch.empty((rows, k), dtype=torch.float32, device=scores.device)
     st = _lib.load().li_topk_hist(_ptr(scores), ld, _ptr(lens), rows, int(max_len), int(k), _ptr(idx),
-                                  _ptr(vals) if with_values else None, _ptr(hist), _stream(stream))
+                                  _ptr(vals) if with_values else None, _ptr(hist), int(tokens_per_request),
+                                  _stream(stream))
     _lib.check("li_topk_hist", st)
     return (idx, vals) if with_values else idx
 

@@ -164,6 +164,9 @@ li_status li_index_score(const void* q, const float* w, const void* k, const flo
     if (!q || !w || !k || !scores || scores_ld < d.max_len) return LI_ERR_INVALID_ARG;
     if (d.causal && (cache_batch_rows != 0 || len)) return LI_ERR_INVALID_ARG;
     if (d.causal && (d.causal_offset < 0)) return LI_ERR_INVALID_ARG;
+    const int T = d.tokens_per_request > 1 ? d.tokens_per_request : 1;
+    if (d.rows % T != 0) return LI_ERR_INVALID_ARG;
+    if (T > 1 && (d.causal || d.q_dtype != LI_DTYPE_BF16)) return LI_ERR_UNSUPPORTED;  // multi-token: FP8 decode
     DevErr e;
     if (ready(&e) != LI_OK) return LI_ERR_CUDA;
 
@@ -177,7 +180,7 @@ li_status li_index_score(const void* q, const float* w, const void* k, const flo
     if (!k_scale) return LI_ERR_INVALID_ARG;
     if (d.heads != 64 || d.dim != 128) return LI_ERR_UNSUPPORTED;
     if (!aligned(k, 16) || !aligned(q, 16)) return LI_ERR_INVALID_ARG;
-    const uint64_t total_rows = cache_batch_rows > 0 ? (uint64_t)(d.rows - 1) * cache_batch_rows + d.max_len
+    const uint64_t total_rows = cache_batch_rows > 0 ? (uint64_t)(d.rows / T - 1) * cache_batch_rows + d.max_len
                                                      : (uint64_t)d.max_len;
     if (total_rows >= (1ull << 31)) return LI_ERR_UNSUPPORTED;
     CUtensorMap kmap;
@@ -194,6 +197,7 @@ li_status li_index_score(const void* q, const float* w, const void* k, const flo
         a.batch_rows = cache_batch_rows;
         a.max_len = d.max_len;
         a.w_bulk = aligned(w, 16) ? 1 : 0;
+        a.tokens = T;
         a.err = e;
         const int ntiles = (d.max_len + 127) / 128;
         return launch_stream_score_fp8(kmap, a, d.rows, ntiles, stream);
@@ -223,7 +227,7 @@ li_status li_topk(const float* scores, int64_t scores_ld, const int32_t* len, in
     DevErr e;
     if (ready(&e) != LI_OK) return LI_ERR_CUDA;
     TopkArgs a{scores, scores_ld, len, rows, max_len, causal ? 1 : 0, causal_offset, k, idx, vals, nullptr, 0, 1,
-                nullptr, 0, e};
+                nullptr, 0, 1, e};
     return launch_topk(a, stream);
 }
 
@@ -244,9 +248,11 @@ li_status li_decode_score_hist(const void* q, const float* w, const void* k, con
     if (d.heads != 64 || d.dim != 128) return LI_ERR_UNSUPPORTED;
     if (!q || !w || !k || !k_scale || !scores || !hist || scores_ld < d.max_len) return LI_ERR_INVALID_ARG;
     if (!aligned(k, 16) || !aligned(q, 16) || !aligned(hist, 16)) return LI_ERR_INVALID_ARG;
+    const int T = d.tokens_per_request > 1 ? d.tokens_per_request : 1;
+    if (d.rows % T != 0) return LI_ERR_INVALID_ARG;
     DevErr e;
     if (ready(&e) != LI_OK) return LI_ERR_CUDA;
-    const uint64_t total_rows = cache_batch_rows > 0 ? (uint64_t)(d.rows - 1) * cache_batch_rows + d.max_len
+    const uint64_t total_rows = cache_batch_rows > 0 ? (uint64_t)(d.rows / T - 1) * cache_batch_rows + d.max_len
                                                      : (uint64_t)d.max_len;
     if (total_rows >= (1ull << 31)) return LI_ERR_UNSUPPORTED;
     CUtensorMap kmap;
@@ -262,12 +268,15 @@ li_status li_decode_score_hist(const void* q, const float* w, const void* k, con
     a.max_len = d.max_len;
     a.hist = hist;
     a.w_bulk = aligned(w, 16) ? 1 : 0;
+    a.tokens = T;
     a.err = e;
     return launch_stream_score_fp8_hist(kmap, a, d.rows, (d.max_len + 127) / 128, stream);
 }
 
 li_status li_topk_hist(const float* scores, int64_t scores_ld, const int32_t* len, int rows, int max_len, int k,
-                       int32_t* idx, float* vals, uint32_t* hist, li_stream_t stream) {
+                       int32_t* idx, float* vals, uint32_t* hist, int tokens_per_request, li_stream_t stream) {
+    const int T = tokens_per_request > 1 ? tokens_per_request : 1;
+    if (rows % T != 0) return LI_ERR_INVALID_ARG;
     if (rows < 0 || max_len < 0 || k < 1 || k > LI_TOPK_MAX_LEN || max_len > LI_TOPK_MAX_LEN) return LI_ERR_INVALID_ARG;
     if (rows == 0) return LI_OK;
     if (!idx || !hist || (!scores && max_len > 0) || scores_ld < max_len || (scores_ld % 4) != 0)
@@ -275,7 +284,7 @@ li_status li_topk_hist(const float* scores, int64_t scores_ld, const int32_t* le
     if ((scores && !aligned(scores, 16)) || !aligned(hist, 16)) return LI_ERR_INVALID_ARG;
     DevErr e;
     if (ready(&e) != LI_OK) return LI_ERR_CUDA;
-    TopkArgs a{scores, scores_ld, len, rows, max_len, 0, 0, k, idx, vals, nullptr, 0, 1, hist, 0, e};
+    TopkArgs a{scores, scores_ld, len, rows, max_len, 0, 0, k, idx, vals, nullptr, 0, 1, hist, 0, T, e};
     return launch_topk(a, stream);
 }
 
@@ -292,6 +301,7 @@ li_status li_decode_select(const void* q, const float* w, const void* k, const f
     if (d.heads != 64 || d.dim != 128) return LI_ERR_UNSUPPORTED;
     if (!idx || !workspace || workspace_bytes < li_decode_select_workspace(&d) || !aligned(workspace, 256))
         return LI_ERR_INVALID_ARG;
+    if (d.tokens_per_request > 1 && d.rows % d.tokens_per_request != 0) return LI_ERR_INVALID_ARG;
     if (d.max_len > 0) {
         if (!q || !w || !k || !k_scale || !scores || scores_ld < d.max_len || (scores_ld % 4) != 0)
             return LI_ERR_INVALID_ARG;
@@ -301,7 +311,8 @@ li_status li_decode_select(const void* q, const float* w, const void* k, const f
     const li_status s = li_decode_score_hist(q, w, k, k_scale, cache_batch_rows, len, scores, scores_ld, desc, hist,
                                              stream);
     if (s != LI_OK) return s;
-    return li_topk_hist(scores, d.max_len > 0 ? scores_ld : 4, len, d.rows, d.max_len, k_top, idx, vals, hist, stream);
+    return li_topk_hist(scores, d.max_len > 0 ? scores_ld : 4, len, d.rows, d.max_len, k_top, idx, vals, hist,
+                        d.tokens_per_request, stream);
 }
 
 li_status li_absorb_query_layers(const void* q_bf16, const void* w_dec_bf16, void* q_tilde_bf16, int layers,
@@ -419,7 +430,8 @@ li_status li_hs_refine(const void* c_bf16, int64_t cache_batch_rows, int64_t cac
     DevErr e;
     if (ready(&e) != LI_OK) return LI_ERR_CUDA;
     if (n_cand == 0) {
-        TopkArgs t{nullptr, 4, nullptr, followers * batch, 0, 0, 0, k, out_idx, nullptr, nullptr, 0, 1, nullptr, 0, e};
+        TopkArgs t{nullptr, 4, nullptr, followers * batch, 0, 0, 0, k, out_idx, nullptr, nullptr, 0, 1, nullptr, 0, 1,
+                   e};
         return launch_topk(t, stream);
     }
     if (!c_bf16 || !cand || !q_tilde_bf16 || !w || !aligned(c_bf16, 16) || !aligned(q_tilde_bf16, 16))
@@ -432,7 +444,7 @@ li_status li_hs_refine(const void* c_bf16, int64_t cache_batch_rows, int64_t cac
     li_status s = launch_hs_rescore(h, stream);
     if (s != LI_OK) return s;
     TopkArgs t{sc, ldw, nullptr, followers * batch, n_cand, 0, 0, k, out_idx, nullptr, cand, n_cand, batch,
-               nullptr, 0, e};
+               nullptr, 0, 1, e};
     return launch_topk(t, stream);
 }
 

@@ -25,6 +25,8 @@ struct StreamArgs {
     uint32_t* hist;         // optional: [B, LI_HIST_BINS] counts of order_key(score) >> LI_HIST_SHIFT are
                             // added to it (the caller provides it zeroed)
     int w_bulk;             // FP8: w is 16-byte aligned, so its rows can come in by bulk copy
+    int tokens;             // query rows per request (multi-token decode; >= 1): row r belongs to request
+                            // r / tokens and sees len - (tokens - 1 - r % tokens) positions of its cache
     DevErr err;
 };
 li_status launch_stream_score_fp8(const CUtensorMap& map, const StreamArgs& args, int batch, int ntiles_max,
@@ -103,6 +105,7 @@ struct TopkArgs {
     // digit from it and leaves it all zero
     uint32_t* hist;
     int cand_cap;           // set by the launcher: candidate keys one CTA can hold
+    int tokens;             // query rows per request, as for the scorer (0 or 1: one row per len entry)
     DevErr err;
 };
 li_status launch_topk(const TopkArgs& a, cudaStream_t st);

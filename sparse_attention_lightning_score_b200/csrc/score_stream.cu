@@ -131,11 +131,16 @@ __global__ void __launch_bounds__(StreamCfg<FP8, KBLK, STAGES, NACC, HIST>::THRE
             for (int i = 0; i < QIT; ++i) qw[i] = __ldg(a.w + (size_t)b * C::H + QHPW * ew + 4 * i + g8);
         }
     }
-    int len_b = a.len ? __ldg(a.len + b) : a.max_len;
+    // multi-token decode: row b is token b % tokens of request b / tokens, which sees its request's
+    // cache up to len - (tokens - 1 - b % tokens)
+    const int tokens = a.tokens > 1 ? a.tokens : 1;
+    const int req = b / tokens;
+    int len_b = a.len ? __ldg(a.len + req) : a.max_len;
     if (len_b < 0 || len_b > a.max_len) {
         if (threadIdx.x == 0 && blockIdx.x == 0) record_error(a.err, ERRBIT_BOUNDS);
         len_b = len_b < 0 ? 0 : a.max_len;
     }
+    len_b = max(0, len_b - (tokens - 1 - b % tokens));
     const int ntiles = (len_b + C::M - 1) / C::M;
     const int t0 = blockIdx.x * a.tiles_per_cta;
     const int nt = min(t0 + a.tiles_per_cta, ntiles) - t0;
@@ -146,7 +151,7 @@ __global__ void __launch_bounds__(StreamCfg<FP8, KBLK, STAGES, NACC, HIST>::THRE
         if (lane == 0) {
             tma_prefetch_desc(&kmap);
             const uint64_t pol = l2_policy_evict_first();
-            const long long rowbase = (long long)b * a.batch_rows;
+            const long long rowbase = (long long)req * a.batch_rows;
             int stage = 0;
             uint32_t ph = 0;
             bool ok = true;
@@ -253,7 +258,7 @@ __global__ void __launch_bounds__(StreamCfg<FP8, KBLK, STAGES, NACC, HIST>::THRE
 
         // ------------------------------------------------------------ epilogue
         const int g = warp & 3;  // TMEM lane quarter this warp may access
-        const long long srow = (long long)b * a.batch_rows;
+        const long long srow = (long long)req * a.batch_rows;
         float* out = a.scores + (size_t)b * a.scores_ld;
         for (int it = 0; it < nt; ++it) {
             const int acc = it % NACC;

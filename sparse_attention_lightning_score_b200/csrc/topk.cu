@@ -190,9 +190,12 @@ __global__ void __launch_bounds__(NT) topk_kernel(const TopkArgs a, int row0, in
     const int c = blockIdx.x;  // == cluster rank: the cluster spans gridDim.x
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
-    long long nl = a.causal ? (long long)r + 1 + a.causal_offset : (a.len ? (long long)__ldg(a.len + r) : a.max_len);
+    const int tokens = a.tokens > 1 ? a.tokens : 1;  // multi-token decode: rows per len entry
+    long long nl = a.causal ? (long long)r + 1 + a.causal_offset
+                            : (a.len ? (long long)__ldg(a.len + r / tokens) : a.max_len);
     if (!a.causal && a.len && (nl < 0 || nl > a.max_len) && c == 0 && threadIdx.x == 0) record_error(a.err, ERRBIT_BOUNDS);
     nl = nl < 0 ? 0 : (nl > a.max_len ? a.max_len : nl);
+    if (!a.causal) nl = nl - (tokens - 1 - r % tokens) < 0 ? 0 : nl - (tokens - 1 - r % tokens);
     const int n = (int)nl;
     const int k = a.k;
     const int base = c * chunk;

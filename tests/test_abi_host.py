@@ -119,3 +119,17 @@ def test_latent_fp8_and_layers_reject_bad_arguments_on_host():
     assert lib.li_absorb_query_layers(p, p, p, -1, 1, 64, 128, 256, None) == _lib.LI_ERR_INVALID_ARG
     assert lib.li_absorb_query_layers(p, p, p, 2, 1, 64, 128, 100, None) == _lib.LI_ERR_INVALID_ARG
     assert lib.li_absorb_query_layers(p, p, p, 0, 1, 64, 128, 256, None) == _lib.LI_OK
+
+
+def test_multi_token_descriptor_checked_on_host():
+    lib = _lib.load()
+    p = ctypes.c_void_p(256)
+    d = _lib.ScoreDesc(6, 64, 128, 100, 0, 0, _lib.LI_DTYPE_BF16, _lib.LI_DTYPE_E4M3, 4)  # 6 rows, 4 tokens
+    assert lib.li_index_score(p, p, p, p, 0, None, p, 100, ctypes.byref(d), None, 0, None) == _lib.LI_ERR_INVALID_ARG
+    ws = lib.li_decode_select_workspace(ctypes.byref(d))
+    assert lib.li_decode_select(p, p, p, p, 0, None, p, 100, ctypes.byref(d), 8, p, None, p, ws,
+                                None) == _lib.LI_ERR_INVALID_ARG
+    c = _lib.ScoreDesc(8, 64, 128, 100, 1, 0, _lib.LI_DTYPE_BF16, _lib.LI_DTYPE_E4M3, 2)   # causal with 2 tokens
+    assert lib.li_index_score(p, p, p, p, 0, None, p, 100, ctypes.byref(c), p, 1 << 20,
+                              None) == _lib.LI_ERR_UNSUPPORTED
+    assert lib.li_topk_hist(p, 100, None, 6, 100, 8, p, None, p, 4, None) == _lib.LI_ERR_INVALID_ARG

@@ -125,3 +125,53 @@ def test_decode_select_dirty_workspace_is_reported_and_healed():
     got = api.li_decode_select(q, w, k8, ks, 2048, lens=ln, workspace=ws, with_values=True)
     _assert_same(got, _two_calls(q, w, k8, ks, ln, 2048), ln)
     assert api.li_get_last_error() == LI_OK
+
+
+# ---------------------------------------------------------------------------
+# multi-token decode: T query tokens per request share the request's cache
+# ---------------------------------------------------------------------------
+def _mtp_case(B, T, L, lens, seed):
+    case = synth.dsa_decode(B=B, L=L, seed=seed, lens=lens)
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(B * T, 64, 128, generator=g).to(torch.bfloat16)
+    w = torch.randn(B * T, 64, generator=g) * 0.1
+    return case, q, w
+
+
+@pytest.mark.parametrize("B,T,L,lens", [(4, 2, 5000, [5000, 3000, 2, 1]), (2, 4, 32768, None),
+                                        (3, 3, 2100, [2100, 2049, 2050])])
+def test_multi_token_decode_matches_per_token_calls(B, T, L, lens):
+    case, q, w = _mtp_case(B, T, L, lens, seed=60 + T)
+    k8, ks, ln = case.k8.to(DEV), case.ks.to(DEV), case.lens.to(DEV)
+    qd, wd = q.to(DEV), w.to(DEV)
+    sc, idx, vals = api.li_decode_select(qd, wd, k8, ks, 2048, lens=ln, tokens_per_request=T, with_values=True)
+    sc2 = api.li_index_score(qd, wd, k8, ks, lens=ln, tokens_per_request=T)
+    for t in range(T):
+        rows = [b * T + t for b in range(B)]
+        lt = torch.clamp(case.lens - (T - 1 - t), min=0).to(DEV)
+        sc_t, idx_t, vals_t = api.li_decode_select(qd[rows].contiguous(), wd[rows].contiguous(), k8, ks, 2048,
+                                                   lens=lt, with_values=True)
+        for i, b in enumerate(rows):
+            n = int(lt[i])
+            assert np.array_equal(_np(sc[b, :n]).view(np.uint32), _np(sc_t[i, :n]).view(np.uint32)), (t, b)
+            assert np.array_equal(_np(sc2[b, :n]).view(np.uint32), _np(sc_t[i, :n]).view(np.uint32)), (t, b)
+        assert np.array_equal(_np(idx[rows]), _np(idx_t)), t
+        assert np.array_equal(_np(vals[rows]).view(np.uint32), _np(vals_t).view(np.uint32)), t
+    assert api.li_get_last_error() == LI_OK
+
+
+def test_multi_token_decode_against_oracle():
+    B, T, L = 2, 3, 4000
+    case, q, w = _mtp_case(B, T, L, [4000, 2500], seed=66)
+    sc, idx = api.li_decode_select(q.to(DEV), w.to(DEV), case.k8.to(DEV), case.ks.to(DEV), 512,
+                                   lens=case.lens.to(DEV), tokens_per_request=T)
+    q8, sq, _ = oracle.quantize_query(q, w.numpy())
+    for t in range(T):
+        rows = [b * T + t for b in range(B)]
+        lt = np.maximum(case.lens.numpy() - (T - 1 - t), 0)
+        ref, mag = oracle.index_score(q8[rows], oracle.E4M3, w[rows], case.k8, oracle.E4M3, q_scale=sq[rows],
+                                      k_scale=case.ks, k_batch_rows=L, L=L, lens=lt, with_mag=True)
+        assert_scores_close(_np(sc)[rows, :L], ref, mag, 1e-2, visible=np.isfinite(ref))
+        ridx, _ = oracle.topk(ref, 512, lens=lt)
+        assert_topk_equivalent(_np(idx)[rows], ridx, ref, 1e-2, n_valid=lt)
+    assert api.li_get_last_error() == LI_OK
