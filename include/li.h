@@ -198,6 +198,31 @@ li_status li_topk_hist(const float* scores, int64_t scores_ld, const int32_t* le
                        int32_t* idx, float* vals, uint32_t* hist, int tokens_per_request, li_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* One long context split along L over several shards (GPUs)                */
+/* ------------------------------------------------------------------------ */
+/* Merges per-shard selections into the global top-k.  Each request's cache
+ * is cut into `shards` consecutive slices of shard_len positions; shard p
+ * selected the k best of its slice (li_decode_select or li_topk with values,
+ * positions local to the slice).  The global top-k is the top-k of the union
+ * of those candidates: a position among the k best of the whole cache is
+ * among the k best of its own slice.  Order and ties are those of li_topk over
+ * global positions (p * shard_len + local).
+ *   vals [shards, rows, k] fp32 and idx [shards, rows, k] int32: the shards'
+ *        outputs stacked in shard order (as an all-gather delivers them)
+ *   out_idx [rows, k_out] int32 (global positions, ascending, -1 pads),
+ *   out_vals [rows, k_out] fp32 (nullable)
+ *   workspace  li_merge_shards_workspace(shards, rows, k) bytes, 256-byte aligned
+ * shards * k <= LI_TOPK_MAX_LEN and shards * shard_len < 2^31.  Each shard's
+ * list must hold its valid positions first; a request whose lists leave a
+ * valid candidate after a pad (only possible if a shard other than the last
+ * one the request reaches had fewer than k positions) is reported through
+ * li_get_last_error as LI_ERR_BOUNDS. */
+li_status li_merge_shards(const float* vals, const int32_t* idx, int shards, int rows, int k, int64_t shard_len,
+                          int k_out, int32_t* out_idx, float* out_vals, void* workspace, size_t workspace_bytes,
+                          li_stream_t stream);
+size_t li_merge_shards_workspace(int shards, int rows, int k);
+
+/* ------------------------------------------------------------------------ */
 /* LatentIndex: decoder absorption and latent-cache scoring                  */
 /* ------------------------------------------------------------------------ */
 /* Absorbs one layer's key decoder into its queries (LatentIndex abstract,

@@ -216,6 +216,29 @@ def li_topk_hist(scores: torch.Tensor, k: int, hist: torch.Tensor, *, lens: Opti
     return (idx, vals) if with_values else idx
 
 
+def li_merge_shards(vals: torch.Tensor, idx: torch.Tensor, shard_len: int, k_out: int, *,
+                    with_values: bool = False, out_idx=None, out_vals=None, workspace=None, stream=None):
+    """Global top-k from per-shard selections: vals fp32 / idx int32 [shards, rows, k] (local
+    positions, each shard's list ascending then -1) -> out_idx int32 [rows, k_out] of global
+    positions (shard p covers p*shard_len ..) [, out_vals]."""
+    _need(vals, "vals", torch.float32)
+    _need(idx, "idx", torch.int32)
+    P, R, k = vals.shape
+    lib = _lib.load()
+    need = lib.li_merge_shards_workspace(P, R, k)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(int(need), 256), dtype=torch.uint8, device=vals.device)
+    if out_idx is None:
+        out_idx = torch.empty((R, k_out), dtype=torch.int32, device=vals.device)
+    if with_values and out_vals is None:
+        out_vals = torch.empty((R, k_out), dtype=torch.float32, device=vals.device)
+    st = lib.li_merge_shards(_ptr(vals), _ptr(idx), P, R, k, int(shard_len), int(k_out), _ptr(out_idx),
+                             _ptr(out_vals) if with_values else None, _ptr(workspace), workspace.numel(),
+                             _stream(stream))
+    _lib.check("li_merge_shards", st)
+    return (out_idx, out_vals) if with_values else out_idx
+
+
 def li_absorb_query(q: torch.Tensor, w_dec: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None):
     """q bf16 [B,H,d], W_dec bf16 [H,d,dc] -> q~ bf16 [B,H,dc]."""
     _need(q, "q", torch.bfloat16)

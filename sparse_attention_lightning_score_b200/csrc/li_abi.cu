@@ -315,6 +315,36 @@ li_status li_decode_select(const void* q, const float* w, const void* k, const f
                         d.tokens_per_request, stream);
 }
 
+size_t li_merge_shards_workspace(int shards, int rows, int k) {
+    if (shards <= 0 || rows <= 0 || k <= 0) return 0;
+    const size_t ld = align_up((size_t)shards * k, 4);
+    return align_up((size_t)rows * ld * 4, 256) * 2 + align_up((size_t)rows * 4, 256);
+}
+
+li_status li_merge_shards(const float* vals, const int32_t* idx, int shards, int rows, int k, int64_t shard_len,
+                          int k_out, int32_t* out_idx, float* out_vals, void* workspace, size_t workspace_bytes,
+                          li_stream_t stream) {
+    if (shards <= 0 || rows < 0 || k <= 0 || k_out < 1 || k_out > LI_TOPK_MAX_LEN || shard_len <= 0)
+        return LI_ERR_INVALID_ARG;
+    if ((long long)shards * k > LI_TOPK_MAX_LEN || (long long)shards * shard_len >= (1ll << 31))
+        return LI_ERR_INVALID_ARG;
+    if (rows == 0) return LI_OK;
+    if (!vals || !idx || !out_idx || !workspace || !aligned(workspace, 256) ||
+        workspace_bytes < li_merge_shards_workspace(shards, rows, k))
+        return LI_ERR_INVALID_ARG;
+    DevErr e;
+    if (ready(&e) != LI_OK) return LI_ERR_CUDA;
+    const size_t ld = align_up((size_t)shards * k, 4);
+    float* mvals = static_cast<float*>(workspace);
+    int32_t* mpos = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + align_up((size_t)rows * ld * 4, 256));
+    int32_t* mlen = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(mpos) + align_up((size_t)rows * ld * 4, 256));
+    li_status s = launch_merge_prep(vals, idx, shards, rows, k, shard_len, mvals, mpos, mlen, (long long)ld, e, stream);
+    if (s != LI_OK) return s;
+    TopkArgs t{mvals, (long long)ld, mlen, rows, shards * k, 0, 0, k_out, out_idx, out_vals, mpos, (long long)ld, rows,
+               nullptr, 0, 1, e};
+    return launch_topk(t, stream);
+}
+
 li_status li_absorb_query_layers(const void* q_bf16, const void* w_dec_bf16, void* q_tilde_bf16, int layers,
                                  int batch, int heads, int dim, int latent_dim, li_stream_t stream) {
     if (layers < 0 || layers > 65535 || batch < 0 || heads <= 0 || dim <= 0 || dim > 256 || latent_dim <= 0 ||
