@@ -198,6 +198,25 @@ li_status li_topk_hist(const float* scores, int64_t scores_ld, const int32_t* le
                        int32_t* idx, float* vals, uint32_t* hist, int tokens_per_request, li_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Page-locked host buffers used directly by the kernels                    */
+/* ------------------------------------------------------------------------ */
+/* A decode step's inputs and outputs are small (the query and weights in, k
+ * positions per request out).  DMA copies of them cost more in a step than
+ * their size suggests, so a caller may hand the kernels page-locked host
+ * memory instead.
+ * li_host_device_pointer: the device-side address of page-locked host memory
+ *   (cudaHostGetDevicePointer); LI_ERR_INVALID_ARG when host_ptr is not
+ *   page-locked memory mapped for the current device.  The address can be
+ *   given to li_decode_select / li_topk as idx or vals: the kernels then write
+ *   the selections straight into host memory (visible to the host once the
+ *   stream has been synchronised).
+ * li_copy_from_host: copies `bytes` from such a device-side address of host
+ *   memory into device memory with a kernel (both 16-byte aligned), ordered on
+ *   `stream` like any launch. */
+li_status li_host_device_pointer(const void* host_ptr, void** dev_ptr);
+li_status li_copy_from_host(void* dst, const void* src_mapped, size_t bytes, li_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* One long context split along L over several shards (GPUs)                */
 /* ------------------------------------------------------------------------ */
 /* Merges per-shard selections into the global top-k.  Each request's cache

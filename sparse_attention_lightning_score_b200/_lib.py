@@ -44,6 +44,8 @@ SIGNATURES = {
     "li_latent_score": (i32, [vp, vp, vp, i64, vp, vp, i64, i32, i32, i32, i32, vp]),
     "li_latent_score_hist": (i32, [vp, vp, vp, i64, vp, vp, i64, i32, i32, i32, i32, vp, vp]),
     "li_absorb_query_layers": (i32, [vp, vp, vp, i32, i32, i32, i32, i32, vp]),
+    "li_host_device_pointer": (i32, [vp, ctypes.POINTER(ctypes.c_void_p)]),
+    "li_copy_from_host": (i32, [vp, vp, sz, vp]),
     "li_merge_shards": (i32, [vp, vp, i32, i32, i32, i64, i32, vp, vp, vp, sz, vp]),
     "li_merge_shards_workspace": (sz, [i32, i32, i32]),
     "li_latent_score_fp8": (i32, [vp, vp, vp, vp, i64, vp, vp, i64, i32, i32, i32, i32, vp, vp]),

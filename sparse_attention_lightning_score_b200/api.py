@@ -17,7 +17,36 @@ from ._lib import LiError, ScoreDesc  # noqa: F401  (re-exported)
 
 
 def _ptr(t: Optional[torch.Tensor]):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    """Device address of a tensor: a CUDA tensor's own, or for a page-locked host tensor the
+    address the kernels use to reach it (li_host_device_pointer)."""
+    if t is None:
+        return None
+    if t.is_cuda:
+        return ctypes.c_void_p(t.data_ptr())
+    if not t.is_pinned():
+        raise ValueError("host tensors handed to the kernels must be page-locked (pin_memory())")
+    return ctypes.c_void_p(li_host_device_pointer(t))
+
+
+def li_host_device_pointer(t: torch.Tensor) -> int:
+    """Device-side address of a page-locked host tensor (raises if it is not mapped)."""
+    out = ctypes.c_void_p()
+    st = _lib.load().li_host_device_pointer(ctypes.c_void_p(t.data_ptr()), ctypes.byref(out))
+    _lib.check("li_host_device_pointer", st)
+    return int(out.value)
+
+
+def li_copy_from_host(dst: torch.Tensor, src: torch.Tensor, stream=None):
+    """dst (CUDA) <- src (page-locked host, same byte size), copied by a kernel on `stream`."""
+    _need(dst, "dst")
+    if src.is_cuda or not src.is_pinned() or not src.is_contiguous():
+        raise ValueError("src must be a contiguous page-locked host tensor")
+    nbytes = dst.numel() * dst.element_size()
+    if src.numel() * src.element_size() != nbytes:
+        raise ValueError("dst and src differ in size")
+    st = _lib.load().li_copy_from_host(_ptr(dst), _ptr(src), nbytes, _stream(stream))
+    _lib.check("li_copy_from_host", st)
+    return dst
 
 
 def _stream(stream=None):
@@ -157,7 +186,7 @@ def li_decode_select(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, k_scale:
         scores = torch.empty((R, _round4(L)), dtype=torch.float32, device=q.device)
     if workspace is None:
         workspace = li_decode_select_workspace(R, q.device)
-    if idx is None:
+    if idx is None:  # (idx / vals may also be page-locked host tensors: the top-k writes them directly)
         idx = torch.empty((R, k_top), dtype=torch.int32, device=q.device)
     if with_values and vals is None:
         vals = torch.empty((R, k_top), dtype=torch.float32, device=q.device)

@@ -315,6 +315,26 @@ li_status li_decode_select(const void* q, const float* w, const void* k, const f
                         d.tokens_per_request, stream);
 }
 
+li_status li_host_device_pointer(const void* host_ptr, void** dev_ptr) {
+    if (!host_ptr || !dev_ptr) return LI_ERR_INVALID_ARG;
+    *dev_ptr = nullptr;
+    void* p = nullptr;
+    if (cudaHostGetDevicePointer(&p, const_cast<void*>(host_ptr), 0) != cudaSuccess || !p) {
+        cudaGetLastError();
+        return LI_ERR_INVALID_ARG;  // not page-locked memory mapped for this device
+    }
+    *dev_ptr = p;
+    return LI_OK;
+}
+
+li_status li_copy_from_host(void* dst, const void* src_mapped, size_t bytes, li_stream_t stream) {
+    if (bytes == 0) return LI_OK;
+    if (!dst || !src_mapped || !aligned(dst, 16) || !aligned(src_mapped, 16)) return LI_ERR_INVALID_ARG;
+    DevErr e;
+    if (ready(&e) != LI_OK) return LI_ERR_CUDA;
+    return launch_host_copy(dst, src_mapped, bytes, stream);
+}
+
 size_t li_merge_shards_workspace(int shards, int rows, int k) {
     if (shards <= 0 || rows <= 0 || k <= 0) return 0;
     const size_t ld = align_up((size_t)shards * k, 4);

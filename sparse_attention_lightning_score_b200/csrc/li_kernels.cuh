@@ -68,6 +68,9 @@ struct PrefillArgs {
 li_status launch_prefill_score(const CUtensorMap& qmap, const CUtensorMap& kmap, const PrefillArgs& args,
                                cudaStream_t st);
 
+// ---------------------------------------------------------------- copy from mapped host memory
+li_status launch_host_copy(void* dst, const void* src, size_t bytes, cudaStream_t st);
+
 // ---------------------------------------------------------------- query quantiser
 li_status launch_quantize_query(const void* q, const float* w, int rows, int heads, int dim, uint8_t* q8, float* sq,
                                 float* w_eff, cudaStream_t st);

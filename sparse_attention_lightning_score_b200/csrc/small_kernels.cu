@@ -1,5 +1,7 @@
 // Small kernels of the li library: the standalone query quantiser, the exact
 // fp32 scorer, LatentIndex decoder absorption, and the wait self-test.
+#include <algorithm>
+
 #include "li_common.cuh"
 #include "li_kernels.cuh"
 
@@ -197,7 +199,34 @@ __global__ void selftest_wait_kernel(const DevErr e) {
     if (threadIdx.x == 0) (void)mbar_wait(&bar, 0, e);
 }
 
+// ---------------------------------------------------------------------------
+// Copy from page-locked host memory mapped into the device's address space
+// (a decode step's query and weights): PCIe reads issued by many threads, so
+// that the copy is one kernel of the step instead of a separate DMA transfer.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) host_copy_kernel(uint4* __restrict__ dst, const uint4* __restrict__ src,
+                                                        size_t n16, uint8_t* __restrict__ dst_tail,
+                                                        const uint8_t* __restrict__ src_tail, int tail) {
+    pdl_trigger();
+    pdl_wait();  // the destination may still be read by the previous kernel of the stream
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += stride) dst[i] = src[i];
+    if (blockIdx.x == 0 && (int)threadIdx.x < tail) dst_tail[threadIdx.x] = src_tail[threadIdx.x];
+}
+
 }  // namespace
+
+li_status launch_host_copy(void* dst, const void* src, size_t bytes, cudaStream_t st) {
+    if (bytes == 0) return LI_OK;
+    const size_t n16 = bytes / 16;
+    const int tail = (int)(bytes % 16);
+    const int blocks = (int)std::min<size_t>((n16 + 255) / 256 + 1, 2 * (size_t)host_num_sms());
+    if (launch_pdl(host_copy_kernel, dim3(std::max(blocks, 1)), dim3(256), 0, st, 1, static_cast<uint4*>(dst),
+                   static_cast<const uint4*>(src), n16, static_cast<uint8_t*>(dst) + n16 * 16,
+                   static_cast<const uint8_t*>(src) + n16 * 16, tail) != cudaSuccess)
+        return host_check_launch();
+    return host_check_launch();
+}
 
 li_status launch_quantize_query(const void* q, const float* w, int rows, int heads, int dim, uint8_t* q8, float* sq,
                                 float* w_eff, cudaStream_t st) {

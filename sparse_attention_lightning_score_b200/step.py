@@ -10,8 +10,15 @@ buffers once and captures
     H2D copy of (q, w)  ->  li_decode_select (score + top-k)  ->  D2H copy of the indices
 
 as one CUDA graph; each ``step()`` writes the host inputs and replays it.
-Every kernel in the graph is an li kernel; torch only provides the buffers,
-the stream and the copies.
+
+With ``zero_copy`` the transfers are done by the li kernels themselves instead
+of DMA copies: a copy kernel reads the page-locked inputs through their mapped
+device address, and the top-k writes the selected positions straight into the
+page-locked output buffer.  On the B200 boxes measured it was slower than the
+DMA copies (PCIe reads from a kernel are latency-bound), so it is off by
+default.  Every
+kernel in the graph is an li kernel; torch only provides the buffers and the
+stream.
 """
 from __future__ import annotations
 
@@ -31,10 +38,12 @@ class DecodeIndexer:
     the visible length per request.
     """
 
-    def __init__(self, k8: torch.Tensor, ks: torch.Tensor, heads: int, k: int, lens: Optional[torch.Tensor] = None):
+    def __init__(self, k8: torch.Tensor, ks: torch.Tensor, heads: int, k: int, lens: Optional[torch.Tensor] = None,
+                 zero_copy: bool = False):
         if not (k8.is_cuda and ks.is_cuda):
             raise ValueError("the key cache must be resident on a CUDA device")
         self.k8, self.ks, self.lens = k8, ks, lens
+        self.zero_copy = zero_copy
         B, L, d = k8.shape
         self.B, self.L, self.d, self.H, self.k = B, L, d, heads, k
         dev = k8.device
@@ -58,6 +67,11 @@ class DecodeIndexer:
             self._launch()
 
     def _launch(self):
+        if self.zero_copy:
+            api.li_copy_from_host(self.in_dev, self.in_host)
+            api.li_decode_select(self.q_dev, self.w_dev, self.k8, self.ks, self.k, lens=self.lens,
+                                 scores=self.scores, workspace=self.ws, idx=self.idx_host)
+            return
         self.in_dev.copy_(self.in_host, non_blocking=True)
         api.li_decode_select(self.q_dev, self.w_dev, self.k8, self.ks, self.k, lens=self.lens, scores=self.scores,
                              workspace=self.ws, idx=self.idx_dev)

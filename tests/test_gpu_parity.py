@@ -273,4 +273,18 @@ def test_decode_indexer_graph_step():
     got2 = ix.step(case2.q, case2.w).numpy().copy()
     assert_topk_equivalent(got2, ridx2, ref2, 1e-2, n_valid=case.lens.numpy())
     assert ix.h2d_bytes == 3 * 64 * 128 * 2 + 3 * 64 * 4 and ix.d2h_bytes == 3 * 300 * 4
+    # the same steps through DMA copies instead of the kernels' own transfers
+    ix2 = DecodeIndexer(case.k8.to(DEV), case.ks.to(DEV), heads=64, k=300, lens=case.lens.to(DEV), zero_copy=False)
+    assert np.array_equal(ix2.step(case2.q, case2.w).numpy(), got2)
+    assert np.array_equal(ix.step(case.q, case.w).numpy(), got)
+    assert api.li_get_last_error() == LI_OK
+
+
+def test_copy_from_host_kernel():
+    src = torch.arange(1000 * 16 + 7, dtype=torch.uint8).pin_memory()  # a tail that is not 16 bytes
+    dst = torch.zeros(src.numel(), dtype=torch.uint8, device=DEV)
+    api.li_copy_from_host(dst, src)
+    assert torch.equal(dst.cpu(), src)
+    with pytest.raises(ValueError):
+        api.li_copy_from_host(dst, src.clone())  # not page-locked
     assert api.li_get_last_error() == LI_OK
