@@ -84,6 +84,40 @@ def test_quantize_query_near_rounding_midpoints():
     assert_scores_close(_np(sc)[:, :300], ref, mag, 1e-2)
 
 
+def _sweep_heads(absmax_bits):
+    """Heads of 128 bf16 values: per absmax A, element 0 of every head is +-A and the other 127 run
+    through every bf16 value x with |x| <= A, both signs (NaN excluded)."""
+    heads = []
+    for ab in absmax_bits:
+        a = np.array([ab << 16], np.uint32).view(np.float32)[0]
+        mags = (np.arange(0, ab + 1, dtype=np.uint32) << 16).view(np.float32)
+        vals = np.concatenate([mags, -mags])
+        n = -(-vals.size // 127)
+        vals = np.concatenate([vals, np.zeros(n * 127 - vals.size, np.float32)]).reshape(n, 127)
+        first = np.where(np.arange(n) % 2 == 0, a, -a).astype(np.float32)[:, None]
+        heads.append(np.concatenate([first, vals], axis=1))
+    h = np.concatenate(heads)
+    pad = -h.shape[0] % 64
+    h = np.concatenate([h, np.zeros((pad, 128), np.float32)])
+    return torch.from_numpy(h).view(-1, 64, 128).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("absmax_bits", [
+    [0x0b00, 0x1e40, 0x2d07, 0x3a91, 0x3f80, 0x3fe0, 0x40a5, 0x4122, 0x43e0, 0x4661],
+    [0x0080, 0x0100, 0x0d80, 0x3c00, 0x4000, 0x42f3, 0x5555, 0x6a00, 0x7f00, 0x7f7f],
+])
+def test_quantize_query_every_bf16_below_absmax(absmax_bits):
+    # the quantiser's division-free rounding decision against the oracle's IEEE division for every bf16
+    # input below each absmax: subnormal scales, tiny and huge absmax, exact e4m3 rounding midpoints
+    q = _sweep_heads(absmax_bits)
+    w = torch.randn(q.shape[:2], generator=torch.Generator().manual_seed(7))
+    q8_o, sq_o, we_o = oracle.quantize_query(q, w.numpy())
+    q8, sq, we = api.li_quantize_query(q.to(DEV), w.to(DEV))
+    assert np.array_equal(_np(q8), q8_o)
+    assert np.array_equal(_np(sq).view(np.uint32), sq_o.view(np.uint32))
+    assert np.array_equal(_np(we).view(np.uint32), we_o.view(np.uint32))
+
+
 # ---------------------------------------------------------------------------
 # tiny fp32 case: exact scalar path, tolerance 1e-4
 # ---------------------------------------------------------------------------
