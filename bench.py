@@ -186,10 +186,10 @@ def cpu_baseline_sample():
 # ---------------------------------------------------------------------------
 # li arm
 # ---------------------------------------------------------------------------
-def make_sets(dev, Lx, seed):
+def make_sets(dev, Lx, seed, heads=H):
     """Key caches for B requests of length Lx, copied until they exceed 1.5x L2."""
     from sparse_attention_lightning_score_b200 import synth
-    case = synth.dsa_decode(B=B, L=Lx, k_top=KTOP, seed=seed)
+    case = synth.dsa_decode(B=B, L=Lx, H=heads, k_top=KTOP, seed=seed)
     per_set = B * Lx * (D + 4)
     nsets = max(2, math.ceil(1.5 * L2_BYTES / per_set))
     k8 = case.k8.to(dev)
@@ -218,12 +218,13 @@ class DecodeBench:
     into a scratch histogram, the top-k from a saved histogram restored by a
     device copy before each launch (the copy's own time is subtracted)."""
 
-    def __init__(self, dev, Lx, seed):
+    def __init__(self, dev, Lx, seed, heads=H):
         import torch
         from sparse_attention_lightning_score_b200 import api
         self.api = api
         self.Lx = Lx
-        self.case, self.sets, self.set_bytes = make_sets(dev, Lx, seed)
+        self.heads = heads
+        self.case, self.sets, self.set_bytes = make_sets(dev, Lx, seed, heads)
         self.n = len(self.sets)
         self.q, self.w = self.case.q.to(dev), self.case.w.to(dev)
         self.sc = torch.empty((B, Lx), dtype=torch.float32, device=dev)
@@ -508,15 +509,15 @@ class LatentBench:
     """LatentIndex G=4 group decode: 4 x (absorb + latent score + top-2048), B=4, L=65536; each
     layer's scan counts its first radix digit for the top-k.  kind "bf16": the d_c = 256 bf16
     latent cache; kind "fp8_192": DeepSeek-V3.2's 64 RoPE + 128 NoPE latent as an e4m3 cache
-    with per-row scales."""
+    with per-row scales.  heads = 32 gives GLM-5's indexer shape on the bf16 cache."""
 
-    def __init__(self, dev, B=4, Lx=65536, kind="bf16"):
+    def __init__(self, dev, B=4, Lx=65536, kind="bf16", heads=H):
         import torch
         from sparse_attention_lightning_score_b200 import api, synth
         self.api = api
-        self.B, self.L, self.kind = B, Lx, kind
+        self.B, self.L, self.kind, self.heads = B, Lx, kind, heads
         if kind == "bf16":
-            case = synth.latent_group(B=B, L=Lx)
+            case = synth.latent_group(B=B, L=Lx, H=heads)
             self.c = [(case.c.to(dev), None)]
             per = case.c.numel() * 2
             self.dc, self.key_bytes = 256, 512
@@ -532,7 +533,7 @@ class LatentBench:
         self.hist = api.li_decode_select_workspace(B, dev).view(torch.int32)[:B * 2048]
         self.hist_scratch = api.li_decode_select_workspace(B, dev).view(torch.int32)[:B * 2048]
         self.w = [case.w[l].to(dev) for l in range(4)]
-        self.qt = torch.empty((B, H, self.dc), dtype=torch.bfloat16, device=dev)
+        self.qt = torch.empty((B, heads, self.dc), dtype=torch.bfloat16, device=dev)
         self.sc = torch.empty((B, Lx), dtype=torch.float32, device=dev)
         self.idx = torch.empty((4, B, KTOP), dtype=torch.int32, device=dev)
 
@@ -645,7 +646,25 @@ def run_other(args, rank, world, local_rank):
     hbm, which = peaks()
     fp8_burst, fp8_sust, fp8_src = fp8_peak_tflops()
     clocks = ClockSampler(local_rank)
-    if args.workload == "prefill":
+    if args.workload == "glm5_decode":
+        # GLM-5's indexer shape (32 heads, d = 128, FP8 keys) on the decode step of the default workload
+        bx = DecodeBench(dev, L, seed=1, heads=32)
+        bx.build_graphs(args.warmup)
+        clocks.start()
+        time.sleep(0.3)
+        ms = bx.time_steps(args.steps)
+        clk = clocks.stop()
+        sc_ms, tk_ms = bx.time_kernel("score"), bx.time_kernel("topk")
+        algo = B * L * decode_bytes_per_key() + B * 32 * D * 2 + B * 32 * 4
+        out = {"metric": METRIC, "value": B * L / (ms * 1e-3), "unit": "keys/s", "ms_per_step": ms,
+               "us_per_step": ms * 1e3, "higher_is_better": True, "dtype": "e4m3",
+               "config": {"workload": "glm5_decode_b8_l32k", "B": B, "L": L, "H": 32, "d": D, "k": KTOP,
+                          "l2": f"{bx.n} rotating key-cache copies"},
+               "roofline": {"bound": "hbm", "kernel": SCORER_KERNEL, "achieved": algo / (sc_ms * 1e-3) / 1e9,
+                            "peak": hbm, "peak_source": which, "unit": "GB/s",
+                            "frac": algo / (sc_ms * 1e-3) / 1e9 / hbm, "kernel_us": sc_ms * 1e3},
+               "topk": {"us": tk_ms * 1e3}, "gpu_launches": 2 * args.steps, "clocks": clk}
+    elif args.workload == "prefill":
         bx = PrefillBench(dev)
         clocks.start()
         r = bx.run(args.steps, args.warmup)
@@ -660,8 +679,9 @@ def run_other(args, rank, world, local_rank):
                             "frac": achieved / fp8_burst, "frac_of_sustained": achieved / fp8_sust,
                             "score_ms": r["score"]},
                "topk": {"ms": r["topk"], "rows_per_s": bx.T / (r["topk"] * 1e-3)}, "clocks": clk}
-    elif args.workload in ("latent", "latent192"):
-        bx = LatentBench(dev, kind="bf16" if args.workload == "latent" else "fp8_192")
+    elif args.workload in ("latent", "latent192", "latent_glm5"):
+        bx = LatentBench(dev, kind="fp8_192" if args.workload == "latent192" else "bf16",
+                         heads=32 if args.workload == "latent_glm5" else H)
         clocks.start()
         r = bx.run(args.steps, args.warmup)
         clk = clocks.stop()
@@ -671,8 +691,10 @@ def run_other(args, rank, world, local_rank):
         out = {"metric": METRIC, "value": 4 * bx.B * bx.L / (r["step"] * 1e-3), "unit": "keys/s",
                "ms_per_step": r["step"], "us_per_layer": r["step"] * 1e3 / 4, "higher_is_better": True,
                "dtype": "e4m3" if fp8 else "bf16",
-               "config": {"workload": "latent_fp8_dc192_g4_b4_l64k" if fp8 else "latent_g4_b4_l64k", "B": bx.B,
-                          "L": bx.L, "G": 4, "d_c": bx.dc, "k": KTOP, "l2": f"{len(bx.c)} rotating cache copies"},
+               "config": {"workload": ("latent_fp8_dc192_g4_b4_l64k" if fp8 else
+                                       "latent_h32_g4_b4_l64k" if bx.heads == 32 else "latent_g4_b4_l64k"),
+                          "B": bx.B, "L": bx.L, "H": bx.heads, "G": 4, "d_c": bx.dc, "k": KTOP,
+                          "l2": f"{len(bx.c)} rotating cache copies"},
                "roofline": {"bound": "hbm", "kernel": "latent8_score_kernel" if fp8 else "stream_score_kernel<bf16>",
                             "achieved": achieved, "peak": hbm, "peak_source": which, "unit": "GB/s",
                             "frac": achieved / hbm, "kernel_us": r["score"] * 1e3}, "clocks": clk}
@@ -705,7 +727,7 @@ def main():
     ap.add_argument("--impl", default="li", choices=["li", "reference"])
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "latent", "latent192", "hs_b1", "hs_b16"],
+    ap.add_argument("--workload", default="decode", choices=["decode", "glm5_decode", "prefill", "latent", "latent192", "latent_glm5", "hs_b1", "hs_b16"],
                     help="decode (default) is the benchmarked configuration; the others time the other "
                          "configurations of the parity tests")
     args = ap.parse_args()

@@ -120,7 +120,9 @@ typedef struct {
  *   k_scale  one fp32 per key row, same row numbering as k (E4M3 only)
  *   len      [rows] int32 visible lengths (decode; NULL = max_len; each must lie in [0, max_len])
  *   scores   fp32, row r at scores + r * scores_ld; only visible positions are written
- * Tensor-core path: heads == 64, dim == 128, k base 16-byte aligned, k_dtype E4M3.
+ * Tensor-core path: dim == 128, k base 16-byte aligned, k_dtype E4M3; heads == 64
+ * (DeepSeek-V3.2's indexer) or, for decode (causal == 0), heads == 32 (GLM-5's;
+ * Multi-layer Indexer, Appendix settings table).
  * workspace: li_index_score_workspace(desc) bytes (0 for decode; may be NULL then). */
 li_status li_index_score(const void* q, const float* w, const void* k, const float* k_scale,
                          int64_t cache_batch_rows, const int32_t* len, float* scores, int64_t scores_ld,
@@ -159,7 +161,7 @@ li_status li_topk(const float* scores, int64_t scores_ld, const int32_t* len, in
  * counts instead of sweeping the row for it.
  *   q, w, k, k_scale, cache_batch_rows, len, scores, scores_ld, desc
  *           as li_index_score (desc->causal must be 0; tensor-core path only:
- *           BF16 query, E4M3 keys, heads 64, dim 128).  scores_ld must be a
+ *           BF16 query, E4M3 keys, heads 64 or 32, dim 128).  scores_ld must be a
  *           multiple of 4 and scores 16-byte aligned, as li_topk requires.
  *   k_top, idx, vals   as li_topk's k, idx, vals.
  *   workspace  li_decode_select_workspace(desc) bytes of device memory,
@@ -266,7 +268,8 @@ li_status li_absorb_query_layers(const void* q_bf16, const void* w_dec_bf16, voi
  *   q_tilde [batch, heads, latent_dim] bf16     w [batch, heads] fp32
  *   c       latent rows of latent_dim bf16; request b's rows begin at row b * cache_batch_rows
  *   len     [batch] int32 or NULL (= max_len)
- * Tensor-core path (bf16): heads == 64, latent_dim == 256, c base 16-byte aligned. */
+ * Tensor-core path (bf16): heads == 64 or 32, latent_dim == 256, c base 16-byte
+ * aligned. */
 li_status li_latent_score(const void* q_tilde_bf16, const float* w, const void* c_bf16, int64_t cache_batch_rows,
                           const int32_t* len, float* scores, int64_t scores_ld, int batch, int heads, int latent_dim,
                           int max_len, li_stream_t stream);
@@ -315,8 +318,8 @@ li_status li_latent_score_fp8(const void* q_tilde_bf16, const float* w, const vo
  *   q_tilde [followers, batch, heads, latent_dim] bf16   w [followers, batch, heads] fp32
  *   out_idx [followers, batch, k] int32 (out)
  * Candidates outside [0, rows of c) are reported as LI_ERR_BOUNDS by
- * li_get_last_error and are not read.  heads == 64, latent_dim == 256,
- * followers * heads <= 256, n_cand <= LI_TOPK_MAX_LEN.
+ * li_get_last_error and are not read.  heads == 64 or 32, latent_dim == 256,
+ * 1 <= followers <= 4, n_cand <= LI_TOPK_MAX_LEN.
  * workspace: li_hs_refine_workspace(...) bytes. */
 li_status li_hs_refine(const void* c_bf16, int64_t cache_batch_rows, int64_t cache_rows, const int32_t* cand,
                        int batch, int n_cand, const void* q_tilde_bf16, const float* w, int followers, int heads,

@@ -5,7 +5,8 @@
 //
 //     I_f[b,i] = sum_j w[f,b,j] * ReLU(q~[f,b,j,:] . c[b, cand[b,i], :])
 //
-// MMA tile: 128 gathered candidates (M) x F*64 follower-heads (N <= 256) x 256
+// MMA tile: 128 gathered candidates (M) x F*H follower-heads (N <= 256; H = 64
+// for DeepSeek-V3.2's indexer, 32 for GLM-5's) x 256
 // latent dims (four 128-byte K blocks, 16 tcgen05.mma.kind::f16 with K = 16).
 // Rows are gathered with 16-byte cp.async into the 128-byte-swizzled K-major
 // layout the MMA reads; padding (negative) candidates are zero-filled and
@@ -22,7 +23,6 @@ namespace li {
 namespace {
 
 constexpr int HS_M = 128;
-constexpr int HS_H = 64;
 constexpr int HS_DC = 256;
 constexpr int HS_KBLK = 4;
 constexpr int HS_STAGES = 6;
@@ -30,9 +30,10 @@ constexpr int HS_STAGE_BYTES = HS_M * 128;
 constexpr int HS_DEPTH = 3;  // cp.async groups in flight per producer thread
 constexpr int HS_THREADS = 288;
 
-template <int F>
+template <int F, int H>
 struct HsCfg {
-    static constexpr int N = F * HS_H;
+    static_assert(H == 64 || H == 32, "head count");
+    static constexpr int N = F * H;
     static constexpr int Q_BYTES = HS_KBLK * N * 128;
     static constexpr int OFF_Q = HS_STAGES * HS_STAGE_BYTES;
     static constexpr int OFF_W = OFF_Q + Q_BYTES;
@@ -54,9 +55,9 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-template <int F>
+template <int F, int H>
 __global__ void __launch_bounds__(HS_THREADS, 1) hs_rescore_kernel(const HsArgs a, int tiles_per_cta) {
-    using C = HsCfg<F>;
+    using C = HsCfg<F, H>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     const int b = blockIdx.y;
@@ -185,10 +186,10 @@ __global__ void __launch_bounds__(HS_THREADS, 1) hs_rescore_kernel(const HsArgs 
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int ci = et + 128 * (g0 + u);
-                const int r = ci / CH, cc = ci % CH;  // r = f * 64 + j
-                const int f = r / HS_H, j = r % HS_H;
+                const int r = ci / CH, cc = ci % CH;  // r = f * H + j
+                const int f = r / H, j = r % H;
                 v[u] = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.qt) +
-                                                            (((size_t)f * a.B + b) * HS_H + j) * HS_DC) + cc);
+                                                            (((size_t)f * a.B + b) * H + j) * HS_DC) + cc);
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
@@ -198,8 +199,8 @@ __global__ void __launch_bounds__(HS_THREADS, 1) hs_rescore_kernel(const HsArgs 
             }
         }
         for (int r = et; r < C::N; r += 128) {
-            const int f = r / HS_H, j = r % HS_H;
-            wsm[r] = __ldg(a.w + ((size_t)f * a.B + b) * HS_H + j);
+            const int f = r / H, j = r % H;
+            wsm[r] = __ldg(a.w + ((size_t)f * a.B + b) * H + j);
         }
         fence_proxy_async_smem();
         mbar_arrive(qready);
@@ -216,12 +217,19 @@ __global__ void __launch_bounds__(HS_THREADS, 1) hs_rescore_kernel(const HsArgs 
             float res[F];
 #pragma unroll
             for (int f = 0; f < F; ++f) {
-                const uint32_t tb = tmem_base + ((uint32_t)(g * 32) << 16) + (uint32_t)(acc * C::N + f * HS_H);
-                uint32_t v0[32], v1[32];
-                tmem_ld32(tb, v0);
-                tmem_ld32(tb + 32, v1);
-                tmem_ld_wait();
-                res[f] = relu_dot32(v0, wsm + f * HS_H) + relu_dot32(v1, wsm + f * HS_H + 32);
+                const uint32_t tb = tmem_base + ((uint32_t)(g * 32) << 16) + (uint32_t)(acc * C::N + f * H);
+                if constexpr (H == 64) {
+                    uint32_t v0[32], v1[32];
+                    tmem_ld32(tb, v0);
+                    tmem_ld32(tb + 32, v1);
+                    tmem_ld_wait();
+                    res[f] = relu_dot32(v0, wsm + f * H) + relu_dot32(v1, wsm + f * H + 32);
+                } else {
+                    uint32_t v0[32];
+                    tmem_ld32(tb, v0);
+                    tmem_ld_wait();
+                    res[f] = relu_dot32(v0, wsm + f * H);
+                }
             }
             tc_fence_before();
             mbar_arrive(&acce[acc]);
@@ -240,14 +248,14 @@ __global__ void __launch_bounds__(HS_THREADS, 1) hs_rescore_kernel(const HsArgs 
     }
 }
 
-template <int F>
+template <int F, int H>
 li_status launch_f(const HsArgs& a, cudaStream_t st) {
-    using C = HsCfg<F>;
+    using C = HsCfg<F, H>;
     static bool attr_done[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && !attr_done[dev]) {
-        if (cudaFuncSetAttribute(hs_rescore_kernel<F>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
+        if (cudaFuncSetAttribute(hs_rescore_kernel<F, H>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
             cudaSuccess)
             return host_check_launch();
         attr_done[dev] = true;
@@ -257,7 +265,7 @@ li_status launch_f(const HsArgs& a, cudaStream_t st) {
     int cpr = max(1, sms / max(1, a.B));
     int tpc = max(1, (ntiles + cpr - 1) / cpr);
     cpr = (ntiles + tpc - 1) / tpc;
-    hs_rescore_kernel<F><<<dim3(cpr, a.B), HS_THREADS, C::SMEM, st>>>(a, tpc);
+    hs_rescore_kernel<F, H><<<dim3(cpr, a.B), HS_THREADS, C::SMEM, st>>>(a, tpc);
     return host_check_launch();
 }
 
@@ -265,13 +273,25 @@ li_status launch_f(const HsArgs& a, cudaStream_t st) {
 
 li_status launch_hs_rescore(const HsArgs& a, cudaStream_t st) {
     if (a.B <= 0 || a.C <= 0) return LI_OK;
-    switch (a.F) {
-    case 1: return launch_f<1>(a, st);
-    case 2: return launch_f<2>(a, st);
-    case 3: return launch_f<3>(a, st);
-    case 4: return launch_f<4>(a, st);
-    default: return LI_ERR_UNSUPPORTED;
+    if (a.H == 64) {
+        switch (a.F) {
+        case 1: return launch_f<1, 64>(a, st);
+        case 2: return launch_f<2, 64>(a, st);
+        case 3: return launch_f<3, 64>(a, st);
+        case 4: return launch_f<4, 64>(a, st);
+        default: return LI_ERR_UNSUPPORTED;
+        }
     }
+    if (a.H == 32) {
+        switch (a.F) {
+        case 1: return launch_f<1, 32>(a, st);
+        case 2: return launch_f<2, 32>(a, st);
+        case 3: return launch_f<3, 32>(a, st);
+        case 4: return launch_f<4, 32>(a, st);
+        default: return LI_ERR_UNSUPPORTED;
+        }
+    }
+    return LI_ERR_UNSUPPORTED;
 }
 
 }  // namespace li

@@ -167,18 +167,21 @@ li_status li_index_score(const void* q, const float* w, const void* k, const flo
     const int T = d.tokens_per_request > 1 ? d.tokens_per_request : 1;
     if (d.rows % T != 0) return LI_ERR_INVALID_ARG;
     if (T > 1 && (d.causal || d.q_dtype != LI_DTYPE_BF16)) return LI_ERR_UNSUPPORTED;  // multi-token: FP8 decode
+    const bool f32 = d.q_dtype == LI_DTYPE_F32 && d.k_dtype == LI_DTYPE_F32;
+    if (!f32) {
+        if (d.q_dtype != LI_DTYPE_BF16 || d.k_dtype != LI_DTYPE_E4M3) return LI_ERR_UNSUPPORTED;
+        if ((d.heads != 64 && (d.heads != 32 || d.causal)) || d.dim != 128) return LI_ERR_UNSUPPORTED;
+    }
     DevErr e;
     if (ready(&e) != LI_OK) return LI_ERR_CUDA;
 
-    if (d.q_dtype == LI_DTYPE_F32 && d.k_dtype == LI_DTYPE_F32) {
+    if (f32) {
         if (k_scale || (size_t)d.heads * d.dim > 12000) return LI_ERR_UNSUPPORTED;
         SimtArgs a{static_cast<const float*>(q), w, static_cast<const float*>(k), len, scores, scores_ld,
                    cache_batch_rows, d.rows, d.heads, d.dim, d.max_len, d.causal, d.causal_offset, e};
         return launch_simt_score(a, stream);
     }
-    if (d.q_dtype != LI_DTYPE_BF16 || d.k_dtype != LI_DTYPE_E4M3) return LI_ERR_UNSUPPORTED;
     if (!k_scale) return LI_ERR_INVALID_ARG;
-    if (d.heads != 64 || d.dim != 128) return LI_ERR_UNSUPPORTED;
     if (!aligned(k, 16) || !aligned(q, 16)) return LI_ERR_INVALID_ARG;
     const uint64_t total_rows = cache_batch_rows > 0 ? (uint64_t)(d.rows / T - 1) * cache_batch_rows + d.max_len
                                                      : (uint64_t)d.max_len;
@@ -198,6 +201,7 @@ li_status li_index_score(const void* q, const float* w, const void* k, const flo
         a.max_len = d.max_len;
         a.w_bulk = aligned(w, 16) ? 1 : 0;
         a.tokens = T;
+        a.heads = d.heads;
         a.err = e;
         const int ntiles = (d.max_len + 127) / 128;
         return launch_stream_score_fp8(kmap, a, d.rows, ntiles, stream);
@@ -245,7 +249,7 @@ li_status li_decode_score_hist(const void* q, const float* w, const void* k, con
         return LI_ERR_INVALID_ARG;
     if (d.rows == 0 || d.max_len == 0) return LI_OK;
     if (d.q_dtype != LI_DTYPE_BF16 || d.k_dtype != LI_DTYPE_E4M3) return LI_ERR_UNSUPPORTED;
-    if (d.heads != 64 || d.dim != 128) return LI_ERR_UNSUPPORTED;
+    if ((d.heads != 64 && d.heads != 32) || d.dim != 128) return LI_ERR_UNSUPPORTED;
     if (!q || !w || !k || !k_scale || !scores || !hist || scores_ld < d.max_len) return LI_ERR_INVALID_ARG;
     if (!aligned(k, 16) || !aligned(q, 16) || !aligned(hist, 16)) return LI_ERR_INVALID_ARG;
     const int T = d.tokens_per_request > 1 ? d.tokens_per_request : 1;
@@ -269,6 +273,7 @@ li_status li_decode_score_hist(const void* q, const float* w, const void* k, con
     a.hist = hist;
     a.w_bulk = aligned(w, 16) ? 1 : 0;
     a.tokens = T;
+    a.heads = d.heads;
     a.err = e;
     return launch_stream_score_fp8_hist(kmap, a, d.rows, (d.max_len + 127) / 128, stream);
 }
@@ -298,7 +303,7 @@ li_status li_decode_select(const void* q, const float* w, const void* k, const f
     if (k_top < 1 || k_top > LI_TOPK_MAX_LEN || d.max_len > LI_TOPK_MAX_LEN) return LI_ERR_INVALID_ARG;
     if (d.rows == 0) return LI_OK;
     if (d.q_dtype != LI_DTYPE_BF16 || d.k_dtype != LI_DTYPE_E4M3) return LI_ERR_UNSUPPORTED;
-    if (d.heads != 64 || d.dim != 128) return LI_ERR_UNSUPPORTED;
+    if ((d.heads != 64 && d.heads != 32) || d.dim != 128) return LI_ERR_UNSUPPORTED;
     if (!idx || !workspace || workspace_bytes < li_decode_select_workspace(&d) || !aligned(workspace, 256))
         return LI_ERR_INVALID_ARG;
     if (d.tokens_per_request > 1 && d.rows % d.tokens_per_request != 0) return LI_ERR_INVALID_ARG;
@@ -390,7 +395,7 @@ static li_status latent_score_impl(const void* q_tilde_bf16, const float* w, con
     if (batch < 0 || heads <= 0 || latent_dim <= 0 || max_len < 0 || cache_batch_rows < 0) return LI_ERR_INVALID_ARG;
     if (batch == 0 || max_len == 0) return LI_OK;
     if (!q_tilde_bf16 || !w || !c_bf16 || !scores || scores_ld < max_len) return LI_ERR_INVALID_ARG;
-    if (heads != 64 || latent_dim != 256) return LI_ERR_UNSUPPORTED;
+    if ((heads != 64 && heads != 32) || latent_dim != 256) return LI_ERR_UNSUPPORTED;
     if (!aligned(c_bf16, 16) || !aligned(q_tilde_bf16, 16) || (hist && !aligned(hist, 16))) return LI_ERR_INVALID_ARG;
     DevErr e;
     if (ready(&e) != LI_OK) return LI_ERR_CUDA;
@@ -410,6 +415,7 @@ static li_status latent_score_impl(const void* q_tilde_bf16, const float* w, con
     a.batch_rows = cache_batch_rows;
     a.max_len = max_len;
     a.hist = hist;
+    a.heads = heads;
     a.err = e;
     const int ntiles = (max_len + 127) / 128;
     return hist ? launch_stream_score_bf16_hist(cmap, a, batch, ntiles, stream)
@@ -476,7 +482,7 @@ li_status li_hs_refine(const void* c_bf16, int64_t cache_batch_rows, int64_t cac
         return LI_ERR_INVALID_ARG;
     if (batch == 0) return LI_OK;
     if (!out_idx) return LI_ERR_INVALID_ARG;
-    if (heads != 64 || latent_dim != 256 || followers * heads > 256) return LI_ERR_UNSUPPORTED;
+    if ((heads != 64 && heads != 32) || latent_dim != 256 || followers > 4) return LI_ERR_UNSUPPORTED;
     DevErr e;
     if (ready(&e) != LI_OK) return LI_ERR_CUDA;
     if (n_cand == 0) {
@@ -490,7 +496,7 @@ li_status li_hs_refine(const void* c_bf16, int64_t cache_batch_rows, int64_t cac
     if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) return LI_ERR_INVALID_ARG;
     const int ldw = (int)align_up((size_t)n_cand, 4);
     float* sc = static_cast<float*>(workspace);
-    HsArgs h{c_bf16, cache_batch_rows, cache_rows, cand, batch, n_cand, followers, q_tilde_bf16, w, sc, e};
+    HsArgs h{c_bf16, cache_batch_rows, cache_rows, cand, batch, n_cand, followers, heads, q_tilde_bf16, w, sc, e};
     li_status s = launch_hs_rescore(h, stream);
     if (s != LI_OK) return s;
     TopkArgs t{sc, ldw, nullptr, followers * batch, n_cand, 0, 0, k, out_idx, nullptr, cand, n_cand, batch,

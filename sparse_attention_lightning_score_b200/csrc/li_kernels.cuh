@@ -13,8 +13,9 @@ namespace li {
 
 // ---------------------------------------------------------------- streaming scorer
 struct StreamArgs {
-    const void* q;          // FP8 kind: bf16 [B,64,128]; BF16 kind: bf16 [B,64,256]
-    const float* w;         // [B,64]
+    const void* q;          // FP8 kind: bf16 [B,H,128]; BF16 kind: bf16 [B,H,256]
+    const float* w;         // [B,H]
+    int heads;              // H: 64 or 32
     const float* kscale;    // FP8 kind: one per cache row
     const int32_t* len;     // [B] or nullptr
     float* scores;
@@ -129,8 +130,9 @@ struct HsArgs {
     long long cache_rows;   // rows addressable from c
     const int32_t* cand;    // [B, C]
     int B, C, F;
-    const void* qt;         // bf16 [F,B,64,256]
-    const float* w;         // [F,B,64]
+    int H;                  // heads per follower: 64 or 32
+    const void* qt;         // bf16 [F,B,H,256]
+    const float* w;         // [F,B,H]
     float* out;             // [F,B,C] candidate scores (workspace)
     DevErr err;
 };

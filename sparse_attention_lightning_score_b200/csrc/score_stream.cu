@@ -9,9 +9,10 @@
 //                            scoring the shared latent cache with the absorbed
 //                            query (LatentIndex abstract and Figure 1).
 //
-// The logits q.k form a [128 keys x 64 heads] tile per step: a dense
+// The logits q.k form a [128 keys x H heads] tile per step: a dense
 // contraction, so it runs on the tcgen05 tensor cores with the keys as the
-// M=128 operand (one TMEM lane per key) and the heads as N=64.  The head
+// M=128 operand (one TMEM lane per key) and the heads as N = H (64 for
+// DeepSeek-V3.2's indexer, 32 for GLM-5's).  The head
 // reduction, ReLU and key scale happen in registers after one tcgen05.ld per
 // 32 columns, so the [H, L] logits never reach HBM; only one fp32 score per
 // key is written.
@@ -37,9 +38,10 @@ namespace li {
 
 namespace {
 
-template <bool FP8, int KBLK, int STAGES, int NACC, bool HIST>
+template <int NH, bool FP8, int KBLK, int STAGES, int NACC, bool HIST>
 struct StreamCfg {
-    static constexpr int H = 64;                       // heads = MMA N
+    static constexpr int H = NH;                       // heads = MMA N (64: DeepSeek-V3.2, 32: GLM-5)
+    static_assert(NH == 32 || NH == 64, "head count");
     static constexpr int M = 128;                      // keys per tile = MMA M = TMEM lanes
     static constexpr int STAGE_BYTES = M * 128;        // one 128-byte K block of 128 keys
     static constexpr int Q_BYTES = KBLK * H * 128;     // query operand, same K blocks
@@ -62,10 +64,10 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-template <bool FP8, int KBLK, int STAGES, int NACC, bool HIST>
-__global__ void __launch_bounds__(StreamCfg<FP8, KBLK, STAGES, NACC, HIST>::THREADS, 2)
+template <int NH, bool FP8, int KBLK, int STAGES, int NACC, bool HIST>
+__global__ void __launch_bounds__(StreamCfg<NH, FP8, KBLK, STAGES, NACC, HIST>::THREADS, 2)
     stream_score_kernel(const __grid_constant__ CUtensorMap kmap, const StreamArgs a) {
-    using C = StreamCfg<FP8, KBLK, STAGES, NACC, HIST>;
+    using C = StreamCfg<NH, FP8, KBLK, STAGES, NACC, HIST>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
 
@@ -269,13 +271,23 @@ __global__ void __launch_bounds__(StreamCfg<FP8, KBLK, STAGES, NACC, HIST>::THRE
             if (!mbar_wait(&accf[acc], aph, a.err)) break;
             tc_fence_after();
             const uint32_t tb = tmem_base + ((uint32_t)(g * 32) << 16) + (uint32_t)(acc * C::H);
-            uint32_t v0[32], v1[32];
-            tmem_ld32(tb, v0);
-            tmem_ld32(tb + 32, v1);
-            tmem_ld_wait();
-            tc_fence_before();
-            mbar_arrive(&acce[acc]);
-            const float sum = relu_dot32(v0, wsm) + relu_dot32(v1, wsm + 32);
+            float sum;
+            if constexpr (C::H == 64) {
+                uint32_t v0[32], v1[32];
+                tmem_ld32(tb, v0);
+                tmem_ld32(tb + 32, v1);
+                tmem_ld_wait();
+                tc_fence_before();
+                mbar_arrive(&acce[acc]);
+                sum = relu_dot32(v0, wsm) + relu_dot32(v1, wsm + 32);
+            } else {
+                uint32_t v0[32];
+                tmem_ld32(tb, v0);
+                tmem_ld_wait();
+                tc_fence_before();
+                mbar_arrive(&acce[acc]);
+                sum = relu_dot32(v0, wsm);
+            }
             if (s < len_b) {
                 const float sc = FP8 ? sum * sk : sum;
                 out[s] = sc;
@@ -304,10 +316,10 @@ done:
     }
 }
 
-template <bool FP8, int KBLK, int STAGES, int NACC, bool HIST = false>
-li_status launch_impl(const CUtensorMap& map, const StreamArgs& args, int batch, int ntiles_max, cudaStream_t st) {
-    using C = StreamCfg<FP8, KBLK, STAGES, NACC, HIST>;
-    auto kern = stream_score_kernel<FP8, KBLK, STAGES, NACC, HIST>;
+template <int NH, bool FP8, int KBLK, int STAGES, int NACC, bool HIST = false>
+li_status launch_one(const CUtensorMap& map, const StreamArgs& args, int batch, int ntiles_max, cudaStream_t st) {
+    using C = StreamCfg<NH, FP8, KBLK, STAGES, NACC, HIST>;
+    auto kern = stream_score_kernel<NH, FP8, KBLK, STAGES, NACC, HIST>;
     static bool attr_done[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -327,6 +339,13 @@ li_status launch_impl(const CUtensorMap& map, const StreamArgs& args, int batch,
     dim3 grid(max(cpr, 1), batch);
     if (launch_pdl(kern, grid, dim3(C::THREADS), C::SMEM, st, 1, map, a) != cudaSuccess) return host_check_launch();
     return host_check_launch();
+}
+
+template <bool FP8, int KBLK, int STAGES, int NACC, bool HIST = false>
+li_status launch_impl(const CUtensorMap& map, const StreamArgs& args, int batch, int ntiles_max, cudaStream_t st) {
+    if (args.heads == 64) return launch_one<64, FP8, KBLK, STAGES, NACC, HIST>(map, args, batch, ntiles_max, st);
+    if (args.heads == 32) return launch_one<32, FP8, KBLK, STAGES, NACC, HIST>(map, args, batch, ntiles_max, st);
+    return LI_ERR_UNSUPPORTED;
 }
 
 }  // namespace

@@ -75,8 +75,10 @@ def test_decode_select_rejects_bad_arguments_on_host():
     assert call(d, scores=ctypes.c_void_p(264)) == _lib.LI_ERR_INVALID_ARG  # scores not 16-byte aligned
     c = _lib.ScoreDesc(2, 64, 128, 100, 1, 0, _lib.LI_DTYPE_BF16, _lib.LI_DTYPE_E4M3)
     assert call(c) == _lib.LI_ERR_INVALID_ARG                               # causal is not a decode step
-    u = _lib.ScoreDesc(2, 32, 128, 100, 0, 0, _lib.LI_DTYPE_BF16, _lib.LI_DTYPE_E4M3)
-    assert call(u) == _lib.LI_ERR_UNSUPPORTED                               # only the tensor-core shape
+    u = _lib.ScoreDesc(2, 48, 128, 100, 0, 0, _lib.LI_DTYPE_BF16, _lib.LI_DTYPE_E4M3)
+    assert call(u) == _lib.LI_ERR_UNSUPPORTED                               # only the tensor-core shapes: 64 or 32 heads
+    u = _lib.ScoreDesc(2, 64, 64, 100, 0, 0, _lib.LI_DTYPE_BF16, _lib.LI_DTYPE_E4M3)
+    assert call(u) == _lib.LI_ERR_UNSUPPORTED                               # dim 128 only
     f = _lib.ScoreDesc(2, 64, 128, 100, 0, 0, _lib.LI_DTYPE_F32, _lib.LI_DTYPE_F32)
     assert call(f) == _lib.LI_ERR_UNSUPPORTED
     z = _lib.ScoreDesc(0, 64, 128, 100, 0, 0, _lib.LI_DTYPE_BF16, _lib.LI_DTYPE_E4M3)
@@ -119,6 +121,21 @@ def test_latent_fp8_and_layers_reject_bad_arguments_on_host():
     assert lib.li_absorb_query_layers(p, p, p, -1, 1, 64, 128, 256, None) == _lib.LI_ERR_INVALID_ARG
     assert lib.li_absorb_query_layers(p, p, p, 2, 1, 64, 128, 100, None) == _lib.LI_ERR_INVALID_ARG
     assert lib.li_absorb_query_layers(p, p, p, 0, 1, 64, 128, 256, None) == _lib.LI_OK
+
+
+def test_head_counts_checked_on_host():
+    lib = _lib.load()
+    p = ctypes.c_void_p(256)
+    # GLM-5's 32 indexer heads are a decode shape; prefill keeps 64
+    c = _lib.ScoreDesc(8, 32, 128, 100, 1, 0, _lib.LI_DTYPE_BF16, _lib.LI_DTYPE_E4M3)
+    assert lib.li_index_score(p, p, p, p, 0, None, p, 100, ctypes.byref(c), p, 1 << 20,
+                              None) == _lib.LI_ERR_UNSUPPORTED
+    # (q~, w, c, cache_batch_rows, len, scores, ld, batch, heads, latent_dim, max_len, stream)
+    assert lib.li_latent_score(p, p, p, 0, None, p, 100, 2, 16, 256, 100, None) == _lib.LI_ERR_UNSUPPORTED
+    assert lib.li_latent_score(p, p, p, 0, None, p, 100, 2, 32, 192, 100, None) == _lib.LI_ERR_UNSUPPORTED
+    # (c, cache_batch_rows, cache_rows, cand, batch, n_cand, q~, w, followers, heads, latent_dim, k, out, ws, bytes, st)
+    assert lib.li_hs_refine(p, 0, 100, p, 1, 64, p, p, 5, 32, 256, 8, p, p, 1 << 20, None) == _lib.LI_ERR_UNSUPPORTED
+    assert lib.li_hs_refine(p, 0, 100, p, 1, 64, p, p, 2, 48, 256, 8, p, p, 1 << 20, None) == _lib.LI_ERR_UNSUPPORTED
 
 
 def test_multi_token_descriptor_checked_on_host():

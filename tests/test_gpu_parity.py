@@ -280,12 +280,14 @@ def test_bad_length_reports_bounds():
 
 
 def test_unsupported_shapes_raise():
-    q = torch.zeros(2, 32, 128, dtype=torch.bfloat16, device=DEV)
-    w = torch.zeros(2, 32, device=DEV)
+    q = torch.zeros(2, 48, 128, dtype=torch.bfloat16, device=DEV)
+    w = torch.zeros(2, 48, device=DEV)
     k = torch.zeros(2, 64, 128, dtype=torch.uint8, device=DEV)
     ks = torch.ones(2, 64, device=DEV)
     with pytest.raises(LiError):
-        api.li_index_score(q, w, k, ks)
+        api.li_index_score(q, w, k, ks)            # 48 heads: neither indexer shape
+    with pytest.raises(LiError):                   # 32 heads are a decode shape only
+        api.li_index_score(q[:, :32].contiguous(), w[:, :32].contiguous(), k[0], ks[0], causal=True)
 
 
 # ---------------------------------------------------------------------------
