@@ -353,6 +353,37 @@ li_status li_hs_refine_noalloc(const void* c_bf16, int64_t cache_batch_rows, int
                                int heads, int latent_dim, int k, int32_t* out_idx, li_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* The consumer: sparse attention over a selection                           */
+/* ------------------------------------------------------------------------ */
+/* Each new token of a DSA layer attends only the positions its indexer
+ * selected (Multi-layer Indexer, long-version transcript: 2048 tokens per
+ * layer, and the selection is the only link between indexer and attention).
+ * This call is that attention in DeepSeek-V3.2's absorbed-MLA decode form: a
+ * cache row is one 576-element bf16 vector (512 latent + 64 RoPE) shared by
+ * every query head, the key is the whole row and the value its first 512
+ * elements:
+ *     out[b,h,:] = sum_i p_i * kv[b, sel[b,i], 0:512],
+ *     p = softmax over the valid i of scale * (q[b,h,:] . kv[b, sel[b,i], :])
+ * A selection is valid when 0 <= sel < cache_rows; -1 (a top-k pad) is skipped
+ * and any other value outside that range is skipped and reported as
+ * LI_ERR_BOUNDS by li_get_last_error.  A request with no valid selection gets
+ * out = 0.
+ *   q_bf16   [batch, heads, 576] bf16, 16-byte aligned; heads a multiple of 64
+ *   kv_bf16  rows of 576 bf16 (1152 bytes); request b's rows begin at row
+ *            b * cache_batch_rows (0 = one cache shared by every request)
+ *   cache_rows  rows a selection may address (<= cache_batch_rows when that is > 0)
+ *   sel      [batch, k] int32 cache rows (li_topk's output, any order)
+ *   scale    softmax scale, finite and > 0
+ *   out      [batch, heads, 512] fp32 (out), 16-byte aligned
+ *   workspace  li_sparse_attention_workspace(batch, heads, k) bytes of device
+ *            memory, 256-byte aligned (per 256 selections and head: 512 + 2 fp32)
+ * Nothing is allocated and the host is not synchronised. */
+size_t li_sparse_attention_workspace(int batch, int heads, int k);
+li_status li_sparse_attention(const void* q_bf16, const void* kv_bf16, int64_t cache_batch_rows, int64_t cache_rows,
+                              const int32_t* sel, int batch, int heads, int k, float scale, float* out,
+                              void* workspace, size_t workspace_bytes, li_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* Diagnostics                                                               */
 /* ------------------------------------------------------------------------ */
 /* Launches one block whose only work is the library's bounded wait on an

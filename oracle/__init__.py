@@ -249,3 +249,49 @@ def hs_refine(qt, qt_dtype, w, c_bf16, cand, k, *, c_batch_rows=None, nthreads=N
     lib().orc_hs_refine(qt_dtype, _p(q), _p(wa), _p(c), ctypes.c_longlong(c_batch_rows), _p(cd), F, B, H, dc,
                         C, int(k), _p(out), _p(cs), nthreads or nthreads_default())
     return (out, cs) if with_scores else out
+
+
+# ---------------------------------------------------------------------------
+# the consumer: sparse attention over a selection
+# ---------------------------------------------------------------------------
+def _bf16_f64(bits: np.ndarray) -> np.ndarray:
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def sparse_attention(q_bf16, kv_bf16, sel, scale, *, dv=512, with_mag=False):
+    """Each query head's attention over the selected cache rows, in fp64.
+
+    Multi-layer Indexer (long-version transcript): a DSA layer attends, for each
+    new token, only the positions its indexer selected.  Reading of the shape
+    (the pages give none): DeepSeek-V3.2's absorbed-MLA decode form, where one
+    cache row per position is the key and its first ``dv`` elements the value.
+
+        o[b,h,:] = sum_i p_i kv[b, s_i, :dv],
+        p = softmax over i of scale * (q[b,h,:] . kv[b, s_i, :])
+
+    over the valid selections s_i (0 <= s_i < cache rows; duplicates count
+    once per listing); a request without any gets o = 0.
+    q [B,H,D] bf16; kv [B,L,D] bf16 (or one shared [L,D]); sel int [B,k].
+    Returns o [B,H,dv] (and mag = sum_i p_i |kv[b,s_i,:dv]|, the scale of each
+    output's sum, when ``with_mag``).  Matrix products and exp are numpy's.
+    """
+    q = _bf16_f64(_raw(q_bf16, BF16))
+    kv = _bf16_f64(_raw(kv_bf16, BF16))
+    sel = np.asarray(sel)
+    B, H, D = q.shape
+    out = np.zeros((B, H, dv))
+    mag = np.zeros((B, H, dv))
+    for b in range(B):
+        cache = kv[b] if kv.ndim == 3 else kv
+        s = sel[b]
+        s = s[(s >= 0) & (s < cache.shape[0])]
+        if s.size == 0:
+            continue
+        keys = cache[s]                              # [n, D]
+        logits = scale * (q[b] @ keys.T)             # [H, n]
+        logits = logits - logits.max(axis=1, keepdims=True)
+        p = np.exp(logits)
+        p = p / p.sum(axis=1, keepdims=True)         # softmax over the selected positions
+        out[b] = p @ keys[:, :dv]
+        mag[b] = p @ np.abs(keys[:, :dv])
+    return (out, mag) if with_mag else out

@@ -385,6 +385,38 @@ def li_hs_refine(c: torch.Tensor, cand: torch.Tensor, q_tilde: torch.Tensor, w: 
     return out
 
 
+def li_sparse_attention_workspace(batch: int, heads: int, k: int, device) -> torch.Tensor:
+    need = _lib.load().li_sparse_attention_workspace(int(batch), int(heads), int(k))
+    return torch.empty(max(int(need), 256), dtype=torch.uint8, device=device)
+
+
+def li_sparse_attention(q: torch.Tensor, kv: torch.Tensor, sel: torch.Tensor, scale: float, *,
+                        out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None, stream=None):
+    """Attention of each query head over the selected cache rows (absorbed-MLA decode form).
+
+    q bf16 [B,H,576] (H a multiple of 64); kv bf16 [B,L,576] (or one shared [L,576]); sel int32 [B,k]
+    cache rows, -1 = none -> out fp32 [B,H,512] = softmax(scale * q . kv[sel]) @ kv[sel, :512].
+    """
+    _need(q, "q", torch.bfloat16)
+    _need(kv, "kv", torch.bfloat16)
+    _need(sel, "sel", torch.int32)
+    B, H, D = q.shape
+    k = sel.shape[1]
+    batch_rows = kv.shape[1] if kv.dim() == 3 else 0
+    cache_rows = kv.shape[-2]
+    if out is None:
+        out = torch.empty((B, H, 512), dtype=torch.float32, device=q.device)
+    lib = _lib.load()
+    need = lib.li_sparse_attention_workspace(B, H, k)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = li_sparse_attention_workspace(B, H, k, q.device)
+    st = lib.li_sparse_attention(_ptr(q), _ptr(kv), batch_rows, cache_rows, _ptr(sel), B, H, k, float(scale),
+                                 _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                 _stream(stream))
+    _lib.check("li_sparse_attention", st)
+    return out
+
+
 def li_selftest_wait_timeout(limit_ns: int, stream=None):
     st = _lib.load().li_selftest_wait_timeout(int(limit_ns), _stream(stream))
     _lib.check("li_selftest_wait_timeout", st)

@@ -504,6 +504,55 @@ li_status li_hs_refine(const void* c_bf16, int64_t cache_batch_rows, int64_t cac
     return launch_topk(t, stream);
 }
 
+size_t li_sparse_attention_workspace(int batch, int heads, int k) {
+    if (batch <= 0 || heads <= 0 || k <= 0) return 0;
+    return sparse_attn_workspace_bytes(batch, heads, k);
+}
+
+li_status li_sparse_attention(const void* q_bf16, const void* kv_bf16, int64_t cache_batch_rows, int64_t cache_rows,
+                              const int32_t* sel, int batch, int heads, int k, float scale, float* out,
+                              void* workspace, size_t workspace_bytes, li_stream_t stream) {
+    if (batch < 0 || heads <= 0 || k < 0 || cache_batch_rows < 0 || cache_rows < 0) return LI_ERR_INVALID_ARG;
+    if (cache_batch_rows > 0 && cache_rows > cache_batch_rows) return LI_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !(scale < 3.0e38f)) return LI_ERR_INVALID_ARG;
+    if (heads % 64 != 0 || heads > 65535 || batch > 65535) return LI_ERR_UNSUPPORTED;
+    if (batch == 0) return LI_OK;
+    if (!q_bf16 || !kv_bf16 || !out || (k > 0 && !sel)) return LI_ERR_INVALID_ARG;
+    if (!aligned(q_bf16, 16) || !aligned(kv_bf16, 16) || !aligned(out, 16)) return LI_ERR_INVALID_ARG;
+    DevErr e;
+    if (ready(&e) != LI_OK) return LI_ERR_CUDA;
+    if (k == 0) {  // nothing selected: every output is 0
+        if (cudaMemsetAsync(out, 0, (size_t)batch * heads * 512 * sizeof(float), stream) != cudaSuccess)
+            return LI_ERR_CUDA;
+        return LI_OK;
+    }
+    const size_t need = sparse_attn_workspace_bytes(batch, heads, k);
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return LI_ERR_INVALID_ARG;
+    const uint64_t total_rows = cache_batch_rows > 0 ? (uint64_t)(batch - 1) * cache_batch_rows + cache_rows
+                                                     : (uint64_t)cache_rows;
+    if (total_rows >= (1ull << 31) - 1 || (uint64_t)batch * heads >= (1ull << 31)) return LI_ERR_UNSUPPORTED;
+    CUtensorMap qmap;
+    if (!encode_map_2d(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q_bf16, 576, (uint64_t)batch * heads, 1152, 64, 64))
+        return LI_ERR_CUDA;
+    const size_t parts = (size_t)batch * sparse_attn_splits(k) * heads;
+    SparseAttnArgs a{};
+    a.q = q_bf16;
+    a.kv = kv_bf16;
+    a.batch_rows = cache_batch_rows;
+    a.rows_visible = cache_rows;
+    a.sel = sel;
+    a.batch = batch;
+    a.heads = heads;
+    a.k = k;
+    a.scale = scale;
+    a.opart = static_cast<float*>(workspace);
+    a.mpart = a.opart + parts * 512;
+    a.lpart = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(a.mpart) + align_up(parts * 4, 256));
+    a.out = out;
+    a.err = e;
+    return launch_sparse_attn(qmap, a, stream);
+}
+
 li_status li_selftest_wait_timeout(uint64_t limit_ns, li_stream_t stream) {
     DevErr e;
     if (ready(&e) != LI_OK) return LI_ERR_CUDA;

@@ -138,6 +138,27 @@ struct HsArgs {
 };
 li_status launch_hs_rescore(const HsArgs& a, cudaStream_t st);
 
+// ---------------------------------------------------------------- sparse attention over a selection
+struct SparseAttnArgs {
+    const void* q;          // bf16 [batch, heads, 576]
+    const void* kv;         // bf16 rows of 576; request b's rows begin at row b * batch_rows
+    long long batch_rows;   // 0 = one cache shared by every request
+    long long rows_visible; // rows a selection may address
+    const int32_t* sel;     // [batch, k] cache rows, -1 = none
+    int batch, heads, k;
+    int splits;             // set by the launcher: ceil(k / 256)
+    float scale;            // softmax scale applied to q . kv
+    float* opart;           // [batch, splits, heads, 512] unnormalised split outputs (workspace)
+    float* mpart;           // [batch, splits, heads] split maxima, log2 domain (workspace)
+    float* lpart;           // [batch, splits, heads] split sums of exponentials (workspace)
+    float* out;             // fp32 [batch, heads, 512]
+    DevErr err;
+};
+size_t sparse_attn_workspace_bytes(int batch, int heads, int k);
+int sparse_attn_splits(int k);
+// qmap: q as [batch * heads, 576] bf16, box 64 x 64, 128-byte swizzle
+li_status launch_sparse_attn(const CUtensorMap& qmap, SparseAttnArgs a, cudaStream_t st);
+
 // ---------------------------------------------------------------- diagnostics
 li_status launch_selftest_wait(unsigned long long limit_ns, cudaStream_t st);
 

@@ -407,3 +407,78 @@ def test_hs_padding_and_position_tie_break():
     assert out[0, 0].tolist() == [3]
     out = oracle.hs_refine(qt, oracle.F64, w, c, np.array([[7, -1, -1, -1]]), 3)
     assert out[0, 0].tolist() == [7, -1, -1]
+
+
+# ---------------------------------------------------------------------------
+# the consumer: sparse attention over a selection
+# ---------------------------------------------------------------------------
+def test_sparse_attention_hand_example():
+    ex = GOLD["sparse_attention_small"]
+    q = torch.tensor(ex["q"], dtype=torch.bfloat16)
+    kv = torch.tensor(ex["kv_rows"], dtype=torch.bfloat16)
+    got = oracle.sparse_attention(q, kv, np.array(ex["sel"]), math.log(3.0), dv=ex["dv"])
+    np.testing.assert_allclose(got, np.array(ex["out"]), rtol=1e-15, atol=1e-15)
+
+
+def _attn_case(seed=3, B=2, H=3, L=40, D=12, dv=8, k=10):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(B, H, D, generator=g).to(torch.bfloat16)
+    kv = torch.randn(B, L, D, generator=g).to(torch.bfloat16)
+    sel = np.stack([np.sort(np.random.default_rng(seed + b).choice(L, k, replace=False)) for b in range(B)])
+    return q, kv, sel, dv
+
+
+def test_sparse_attention_uniform_and_hard_limits():
+    q, kv, sel, dv = _attn_case()
+    vals = kv.double().numpy()
+    # scale -> 0: every selected position gets the same weight, o = mean of the values
+    o0 = oracle.sparse_attention(q, kv, sel, 1e-12, dv=dv)
+    for b in range(2):
+        np.testing.assert_allclose(o0[b], np.tile(vals[b, sel[b], :dv].mean(0), (3, 1)), rtol=1e-9, atol=1e-9)
+    # scale -> large: the position with the largest logit takes all the weight
+    oh = oracle.sparse_attention(q, kv, sel, 1e4, dv=dv)
+    qd = q.double().numpy()
+    for b in range(2):
+        for h in range(3):
+            best = sel[b][np.argmax(vals[b, sel[b]] @ qd[b, h])]
+            np.testing.assert_allclose(oh[b, h], vals[b, best, :dv], rtol=1e-12, atol=1e-12)
+
+
+def test_sparse_attention_two_positions_closed_form():
+    # two selections with logits l0, l1: o = (e^l0 v0 + e^l1 v1) / (e^l0 + e^l1); listing a position
+    # twice doubles its weight
+    q, kv, sel, dv = _attn_case(B=1, H=1, k=2)
+    s = 0.37
+    v = kv.double().numpy()[0]
+    l = [s * float(v[i] @ q.double().numpy()[0, 0]) for i in sel[0]]
+    e = [math.exp(x) for x in l]
+    want = (e[0] * v[sel[0][0], :dv] + e[1] * v[sel[0][1], :dv]) / (e[0] + e[1])
+    np.testing.assert_allclose(oracle.sparse_attention(q, kv, sel, s, dv=dv)[0, 0], want, rtol=1e-12)
+    twice = np.array([[sel[0][0], sel[0][1], sel[0][0]]])
+    want2 = (2 * e[0] * v[sel[0][0], :dv] + e[1] * v[sel[0][1], :dv]) / (2 * e[0] + e[1])
+    np.testing.assert_allclose(oracle.sparse_attention(q, kv, twice, s, dv=dv)[0, 0], want2, rtol=1e-12)
+
+
+def test_sparse_attention_invariants():
+    q, kv, sel, dv = _attn_case()
+    o = oracle.sparse_attention(q, kv, sel, 0.5, dv=dv)
+    # the order of the selection does not matter; pads and out-of-range rows are skipped
+    perm = np.stack([s[::-1] for s in sel])
+    padded = np.concatenate([perm, np.full((2, 3), -1), np.full((2, 1), 10 ** 6)], axis=1)
+    np.testing.assert_allclose(oracle.sparse_attention(q, kv, padded, 0.5, dv=dv), o, rtol=1e-13, atol=1e-13)
+    # each head attends on its own (the softmax runs over positions, not heads)
+    for h in range(3):
+        oh = oracle.sparse_attention(q[:, h:h + 1].contiguous(), kv, sel, 0.5, dv=dv)
+        np.testing.assert_allclose(oh[:, 0], o[:, h], rtol=1e-13, atol=1e-13)
+    # a request reads its own cache: request 1 alone against a shared copy of its rows
+    o1 = oracle.sparse_attention(q[1:], kv[1], sel[1:], 0.5, dv=dv)
+    np.testing.assert_allclose(o1[0], o[1], rtol=1e-13, atol=1e-13)
+    # the output is a convex combination of the selected values, and mag bounds it
+    o, mag = oracle.sparse_attention(q, kv, sel, 0.5, dv=dv, with_mag=True)
+    assert np.all(np.abs(o) <= mag + 1e-12)
+    for b in range(2):
+        vals = kv.double().numpy()[b, sel[b], :dv]
+        assert np.all(o[b] <= vals.max(0) + 1e-12) and np.all(o[b] >= vals.min(0) - 1e-12)
+    # no valid selection: zero
+    none = np.full((2, 4), -1)
+    assert np.all(oracle.sparse_attention(q, kv, none, 0.5, dv=dv) == 0.0)
