@@ -638,6 +638,60 @@ class HsBench:
         return {"step": e0.elapsed_time(e1) / steps}
 
 
+def run_schedules(dev, args, clocks, n_layers=8):
+    """Decode steps over n_layers DSA layers (indexer + sparse attention [+ a dense block]) under the
+    IndexCache and Multi-layer Indexer schedules: each plan serial and with its indexers on a side
+    stream, as one CUDA graph per step."""
+    import torch
+    from sparse_attention_lightning_score_b200.schedule import DecodeLayerStack, indexcache_plan, mli_plan
+    stack = DecodeLayerStack(n_layers=n_layers, B=B, L=L, k=KTOP, dense=(7168, 4096), device=dev, seed=1)
+    plans = {"dsa": mli_plan(n_layers, lag=0), "mli_lag1": mli_plan(n_layers, lag=1),
+             "mli_lag2": mli_plan(n_layers, lag=2), "indexcache_half": indexcache_plan(n_layers, retention=0.5),
+             "indexcache_half_mli_lag1": mli_plan(n_layers, lag=1, retention=0.5)}
+    main, side = torch.cuda.current_stream(), torch.cuda.Stream()
+    reps = max(3, args.steps // 5)
+
+    def time_step(plan, overlap, with_rest):
+        step = stack.bind(plan, overlap=overlap, with_rest=with_rest)
+        for _ in range(args.warmup):
+            step.run(main, side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step.run(torch.cuda.current_stream(), side)
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        del g
+        return e0.elapsed_time(e1) * 1e3 / reps
+
+    clocks.start()
+    res = {}
+    for with_rest in (False, True):
+        key = "with_dense" if with_rest else "indexer_and_attention"
+        res[key] = {}
+        for name, plan in plans.items():
+            res[key][name] = {"serial_us": round(time_step(plan, False, with_rest), 2)}
+            if name != "dsa":
+                res[key][name]["overlapped_us"] = round(time_step(plan, True, with_rest), 2)
+    clk = clocks.stop()
+    base = res["indexer_and_attention"]["dsa"]["serial_us"]
+    best = min(v.get("overlapped_us", v["serial_us"]) for v in res["indexer_and_attention"].values())
+    return {"metric": "decode step µs over the layers (indexer + sparse attention per layer)",
+            "value": base, "unit": "µs/step (DSA, serial)", "higher_is_better": False,
+            "dtype": "e4m3 indexer, bf16 attention",
+            "config": {"workload": f"schedules_{n_layers}layers_b{B}_l32k", "layers": n_layers, "B": B, "L": L,
+                       "k": KTOP, "indexer_heads": H, "attention_heads": 128, "kv": "576 bf16 per position",
+                       "dense_block": "x[B,7168] @ W[7168,4096] bf16 per layer (cuBLAS), in with_dense only",
+                       "launch": "one CUDA graph per step; overlapped = indexers on a side stream"},
+            "schedules": res, "best_over_dsa": round(base / best, 3), "gpu_launches": None, "clocks": clk}
+
+
 def run_other(args, rank, world, local_rank):
     import torch
     from sparse_attention_lightning_score_b200 import api
@@ -664,6 +718,8 @@ def run_other(args, rank, world, local_rank):
                             "peak": hbm, "peak_source": which, "unit": "GB/s",
                             "frac": algo / (sc_ms * 1e-3) / 1e9 / hbm, "kernel_us": sc_ms * 1e3},
                "topk": {"us": tk_ms * 1e3}, "gpu_launches": 2 * args.steps, "clocks": clk}
+    elif args.workload == "mli":
+        out = run_schedules(dev, args, clocks)
     elif args.workload == "prefill":
         bx = PrefillBench(dev)
         clocks.start()
@@ -727,7 +783,7 @@ def main():
     ap.add_argument("--impl", default="li", choices=["li", "reference"])
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="decode", choices=["decode", "glm5_decode", "prefill", "latent", "latent192", "latent_glm5", "hs_b1", "hs_b16"],
+    ap.add_argument("--workload", default="decode", choices=["decode", "glm5_decode", "prefill", "latent", "latent192", "latent_glm5", "hs_b1", "hs_b16", "mli"],
                     help="decode (default) is the benchmarked configuration; the others time the other "
                          "configurations of the parity tests")
     args = ap.parse_args()
