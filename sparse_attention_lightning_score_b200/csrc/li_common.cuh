@@ -345,63 +345,40 @@ __device__ __forceinline__ float relu_dot32_x2(const uint32_t (&v)[32], const fl
 }
 
 // e4m3(x / sq) (round to nearest even, saturating) with the quotient rounded as
-// IEEE fp32 division rounds it, without a division in almost every case.
+// IEEE fp32 division rounds it, at the cost of one multiply in most calls.
 // With r the correctly rounded reciprocal of sq, y = x * r lies within 2.5 ulp
-// of the correctly rounded quotient q, so for |y| in e4m3's normal range q lies
-// in y's e4m3 rounding interval or just past one of its ends (where both round
-// to that end's e4m3 value).  Which e4m3 value q rounds to is then decided by
-// q's position relative to the interval's midpoint M (y with its 20 low
-// mantissa bits set to 0x80000) through the residual d = M sq - x, taken with
-// one rounding (FMA):
-//   - d's sign is exact, and d itself is exact whenever |d| is small next to
-//     |M sq| (M has 5 significant bits, x 8), in particular near M;
-//   - q = M exactly when |d| <= ulp(M) / 2 * sq (fp32 ties go to M, whose last
-//     bit is 0), and M then rounds to e4m3 as q does;
-//   - otherwise q lies beyond M (away from zero) when d's sign is opposite to
-//     M's, and M's fp32 neighbour on that side rounds to e4m3 as q does.
-// Products from bf16 data land on e4m3 midpoints often (448 x / absmax is
-// frequently an exact midpoint before sq is rounded), so the exact decision
-// matters.  Checked exhaustively against IEEE division over every pair of bf16
-// absmax and bf16 x with |x| <= absmax.
+// of the correctly rounded quotient q (each of the two roundings is a relative
+// error of at most 2^-24).  y and q then round to the same e4m3 value unless an
+// e4m3 rounding midpoint lies between them.  For |y| in e4m3's normal range,
+// those midpoints are the values whose 20 low mantissa bits are 0x80000.  So
+// only a product within 8 ulp of such a point, or outside [2^-6, 512] (e4m3
+// subnormals, zero, an overflowed reciprocal, NaN), needs the division.
 //
-// The residual and ulp arithmetic needs sq >= 2^-90 (products stay normal) and
-// |y| in [2^-6, 512] (outside: e4m3 subnormals, an overflowed reciprocal, NaN);
-// y == 0 is exact.  There the quotient comes from the IEEE division.
-__device__ __forceinline__ bool quotient_needs_division(float y, float sq) {
+// (An exact division-free decision also exists: the residual M sq - x against
+// the midpoint M is exact near M and decides ties and sides.  It was checked
+// exhaustively and measured; it is built from integer and logic operations,
+// whose pipe then throttles the quantiser, so the division stays.)
+__device__ __forceinline__ bool quotient_needs_division(float y) {
     const float ay = fabsf(y);
-    return !(sq >= 0x1p-90f) || !(ay <= 512.f) || (ay < 0x1p-6f && ay != 0.f);
+    const uint32_t m = __float_as_uint(y) & 0xfffffu;
+    return !(ay >= 0x1p-6f && ay <= 512.f) || (m - 0x7fff8u) <= 16u;
 }
 
-// A value with the e4m3 rounding of fl(x / sq), given y = x * r inside the
-// range quotient_needs_division admits.
-__device__ __forceinline__ float midpoint_decided(float x, float y, float sq) {
-    const uint32_t u = __float_as_uint(y);
-    const uint32_t mb = (u & 0xfff00000u) | 0x80000u;               // M, same sign and exponent as y
-    const float d = __fmaf_rn(__uint_as_float(mb), sq, -x);
-    const float half_ulp_sq = __uint_as_float(__float_as_uint(sq) + (u & 0x7f800000u) - (151u << 23));
-    const uint32_t step = ((__float_as_uint(d) ^ u) >> 31) ? 1u : 0xffffffffu;  // +1: beyond M
-    return __uint_as_float(mb + (fabsf(d) <= half_ulp_sq ? 0u : step));
-}
-
-// y[i] holds a value with the e4m3 rounding of x[i] / sq rounded as IEEE
-// division, for N elements of every lane.  When any lane of the warp has an
-// element outside the decided range, the whole warp divides instead
-// (warp-uniform, so the rare path costs no divergent branch per element).  All
-// 32 lanes must call this together.
+// y[i] = x[i] / sq rounded as IEEE division, for N elements of every lane.  The
+// products are taken first; when any lane of the warp has an element that needs
+// it, the whole warp divides instead (warp-uniform, so the rare path costs no
+// divergent branch per element).  All 32 lanes must call this together.
 template <int N>
 __device__ __forceinline__ void quotients_for_e4m3(const float (&x)[N], float sq, float r, float (&y)[N]) {
     bool need = false;
 #pragma unroll
     for (int i = 0; i < N; ++i) {
         y[i] = x[i] * r;
-        need |= quotient_needs_division(y[i], sq);
+        need |= quotient_needs_division(y[i]);
     }
     if (__any_sync(0xffffffffu, need)) {
 #pragma unroll
         for (int i = 0; i < N; ++i) y[i] = __fdiv_rn(x[i], sq);
-    } else {
-#pragma unroll
-        for (int i = 0; i < N; ++i) y[i] = midpoint_decided(x[i], y[i], sq);
     }
 }
 
