@@ -638,6 +638,57 @@ class HsBench:
         return {"step": e0.elapsed_time(e1) / steps}
 
 
+def run_consumer(dev, args, clocks):
+    """The consumer alone: li_sparse_attention at the decode shape (B = 8 requests, 128 query heads,
+    the indexer's 2048 selections out of L = 32768 cached 576-element rows), rotating through 8
+    selection sets so that the gathered rows (8 x 18.9 MB) exceed L2."""
+    import numpy as np
+    import torch
+    from sparse_attention_lightning_score_b200 import api
+    Ha, D = 128, 576
+    g = torch.Generator(device=dev).manual_seed(1)
+    q = torch.randn(B, Ha, D, device=dev, generator=g).to(torch.bfloat16)
+    kv = torch.randn(B, L, D, device=dev, generator=g).to(torch.bfloat16)
+    rng = np.random.default_rng(1)
+    sels = [torch.from_numpy(np.stack([np.sort(rng.choice(L, KTOP, replace=False)) for _ in range(B)])
+                             .astype(np.int32)).to(dev) for _ in range(8)]
+    out = torch.empty(B, Ha, 512, device=dev)
+    ws = api.li_sparse_attention_workspace(B, Ha, KTOP, dev)
+    scale = 1.0 / 192 ** 0.5
+    for i in range(args.warmup):
+        api.li_sparse_attention(q, kv, sels[i % 8], scale, out=out, workspace=ws)
+    torch.cuda.synchronize()
+    gr = capture([lambda i=i: api.li_sparse_attention(q, kv, sels[i % 8], scale, out=out, workspace=ws)
+                  for i in range(16)])
+    gr.replay()
+    torch.cuda.synchronize()
+    reps = max(2, args.steps // 16)
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        gr.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    us = e0.elapsed_time(e1) * 1e3 / (16 * reps)
+    hbm, which = peaks()
+    bf16_peak = float(json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["bf16_tflops"]) \
+        if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else 1590.0
+    byts = B * KTOP * D * 2 + B * Ha * D * 2 + B * Ha * 512 * 4
+    flops = B * Ha * KTOP * (D + 512) * 2
+    return {"metric": "sparse attention over the selection, µs per call", "value": us, "unit": "µs/call",
+            "higher_is_better": False, "dtype": "bf16",
+            "config": {"workload": "sparse_attention_b8_h128_k2048_l32k", "B": B, "heads": Ha, "k": KTOP, "L": L,
+                       "row": "576 bf16 (512 latent + 64 RoPE); value = first 512",
+                       "l2": "8 rotating selection sets, 151 MB of gathered rows"},
+            "roofline": {"bound": "hbm", "kernel": "sparse_attn_kernel + sparse_attn_merge_kernel",
+                         "achieved": byts / us / 1e3, "peak": hbm, "peak_source": which, "unit": "GB/s",
+                         "frac": byts / us / 1e3 / hbm, "algorithmic_bytes": byts,
+                         "tensor_tflops": flops / us / 1e6, "tensor_frac_of_bf16": flops / us / 1e6 / bf16_peak},
+            "gpu_launches": 2 * 16 * reps, "clocks": clk}
+
+
 def run_schedules(dev, args, clocks, n_layers=8):
     """Decode steps over n_layers DSA layers (indexer + sparse attention [+ a dense block]) under the
     IndexCache and Multi-layer Indexer schedules: each plan serial and with its indexers on a side
@@ -720,6 +771,8 @@ def run_other(args, rank, world, local_rank):
                "topk": {"us": tk_ms * 1e3}, "gpu_launches": 2 * args.steps, "clocks": clk}
     elif args.workload == "mli":
         out = run_schedules(dev, args, clocks)
+    elif args.workload == "sparse_attention":
+        out = run_consumer(dev, args, clocks)
     elif args.workload == "prefill":
         bx = PrefillBench(dev)
         clocks.start()
@@ -783,7 +836,8 @@ def main():
     ap.add_argument("--impl", default="li", choices=["li", "reference"])
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="decode", choices=["decode", "glm5_decode", "prefill", "latent", "latent192", "latent_glm5", "hs_b1", "hs_b16", "mli"],
+    ap.add_argument("--workload", default="decode", choices=["decode", "glm5_decode", "prefill", "latent", "latent192", "latent_glm5", "hs_b1", "hs_b16", "mli",
+                             "sparse_attention"],
                     help="decode (default) is the benchmarked configuration; the others time the other "
                          "configurations of the parity tests")
     args = ap.parse_args()

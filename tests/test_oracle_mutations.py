@@ -75,3 +75,35 @@ def test_pins_catch_mutation(tmp_path, monkeypatch, name):
     finally:
         oracle._lib = saved
     assert caught, f"no pin caught the mutation {name}"
+
+
+# The consumer's oracle is numpy code: mutate its source text instead of oracle.c.
+PY_MUTATIONS = {
+    "attn_softmax_over_heads": ("logits.max(axis=1, keepdims=True)", "logits.max(axis=0, keepdims=True)",
+                                "p.sum(axis=1, keepdims=True)", "p.sum(axis=0, keepdims=True)"),
+    "attn_scale_dropped": ("logits = scale * (q[b] @ keys.T)", "logits = (q[b] @ keys.T)"),
+    "attn_value_wrong_slice": ("out[b] = p @ keys[:, :dv]", "out[b] = p @ keys[:, -dv:]"),
+    "attn_pads_kept": ("s = s[(s >= 0) & (s < cache.shape[0])]", "s = s[s < cache.shape[0]]"),
+    "attn_not_normalised": ("p = p / p.sum(axis=1, keepdims=True)", "p = p"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(PY_MUTATIONS))
+def test_pins_catch_python_oracle_mutation(monkeypatch, name):
+    import inspect
+    import textwrap
+    reps = PY_MUTATIONS[name]
+    src = textwrap.dedent(inspect.getsource(oracle.sparse_attention))
+    for old, new in zip(reps[::2], reps[1::2]):
+        assert old in src, (name, old)
+        src = src.replace(old, new)
+    ns = dict(vars(oracle))
+    exec(compile(src, f"<{name}>", "exec"), ns)
+    monkeypatch.setattr(oracle, "sparse_attention", ns["sparse_attention"])
+    failed = []
+    for t in [n for n in PIN_TESTS if "sparse_attention" in n]:
+        try:
+            getattr(pins, t)()
+        except Exception:
+            failed.append(t)
+    assert failed, f"no pin caught {name}"
