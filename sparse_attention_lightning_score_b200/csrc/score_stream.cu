@@ -162,6 +162,9 @@ __global__ void __launch_bounds__(StreamCfg<NH, FP8, KBLK, STAGES, NACC, HIST>::
                 for (int kb = 0; kb < KBLK; ++kb) {
                     // FP8: the last stage's buffer first holds the query row, until it is quantised
                     if (FP8 && stage == STAGES - 1 && ph == 0u && !mbar_wait(qready, 0, a.err)) { ok = false; break; }
+                    // FP8: one key tile goes out ahead of the query row, the rest once it has landed, so
+                    // that the row does not queue behind every CTA's whole first wave of key loads
+                    if (FP8 && it * KBLK + kb == 1 && !mbar_wait(qload, 0, a.err)) { ok = false; break; }
                     if (!mbar_wait(&empty[stage], ph ^ 1u, a.err)) { ok = false; break; }
                     mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
                     tma_load_2d(smem + stage * C::STAGE_BYTES, &kmap, kb * C::ELEMS_PER_KBLOCK, y, &full[stage],

@@ -17,8 +17,8 @@
 //     of shared-memory slots with 16-byte cp.async (eight threads per 128-byte
 //     row segment, 128-byte swizzle; pads and rejected selections read as
 //     zeros), keeping several chunks in flight per thread;
-//   - warp 4 loads the 64 query rows of the CTA's heads by TMA, then issues
-//     S^T_t = K_t Q^T for both tiles (M = 128 positions, N = 64 heads, K = 576)
+//   - thread 0 loads the 64 query rows of the CTA's heads by TMA at the start;
+//     warp 4 issues S^T_t = K_t Q^T for both tiles (M = 128 positions, N = 64 heads, K = 576)
 //     into TMEM and, once P^T_t is ready, O^T += V_t^T P^T_t (M = 128 value
 //     elements per block, N = 64 heads, K = 128 positions) with V^T and P^T
 //     read MN-major, so nothing is transposed in shared memory;
@@ -75,6 +75,12 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+// 2^x by the SFU's approximation (a couple of ulp; the weights are rounded to bf16 right after).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
@@ -137,6 +143,7 @@ __global__ void __launch_bounds__(SA_THREADS, 1)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_TMEM);
 
     if (threadIdx.x == 0) {
+        tma_prefetch_desc(&qmap);
         for (int i = 0; i < SA_RS; ++i) {
             mbar_init(&full[i], 128);
             mbar_init(&empty[i], 1);
@@ -152,6 +159,12 @@ __global__ void __launch_bounds__(SA_THREADS, 1)
         tmem_relinquish();
     }
     pdl_wait();  // the selections may come from the previous kernel of the stream
+    if (threadIdx.x == 0) {
+        // the 64 query rows of the CTA's heads, first of all (nothing can be consumed before them)
+        mbar_arrive_expect_tx(qfull, SA_CH * SA_QCHUNK);
+        for (int c = 0; c < SA_CH; ++c)
+            tma_load_2d(qs + c * SA_QCHUNK, &qmap, c * 64, b * a.heads + hg * SA_NH, qfull, l2_policy_evict_last());
+    }
     if (warp == 0) {
         // the CTA's selections as rows of kv; pads and rejected ones become -1
         for (int i = lane; i < SA_POS; i += 32) {
@@ -221,9 +234,6 @@ __global__ void __launch_bounds__(SA_THREADS, 1)
     } else if (warp == 4) {
         // ---------------------------------------------------------------- query load and MMA issuer
         if (lane == 0) {
-            mbar_arrive_expect_tx(qfull, SA_CH * SA_QCHUNK);
-            for (int c = 0; c < SA_CH; ++c)
-                tma_load_2d(qs + c * SA_QCHUNK, &qmap, c * 64, b * a.heads + hg * SA_NH, qfull, l2_policy_evict_last());
             const uint32_t ring_s = smem_u32(ring), q_s = smem_u32(qs), p_s = smem_u32(pbuf);
             bool ok = mbar_wait(qfull, 0, a.err);
             tc_fence_after();
@@ -314,8 +324,9 @@ __global__ void __launch_bounds__(SA_THREADS, 1)
                 uint32_t pk[16];
 #pragma unroll
                 for (int h = 0; h < 32; h += 2) {
-                    const float p0 = valid ? exp2f(__uint_as_float(r[h]) * c2 - msm[hh * 32 + h]) : 0.f;
-                    const float p1 = valid ? exp2f(__uint_as_float(r[h + 1]) * c2 - msm[hh * 32 + h + 1]) : 0.f;
+                    const float2 m2 = *reinterpret_cast<const float2*>(msm + hh * 32 + h);
+                    const float p0 = valid ? ex2_approx(__fmaf_rn(__uint_as_float(r[h]), c2, -m2.x)) : 0.f;
+                    const float p1 = valid ? ex2_approx(__fmaf_rn(__uint_as_float(r[h + 1]), c2, -m2.y)) : 0.f;
                     l[hh * 32 + h] += p0;
                     l[hh * 32 + h + 1] += p1;
                     __nv_bfloat162 pp = __floats2bfloat162_rn(p0, p1);
