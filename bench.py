@@ -694,31 +694,31 @@ def run_schedules(dev, args, clocks, n_layers=8):
     IndexCache and Multi-layer Indexer schedules: each plan serial and with its indexers on a side
     stream, as one CUDA graph per step."""
     import torch
-    from sparse_attention_lightning_score_b200.schedule import DecodeLayerStack, indexcache_plan, mli_plan
+    from sparse_attention_lightning_score_b200.schedule import (DecodeLayerStack, StepGraph, indexcache_plan,
+                                                                mli_plan, priority_streams)
     stack = DecodeLayerStack(n_layers=n_layers, B=B, L=L, k=KTOP, dense=(7168, 4096), device=dev, seed=1)
     plans = {"dsa": mli_plan(n_layers, lag=0), "mli_lag1": mli_plan(n_layers, lag=1),
              "mli_lag2": mli_plan(n_layers, lag=2), "indexcache_half": indexcache_plan(n_layers, retention=0.5),
              "indexcache_half_mli_lag1": mli_plan(n_layers, lag=1, retention=0.5)}
-    main, side = torch.cuda.current_stream(), torch.cuda.Stream()
+    main, side = priority_streams()
     reps = max(3, args.steps // 5)
 
     def time_step(plan, overlap, with_rest):
         step = stack.bind(plan, overlap=overlap, with_rest=with_rest)
-        for _ in range(args.warmup):
-            step.run(main, side)
+        with torch.cuda.stream(main):
+            for _ in range(args.warmup):
+                step.run(main, side)
         torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            step.run(torch.cuda.current_stream(), side)
+        g = StepGraph(step, main, side)
         g.replay()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
+        e0.record(main)
         for _ in range(reps):
             g.replay()
-        e1.record()
+        e1.record(main)
         torch.cuda.synchronize()
-        del g
+        g.close()
         return e0.elapsed_time(e1) * 1e3 / reps
 
     clocks.start()
@@ -739,7 +739,8 @@ def run_schedules(dev, args, clocks, n_layers=8):
             "config": {"workload": f"schedules_{n_layers}layers_b{B}_l32k", "layers": n_layers, "B": B, "L": L,
                        "k": KTOP, "indexer_heads": H, "attention_heads": 128, "kv": "576 bf16 per position",
                        "dense_block": "x[B,7168] @ W[7168,4096] bf16 per layer (cuBLAS), in with_dense only",
-                       "launch": "one CUDA graph per step; overlapped = indexers on a side stream"},
+                       "launch": "one CUDA graph per step, instantiated with node priorities; main stream at the "
+                                 "highest priority, overlapped = indexers on a lowest-priority side stream"},
             "schedules": res, "best_over_dsa": round(base / best, 3), "gpu_launches": None, "clocks": clk}
 
 

@@ -384,6 +384,26 @@ li_status li_sparse_attention(const void* q_bf16, const void* kv_bf16, int64_t c
                               void* workspace, size_t workspace_bytes, li_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Graphs whose kernels keep their streams' priorities                       */
+/* ------------------------------------------------------------------------ */
+/* Multi-layer Indexer (long-version transcript): the indexer runs on a second
+ * stream beside attention and the rest of the layer, and the whole pattern is
+ * captured once into the decode graph.  Kernels captured from a stream carry
+ * that stream's priority, but a graph uses it only when it is instantiated
+ * with node priorities; without them a side-stream indexer competes for SMs
+ * on equal terms with the main stream's critical path.
+ *   li_graph_instantiate: `graph` is a captured cudaGraph_t (e.g. torch's
+ *     CUDAGraph(keep_graph=True).raw_cuda_graph()); with use_node_priority != 0
+ *     the executable honours each kernel node's priority.  *exec receives a
+ *     cudaGraphExec_t owned by the caller (li_graph_destroy); the graph itself
+ *     stays the caller's.  LI_ERR_CUDA if the runtime rejects it.
+ *   li_graph_launch: one replay of `exec` on `stream` (asynchronous).
+ *   li_graph_destroy: frees `exec` (NULL is a no-op). */
+li_status li_graph_instantiate(void* graph, int use_node_priority, void** exec);
+li_status li_graph_launch(void* exec, li_stream_t stream);
+li_status li_graph_destroy(void* exec);
+
+/* ------------------------------------------------------------------------ */
 /* Diagnostics                                                               */
 /* ------------------------------------------------------------------------ */
 /* Launches one block whose only work is the library's bounded wait on an

@@ -553,6 +553,33 @@ li_status li_sparse_attention(const void* q_bf16, const void* kv_bf16, int64_t c
     return launch_sparse_attn(qmap, a, stream);
 }
 
+li_status li_graph_instantiate(void* graph, int use_node_priority, void** exec) {
+    if (!graph || !exec) return LI_ERR_INVALID_ARG;
+    *exec = nullptr;
+    cudaGraphExec_t ge = nullptr;
+    const unsigned long long flags = use_node_priority ? cudaGraphInstantiateFlagUseNodePriority : 0ull;
+    if (cudaGraphInstantiateWithFlags(&ge, static_cast<cudaGraph_t>(graph), flags) != cudaSuccess) {
+        cudaGetLastError();
+        return LI_ERR_CUDA;
+    }
+    *exec = ge;
+    return LI_OK;
+}
+
+li_status li_graph_launch(void* exec, li_stream_t stream) {
+    if (!exec) return LI_ERR_INVALID_ARG;
+    if (cudaGraphLaunch(static_cast<cudaGraphExec_t>(exec), stream) != cudaSuccess) {
+        cudaGetLastError();
+        return LI_ERR_CUDA;
+    }
+    return LI_OK;
+}
+
+li_status li_graph_destroy(void* exec) {
+    if (!exec) return LI_OK;
+    return cudaGraphExecDestroy(static_cast<cudaGraphExec_t>(exec)) == cudaSuccess ? LI_OK : LI_ERR_CUDA;
+}
+
 li_status li_selftest_wait_timeout(uint64_t limit_ns, li_stream_t stream) {
     DevErr e;
     if (ready(&e) != LI_OK) return LI_ERR_CUDA;

@@ -14,7 +14,10 @@ Two schedules from the pages, both host-side (no kernel of their own):
   without an indexer copy what their nearest indexer layer attends.  The last
   `lag` indexer layers feed no later layer within the step, so they do not run.
 
-A plan is a list of LayerPlan; lag 0 with every layer retained is plain DSA.
+A plan is a list of LayerPlan; lag 0 with every layer retained is plain DSA.  The step runs on a
+high-priority main stream and a low-priority side stream (`priority_streams`), captured into a graph
+that keeps those priorities (`StepGraph`): with equal priorities the side stream's indexer blocks take
+SMs from the main stream's critical path, and overlap then costs more than it saves.
 """
 from __future__ import annotations
 
@@ -173,6 +176,50 @@ class TwoStreamStep:
             join = torch.cuda.Event()
             join.record(side)
             main.wait_event(join)
+
+
+def priority_streams():
+    """(main, side): a main stream at the highest priority and a side stream at the lowest, so that
+    blocks of the layer's critical path are scheduled before the side stream's indexer blocks."""
+    import torch
+    return torch.cuda.Stream(priority=-32), torch.cuda.Stream(priority=0)
+
+
+class StepGraph:
+    """One TwoStreamStep captured into a CUDA graph instantiated with node priorities: each kernel
+    keeps the priority of the stream it was captured from (the indexers on a low-priority side
+    stream fill SMs the main stream leaves idle instead of taking them from it)."""
+
+    def __init__(self, step: TwoStreamStep, main, side, node_priority: bool = True):
+        import ctypes
+        import torch
+        from . import _lib
+        self._lib = _lib.load()
+        self.main = main
+        self.graph = torch.cuda.CUDAGraph(keep_graph=True)
+        with torch.cuda.graph(self.graph, stream=main):
+            step.run(main, side)
+        exec_ = ctypes.c_void_p()
+        st = self._lib.li_graph_instantiate(ctypes.c_void_p(self.graph.raw_cuda_graph()), int(node_priority),
+                                            ctypes.byref(exec_))
+        _lib.check("li_graph_instantiate", st)
+        self.exec = exec_
+
+    def replay(self):
+        import ctypes
+        from . import _lib
+        _lib.check("li_graph_launch", self._lib.li_graph_launch(self.exec, ctypes.c_void_p(self.main.cuda_stream)))
+
+    def close(self):
+        if self.exec:
+            self._lib.li_graph_destroy(self.exec)
+            self.exec = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 class DecodeLayerStack:

@@ -138,6 +138,15 @@ def test_head_counts_checked_on_host():
     assert lib.li_hs_refine(p, 0, 100, p, 1, 64, p, p, 2, 48, 256, 8, p, p, 1 << 20, None) == _lib.LI_ERR_UNSUPPORTED
 
 
+def test_graph_calls_check_arguments_on_host():
+    lib = _lib.load()
+    out = ctypes.c_void_p()
+    assert lib.li_graph_instantiate(None, 1, ctypes.byref(out)) == _lib.LI_ERR_INVALID_ARG
+    assert lib.li_graph_instantiate(ctypes.c_void_p(256), 1, None) == _lib.LI_ERR_INVALID_ARG
+    assert lib.li_graph_launch(None, None) == _lib.LI_ERR_INVALID_ARG
+    assert lib.li_graph_destroy(None) == _lib.LI_OK
+
+
 def test_multi_token_descriptor_checked_on_host():
     lib = _lib.load()
     p = ctypes.c_void_p(256)

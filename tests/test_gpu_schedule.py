@@ -72,3 +72,23 @@ def test_step_with_dense_block(stack):
     torch.cuda.synchronize()
     assert torch.equal(dense.out, ref)
     assert api.li_get_last_error() == LI_OK
+
+
+@pytest.mark.parametrize("plan", [mli_plan(6, lag=1), mli_plan(6, lag=2, retention=0.5)], ids=["mli1", "ic_half_mli2"])
+def test_priority_graph_matches_serial_reference(stack, plan):
+    # high-priority main stream, low-priority side stream, graph instantiated with node priorities
+    from sparse_attention_lightning_score_b200.schedule import StepGraph, priority_streams
+    ref = _reference(stack, plan)
+    main, side = priority_streams()
+    step = stack.bind(plan, overlap=True)
+    with torch.cuda.stream(main):
+        step.run(main, side)
+    torch.cuda.synchronize()
+    g = StepGraph(step, main, side)
+    stack.out.zero_()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    g.close()
+    assert torch.equal(stack.out, ref)
+    assert api.li_get_last_error() == LI_OK
