@@ -55,7 +55,7 @@ namespace li {
 namespace {
 
 constexpr int TK_SMEM_ROW = 40960;  // longest slice held by one CTA (160 KB of keys)
-constexpr int TK_MAX_CS = 8;        // largest cluster
+constexpr int TK_MAX_CS = 16;       // largest cluster (above 8: non-portable, checked at launch)
 constexpr int TK_SLICE = 4096;      // target slice of a row per cluster CTA
 
 __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v, int lane) {
@@ -600,6 +600,7 @@ cudaError_t launch_one(const TopkArgs& a, int row0, int nr, int cs, int chunk, c
     cudaGetDevice(&dev);
     if (dev < 64 && !attr_done[dev]) {
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TK_SMEM_BUDGET);
+        if (CLUSTER) cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         attr_done[dev] = true;
     }
     TopkArgs b = a;
@@ -615,6 +616,36 @@ cudaError_t launch_one(const TopkArgs& a, int row0, int nr, int cs, int chunk, c
     return launch_pdl(kern, dim3(CLUSTER ? cs : 1, nr), dim3(NT), smem, st, CLUSTER ? cs : 1, b, row0, chunk);
 }
 
+// Whether a cluster of 16 top-k CTAs, each with the whole shared-memory budget, can be resident at
+// once on this device (a non-portable size: it needs 16 free SMs of one GPC); otherwise 8 is the cap.
+int cluster_cap() {
+    static int cap[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && cap[dev]) return cap[dev];
+    int c = 8;
+    auto kern = topk_kernel<512, true, true>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TK_SMEM_BUDGET) == cudaSuccess &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(16, 1, 1);
+        cfg.blockDim = dim3(512, 1, 1);
+        cfg.dynamicSmemBytes = TK_SMEM_BUDGET;
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = 16;
+        attr.val.clusterDim.y = 1;
+        attr.val.clusterDim.z = 1;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n >= 1) c = 16;
+    }
+    cudaGetLastError();
+    if (dev < 64) cap[dev] = c;
+    return c;
+}
+
 }  // namespace
 
 li_status launch_topk(const TopkArgs& a, cudaStream_t st) {
@@ -624,10 +655,12 @@ li_status launch_topk(const TopkArgs& a, cudaStream_t st) {
     auto chunk_of = [&](int csz) { return (((maxl + csz - 1) / csz) + 3) & ~3; };
     // few rows: split each row over a cluster so that about 4K keys land on each CTA
     // (the load and every sweep run on many SMs); many rows: one CTA per row
+    // (a cluster larger than 8 only while every row's cluster still fits beside the others in one wave)
+    const int cap = cluster_cap();
     int cs = 1;
     if (a.rows < sms)
-        while (cs < TK_MAX_CS && chunk_of(cs) > TK_SLICE) cs *= 2;
-    while (cs < TK_MAX_CS && chunk_of(cs) > TK_SMEM_ROW) cs *= 2;
+        while (cs < cap && chunk_of(cs) > TK_SLICE && (cs < 8 || (long long)(2 * cs) * a.rows <= sms)) cs *= 2;
+    while (cs < cap && chunk_of(cs) > TK_SMEM_ROW) cs *= 2;
     const int chunk = chunk_of(cs);
     if (chunk > TK_SMEM_ROW) return LI_ERR_UNSUPPORTED;
     const bool small = chunk <= 8192;
