@@ -689,6 +689,106 @@ def run_consumer(dev, args, clocks):
             "gpu_launches": 2 * 16 * reps, "clocks": clk}
 
 
+def run_table4(dev, args, clocks):
+    """An in-house analogue of the LatentIndex paper's Table 4 (decode indexer latency by context length):
+    one decode token (B = 1) through one 4-layer group, µs per group, at L = 8K..128K:
+      dsa         4 layers x li_decode_select (FP8 keys, 64 heads, d = 128, top-2048);
+      indexcache  1 indexer layer of the 4 (the other 3 reuse its selection: no kernel);
+      latentindex 4 layers x (absorb + bf16 latent scan over the shared d_c = 256 cache + top-2048);
+      hs          anchor (absorb + scan + top-C, C = min(8192, L)) + 3 followers (one absorb launch on a
+                  side stream, gather-once rescoring, top-2048).
+    Every layer reads its own cache copies, rotated so that a group's working set exceeds L2."""
+    import torch
+    from sparse_attention_lightning_score_b200 import api, synth
+    rows = []
+    clocks.start()
+    for Lx in (8192, 16384, 32768, 65536, 131072):
+        dcase = synth.dsa_decode(B=1, L=Lx, k_top=KTOP, seed=3)
+        per = Lx * (D + 4)
+        ncopy = max(4, math.ceil(1.5 * L2_BYTES / per))
+        k8 = [dcase.k8.to(dev).clone() for _ in range(ncopy)]
+        ks = [dcase.ks.to(dev).clone() for _ in range(ncopy)]
+        q = [dcase.q.to(dev)] * 4
+        w = [dcase.w.to(dev)] * 4
+        ws = [api.li_decode_select_workspace(1, dev) for _ in range(4)]
+        sc = torch.empty((1, Lx), dtype=torch.float32, device=dev)
+        idx = torch.empty((4, 1, KTOP), dtype=torch.int32, device=dev)
+        C = min(8192, Lx)
+        lcase = synth.latent_hs(B=1, L=Lx, n_cand=C, seed=4)
+        lper = Lx * 512
+        lcopy = max(2, math.ceil(1.5 * L2_BYTES / lper))
+        cs = [lcase.c.to(dev).clone() for _ in range(lcopy)]
+        ql = [lcase.q[l].to(dev) for l in range(4)]
+        wdl = [lcase.w_dec[l].to(dev) for l in range(4)]
+        wl = [lcase.w[l].to(dev) for l in range(4)]
+        qf, wdf, wf = lcase.q[1:].contiguous().to(dev), lcase.w_dec[1:].contiguous().to(dev), lcase.w[1:].contiguous().to(dev)
+        qt = torch.empty((1, H, 256), dtype=torch.bfloat16, device=dev)
+        qtf = torch.empty((3, 1, H, 256), dtype=torch.bfloat16, device=dev)
+        hist = api.li_decode_select_workspace(1, dev).view(torch.int32)[:2048]
+        lsc = torch.empty((1, Lx), dtype=torch.float32, device=dev)
+        cand = torch.empty((1, C), dtype=torch.int32, device=dev)
+        out = torch.empty((3, 1, KTOP), dtype=torch.int32, device=dev)
+        hws = torch.empty(3 * C * 4, dtype=torch.uint8, device=dev)
+        side = torch.cuda.Stream(device=dev)
+
+        def dsa(i, layers=4):
+            for l in range(layers):
+                j = (4 * i + l) % ncopy
+                api.li_decode_select(q[l], w[l], k8[j], ks[j], KTOP, scores=sc, workspace=ws[l], idx=idx[l])
+
+        def latent(i):
+            c = cs[i % lcopy]
+            for l in range(4):
+                api.li_absorb_query(ql[l], wdl[l], out=qt)
+                api.li_latent_score_hist(qt, wl[l], c, hist, scores=lsc)
+                api.li_topk_hist(lsc, KTOP, hist, idx=idx[l])
+
+        def hs(i):
+            c = cs[i % lcopy]
+            main = torch.cuda.current_stream()
+            side.wait_stream(main)
+            with torch.cuda.stream(side):
+                api.li_absorb_query_layers(qf, wdf, out=qtf)
+            api.li_absorb_query(ql[0], wdl[0], out=qt)
+            api.li_latent_score_hist(qt, wl[0], c, hist, scores=lsc)
+            api.li_topk_hist(lsc, C, hist, idx=cand)
+            main.wait_stream(side)
+            api.li_hs_refine(c, cand, qtf, wf, KTOP, out=out, workspace=hws)
+
+        res = {"L": Lx}
+        for name, fn in (("dsa", lambda i: dsa(i)), ("indexcache", lambda i: dsa(i, 1)), ("latentindex", latent),
+                         ("hs", hs)):
+            for i in range(args.warmup):
+                fn(i)
+            torch.cuda.synchronize()
+            nrep = 8
+            g = capture([lambda i=i: fn(i) for i in range(nrep)])
+            g.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = max(2, args.steps // nrep)
+            e0.record()
+            for _ in range(reps):
+                g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            res[name + "_us_per_group"] = round(e0.elapsed_time(e1) * 1e3 / (reps * nrep), 2)
+            del g
+        res["hs_speedup_over_dsa"] = round(res["dsa_us_per_group"] / res["hs_us_per_group"], 3)
+        res["dsa_ms_per_token_61_layers"] = round(res["dsa_us_per_group"] * 61 / 4 / 1e3, 3)
+        res["hs_ms_per_token_61_layers"] = round(res["hs_us_per_group"] * 61 / 4 / 1e3, 3)
+        rows.append(res)
+        del k8, ks, cs
+        torch.cuda.empty_cache()
+    clk = clocks.stop()
+    return {"metric": "decode indexer µs per 4-layer group, one token (analogue of LatentIndex Table 4)",
+            "value": rows[-1]["hs_speedup_over_dsa"], "unit": "x (HS over DSA at L = 131072)",
+            "higher_is_better": True, "dtype": "e4m3 (DSA), bf16 (latent)",
+            "config": {"workload": "table4_b1_group4", "B": 1, "G": 4, "k": KTOP, "C": "min(8192, L)",
+                       "l2": "per-layer cache copies rotated past 1.5 x L2"},
+            "table4": rows, "gpu_launches": None, "clocks": clk}
+
+
 def run_schedules(dev, args, clocks, n_layers=8):
     """Decode steps over n_layers DSA layers (indexer + sparse attention [+ a dense block]) under the
     IndexCache and Multi-layer Indexer schedules: each plan serial and with its indexers on a side
@@ -774,6 +874,8 @@ def run_other(args, rank, world, local_rank):
         out = run_schedules(dev, args, clocks)
     elif args.workload == "sparse_attention":
         out = run_consumer(dev, args, clocks)
+    elif args.workload == "table4":
+        out = run_table4(dev, args, clocks)
     elif args.workload == "prefill":
         bx = PrefillBench(dev)
         clocks.start()
@@ -838,7 +940,7 @@ def main():
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default="decode", choices=["decode", "glm5_decode", "prefill", "latent", "latent192", "latent_glm5", "hs_b1", "hs_b16", "mli",
-                             "sparse_attention"],
+                             "sparse_attention", "table4"],
                     help="decode (default) is the benchmarked configuration; the others time the other "
                          "configurations of the parity tests")
     args = ap.parse_args()
