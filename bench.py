@@ -696,7 +696,8 @@ def run_table4(dev, args, clocks):
       indexcache  1 indexer layer of the 4 (the other 3 reuse its selection: no kernel);
       latentindex 4 layers x (absorb + bf16 latent scan over the shared d_c = 256 cache + top-2048);
       hs          anchor (absorb + scan + top-C, C = min(8192, L)) + 3 followers (one absorb launch on a
-                  side stream, gather-once rescoring, top-2048).
+                  side stream, gather-once rescoring, top-2048);
+      *_fp8       the same two over DeepSeek-V3.2's d_c = 192 e4m3 latent with per-row scales.
     Every layer reads its own cache copies, rotated so that a group's working set exceeds L2."""
     import torch
     from sparse_attention_lightning_score_b200 import api, synth
@@ -730,6 +731,18 @@ def run_table4(dev, args, clocks):
         out = torch.empty((3, 1, KTOP), dtype=torch.int32, device=dev)
         hws = torch.empty(3 * C * 4, dtype=torch.uint8, device=dev)
         side = torch.cuda.Stream(device=dev)
+        # the same methods over DeepSeek-V3.2's FP8 latent (d_c = 192 e4m3, one scale per row)
+        fcase = synth.latent_rope_nope(B=1, L=Lx, G=4, seed=5)
+        fper = Lx * 196
+        fcopy = max(2, math.ceil(1.5 * L2_BYTES / fper))
+        c8s = [(fcase.c8.to(dev).clone(), fcase.cs.to(dev).clone()) for _ in range(fcopy)]
+        q8l = [fcase.q[l].to(dev) for l in range(4)]
+        wd8 = [fcase.w_dec[l].to(dev) for l in range(4)]
+        w8 = [fcase.w[l].to(dev) for l in range(4)]
+        qf8, wdf8, wf8 = (fcase.q[1:].contiguous().to(dev), fcase.w_dec[1:].contiguous().to(dev),
+                          fcase.w[1:].contiguous().to(dev))
+        qt8 = torch.empty((1, H, 192), dtype=torch.bfloat16, device=dev)
+        qtf8 = torch.empty((3, 1, H, 192), dtype=torch.bfloat16, device=dev)
 
         def dsa(i, layers=4):
             for l in range(layers):
@@ -755,9 +768,28 @@ def run_table4(dev, args, clocks):
             main.wait_stream(side)
             api.li_hs_refine(c, cand, qtf, wf, KTOP, out=out, workspace=hws)
 
+        def latent8(i):
+            c8, cs8 = c8s[i % fcopy]
+            for l in range(4):
+                api.li_absorb_query(q8l[l], wd8[l], out=qt8)
+                api.li_latent_score_fp8(qt8, w8[l], c8, cs8, hist=hist, scores=lsc)
+                api.li_topk_hist(lsc, KTOP, hist, idx=idx[l])
+
+        def hs8(i):
+            c8, cs8 = c8s[i % fcopy]
+            main = torch.cuda.current_stream()
+            side.wait_stream(main)
+            with torch.cuda.stream(side):
+                api.li_absorb_query_layers(qf8, wdf8, out=qtf8)
+            api.li_absorb_query(q8l[0], wd8[0], out=qt8)
+            api.li_latent_score_fp8(qt8, w8[0], c8, cs8, hist=hist, scores=lsc)
+            api.li_topk_hist(lsc, C, hist, idx=cand)
+            main.wait_stream(side)
+            api.li_hs_refine_fp8(c8, cs8, cand, qtf8, wf8, KTOP, out=out, workspace=hws)
+
         res = {"L": Lx}
         for name, fn in (("dsa", lambda i: dsa(i)), ("indexcache", lambda i: dsa(i, 1)), ("latentindex", latent),
-                         ("hs", hs)):
+                         ("hs", hs), ("latentindex_fp8", latent8), ("hs_fp8", hs8)):
             for i in range(args.warmup):
                 fn(i)
             torch.cuda.synchronize()
@@ -775,10 +807,11 @@ def run_table4(dev, args, clocks):
             res[name + "_us_per_group"] = round(e0.elapsed_time(e1) * 1e3 / (reps * nrep), 2)
             del g
         res["hs_speedup_over_dsa"] = round(res["dsa_us_per_group"] / res["hs_us_per_group"], 3)
+        res["hs_fp8_speedup_over_dsa"] = round(res["dsa_us_per_group"] / res["hs_fp8_us_per_group"], 3)
         res["dsa_ms_per_token_61_layers"] = round(res["dsa_us_per_group"] * 61 / 4 / 1e3, 3)
         res["hs_ms_per_token_61_layers"] = round(res["hs_us_per_group"] * 61 / 4 / 1e3, 3)
         rows.append(res)
-        del k8, ks, cs
+        del k8, ks, cs, c8s
         torch.cuda.empty_cache()
     clk = clocks.stop()
     return {"metric": "decode indexer µs per 4-layer group, one token (analogue of LatentIndex Table 4)",

@@ -348,6 +348,21 @@ size_t li_hs_refine_workspace(int batch, int n_cand, int followers);
  *     the GPU (unordered streams) race on it: serialise them.
  *   - The first call on a device looks up the array's device address; make
  *     that first call before any stream capture begins. */
+/* li_hs_refine over DeepSeek-V3.2's FP8 latent (LatentIndex appendix, Table 5:
+ * 64 RoPE + 128 NoPE dimensions), the cache li_latent_score_fp8 scans: e4m3 rows
+ * of 192 bytes with one fp32 scale per row.  Each follower's absorbed query is
+ * quantised per (follower, request, head) as li_quantize_query does, so
+ *     I_f[b,i] = cs[r] * sum_j w_eff[f,b,j] * ReLU(q8[f,b,j,:] . c8[b,r,:]),  r = cand[b,i].
+ *   c_e4m3 / c_scale  rows and scales as in li_latent_score_fp8 (c_e4m3 16-byte aligned)
+ *   q_tilde [followers, batch, 64, 192] bf16   w [followers, batch, 64] fp32
+ * Everything else (candidates, ties, padding, output, errors, workspace) as
+ * li_hs_refine.  heads == 64, latent_dim == 192, 1 <= followers <= 4
+ * (LI_ERR_UNSUPPORTED otherwise). */
+li_status li_hs_refine_fp8(const void* c_e4m3, const float* c_scale, int64_t cache_batch_rows, int64_t cache_rows,
+                           const int32_t* cand, int batch, int n_cand, const void* q_tilde_bf16, const float* w,
+                           int followers, int heads, int latent_dim, int k, int32_t* out_idx, void* workspace,
+                           size_t workspace_bytes, li_stream_t stream);
+
 li_status li_hs_refine_noalloc(const void* c_bf16, int64_t cache_batch_rows, int64_t cache_rows, const int32_t* cand,
                                int batch, int n_cand, const void* q_tilde_bf16, const float* w, int followers,
                                int heads, int latent_dim, int k, int32_t* out_idx, li_stream_t stream);

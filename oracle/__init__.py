@@ -295,3 +295,40 @@ def sparse_attention(q_bf16, kv_bf16, sel, scale, *, dv=512, with_mag=False):
         out[b] = p @ keys[:, :dv]
         mag[b] = p @ np.abs(keys[:, :dv])
     return (out, mag) if with_mag else out
+
+
+def hs_refine_fp8(qt_bf16, w, c_e4m3, c_scale, cand, k, *, with_scores=False):
+    """Followers re-score the anchor's candidates over an FP8 latent (e4m3 rows with one scale per row,
+    DeepSeek-V3.2's d_c = 192 layout) and keep their own top-k: LatentIndex abstract (followers refine
+    the anchor's candidate set), with each follower's absorbed query quantised per (follower, request,
+    head) as quantize_query does.  A composition of quantize_query, index_score (e4m3 keys with row
+    scales) and topk; ties go to the lower cache position (candidates are listed in position order).
+
+    qt [F,B,H,dc] bf16, w [F,B,H], c_e4m3 [B,L,dc] bytes (or shared [L,dc]), c_scale [B,L] (or [L]),
+    cand int [B,C] (negative = padding) -> out int32 [F,B,k] cache positions ascending, -1 pads
+    (and the candidate scores [F,B,C], -inf for padding, with ``with_scores``).
+    """
+    F, B, H, dc = tuple(qt_bf16.shape)
+    c8 = _raw(c_e4m3, E4M3)
+    cs = _raw(c_scale, F32)
+    cd = np.asarray(cand)
+    C = cd.shape[1]
+    out = np.full((F, B, k), -1, np.int32)
+    scores = np.full((F, B, C), -np.inf)
+    for f in range(F):
+        q8, sq, _ = quantize_query(qt_bf16[f], np.asarray(w[f] if not hasattr(w, "numpy") else w[f].numpy()))
+        for b in range(B):
+            rows8 = c8[b] if c8.ndim == 3 else c8
+            rs = cs[b] if cs.ndim == 2 else cs
+            valid = np.nonzero(cd[b] >= 0)[0]
+            if valid.size == 0:
+                continue
+            pos = cd[b, valid]
+            wf = np.asarray(w[f, b] if not hasattr(w, "numpy") else w[f, b].numpy(), np.float32)[None]
+            s = index_score(q8[b:b + 1], E4M3, wf, rows8[pos], E4M3, q_scale=sq[b:b + 1], k_scale=rs[pos])[0]
+            scores[f, b, valid] = s
+            kk = min(k, valid.size)
+            sel, _ = topk(s[None], kk)
+            chosen = np.sort(pos[sel[0][sel[0] >= 0]])
+            out[f, b, :chosen.size] = chosen
+    return (out, scores) if with_scores else out

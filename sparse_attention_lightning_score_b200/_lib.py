@@ -52,6 +52,7 @@ SIGNATURES = {
     "li_hs_refine": (i32, [vp, i64, i64, vp, i32, i32, vp, vp, i32, i32, i32, i32, vp, vp, sz, vp]),
     "li_hs_refine_workspace": (sz, [i32, i32, i32]),
     "li_hs_refine_noalloc": (i32, [vp, i64, i64, vp, i32, i32, vp, vp, i32, i32, i32, i32, vp, vp]),
+    "li_hs_refine_fp8": (i32, [vp, vp, i64, i64, vp, i32, i32, vp, vp, i32, i32, i32, i32, vp, vp, sz, vp]),
     "li_sparse_attention": (i32, [vp, vp, i64, i64, vp, i32, i32, i32, ctypes.c_float, vp, vp, sz, vp]),
     "li_sparse_attention_workspace": (sz, [i32, i32, i32]),
     "li_graph_instantiate": (i32, [vp, i32, ctypes.POINTER(ctypes.c_void_p)]),

@@ -417,6 +417,35 @@ def li_sparse_attention(q: torch.Tensor, kv: torch.Tensor, sel: torch.Tensor, sc
     return out
 
 
+def li_hs_refine_fp8(c8: torch.Tensor, c_scale: torch.Tensor, cand: torch.Tensor, q_tilde: torch.Tensor,
+                     w: torch.Tensor, k: int, *, out: Optional[torch.Tensor] = None,
+                     workspace: Optional[torch.Tensor] = None, stream=None):
+    """li_hs_refine over the FP8 d_c = 192 latent: c8 e4m3/uint8 [B,L,192] (or shared [L,192]) with
+    c_scale fp32 [B,L] (or [L]); cand int32 [B,C]; q~ bf16 [F,B,64,192]; w fp32 [F,B,64]
+    -> out int32 [F,B,k] cache positions."""
+    if c8.dtype == torch.float8_e4m3fn:
+        c8 = c8.view(torch.uint8)
+    _need(c8, "c8", torch.uint8)
+    _need(c_scale, "c_scale", torch.float32)
+    _need(cand, "cand", torch.int32)
+    _need(q_tilde, "q_tilde", torch.bfloat16)
+    _need(w, "w", torch.float32)
+    F, B, H, dc = q_tilde.shape
+    C = cand.shape[1]
+    batch_rows = c8.shape[1] if c8.dim() == 3 else 0
+    cache_rows = c8.numel() // dc
+    lib = _lib.load()
+    need = lib.li_hs_refine_workspace(B, C, F)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=c8.device)
+    if out is None:
+        out = torch.empty((F, B, k), dtype=torch.int32, device=c8.device)
+    st = lib.li_hs_refine_fp8(_ptr(c8), _ptr(c_scale), batch_rows, cache_rows, _ptr(cand), B, C, _ptr(q_tilde),
+                              _ptr(w), F, H, dc, int(k), _ptr(out), _ptr(workspace), need, _stream(stream))
+    _lib.check("li_hs_refine_fp8", st)
+    return out
+
+
 def li_selftest_wait_timeout(limit_ns: int, stream=None):
     st = _lib.load().li_selftest_wait_timeout(int(limit_ns), _stream(stream))
     _lib.check("li_selftest_wait_timeout", st)

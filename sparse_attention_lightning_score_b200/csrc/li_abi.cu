@@ -504,6 +504,37 @@ li_status li_hs_refine(const void* c_bf16, int64_t cache_batch_rows, int64_t cac
     return launch_topk(t, stream);
 }
 
+li_status li_hs_refine_fp8(const void* c_e4m3, const float* c_scale, int64_t cache_batch_rows, int64_t cache_rows,
+                           const int32_t* cand, int batch, int n_cand, const void* q_tilde_bf16, const float* w,
+                           int followers, int heads, int latent_dim, int k, int32_t* out_idx, void* workspace,
+                           size_t workspace_bytes, li_stream_t stream) {
+    if (batch < 0 || n_cand < 0 || followers <= 0 || heads <= 0 || latent_dim <= 0 || k < 1 ||
+        k > LI_TOPK_MAX_LEN || n_cand > LI_TOPK_MAX_LEN || cache_batch_rows < 0 || cache_rows < 0)
+        return LI_ERR_INVALID_ARG;
+    if (heads != 64 || latent_dim != 192 || followers > 4) return LI_ERR_UNSUPPORTED;
+    if (batch == 0) return LI_OK;
+    if (!out_idx) return LI_ERR_INVALID_ARG;
+    DevErr e;
+    if (ready(&e) != LI_OK) return LI_ERR_CUDA;
+    if (n_cand == 0) {
+        TopkArgs t{nullptr, 4, nullptr, followers * batch, 0, 0, 0, k, out_idx, nullptr, nullptr, 0, 1, nullptr, 0, 1,
+                   e};
+        return launch_topk(t, stream);
+    }
+    if (!c_e4m3 || !c_scale || !cand || !q_tilde_bf16 || !w || !aligned(c_e4m3, 16) || !aligned(q_tilde_bf16, 16))
+        return LI_ERR_INVALID_ARG;
+    const size_t need = li_hs_refine_workspace(batch, n_cand, followers);
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) return LI_ERR_INVALID_ARG;
+    const int ldw = (int)align_up((size_t)n_cand, 4);
+    float* sc = static_cast<float*>(workspace);
+    Hs8Args h{c_e4m3, c_scale, cache_batch_rows, cache_rows, cand, batch, n_cand, followers, q_tilde_bf16, w, sc, e};
+    li_status s = launch_hs_rescore8(h, stream);
+    if (s != LI_OK) return s;
+    TopkArgs t{sc, ldw, nullptr, followers * batch, n_cand, 0, 0, k, out_idx, nullptr, cand, n_cand, batch,
+               nullptr, 0, 1, e};
+    return launch_topk(t, stream);
+}
+
 size_t li_sparse_attention_workspace(int batch, int heads, int k) {
     if (batch <= 0 || heads <= 0 || k <= 0) return 0;
     return sparse_attn_workspace_bytes(batch, heads, k);

@@ -138,6 +138,21 @@ struct HsArgs {
 };
 li_status launch_hs_rescore(const HsArgs& a, cudaStream_t st);
 
+// HS over DeepSeek-V3.2's FP8 latent: e4m3 rows of 192 with one fp32 scale per row, 64 heads per follower
+struct Hs8Args {
+    const void* c8;         // e4m3 latent rows of 192 bytes
+    const float* cscale;    // one fp32 per latent row, same numbering
+    long long batch_rows;
+    long long cache_rows;   // rows addressable from c8
+    const int32_t* cand;    // [B, C]
+    int B, C, F;
+    const void* qt;         // bf16 [F,B,64,192]
+    const float* w;         // [F,B,64]
+    float* out;             // [F,B,round4(C)] candidate scores (workspace)
+    DevErr err;
+};
+li_status launch_hs_rescore8(const Hs8Args& a, cudaStream_t st);
+
 // ---------------------------------------------------------------- sparse attention over a selection
 struct SparseAttnArgs {
     const void* q;          // bf16 [batch, heads, 576]

@@ -98,3 +98,40 @@ def test_latent8_full_size_sampled_rows():
     ridx, _ = oracle.topk(ref, 2048)
     assert_topk_equivalent(_np(idx)[rows], ridx, ref, 1e-2)
     assert api.li_get_last_error() == LI_OK
+
+
+# ---------------------------------------------------------------------------
+# hierarchical selection over the FP8 latent (li_hs_refine_fp8)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("B,L,C,k,F,lens", [(2, 3000, 512, 128, 3, None), (3, 2000, 640, 100, 2, [2000, 500, 77]),
+                                            (1, 1000, 130, 130, 1, None), (2, 20000, 8192, 2048, 4, None)])
+def test_hs_fp8_matches_oracle(B, L, C, k, F, lens):
+    case = synth.latent_rope_nope(B=B, L=L, G=1 + F, seed=70 + F, lens=lens)
+    qts = [_absorbed(case, l) for l in range(1 + F)]
+    c8, cs, ln = case.c8.to(DEV), case.cs.to(DEV), case.lens.to(DEV)
+    sc = api.li_latent_score_fp8(qts[0], case.w[0].to(DEV), c8, cs, lens=ln)
+    cand = api.li_topk(sc, C, lens=ln, max_len=L)
+    qt_f = torch.stack(qts[1:]).contiguous()
+    wf = case.w[1:].contiguous()
+    out = api.li_hs_refine_fp8(c8, cs, cand, qt_f, wf.to(DEV), k)
+    ref, cscores = oracle.hs_refine_fp8(qt_f.cpu(), wf, case.c8, case.cs, _np(cand), k, with_scores=True)
+    g = _np(out)
+    for f in range(F):
+        for b in range(B):
+            cb = _np(cand)[b]
+            assert set(g[f, b][g[f, b] >= 0].tolist()) <= set(cb[cb >= 0].tolist())
+            pos = {int(p): i for i, p in enumerate(cb) if p >= 0}
+            gi = np.array([[pos[int(p)] for p in g[f, b] if p >= 0] + [-1] * int((g[f, b] < 0).sum())])
+            ri = np.array([[pos[int(p)] for p in ref[f, b] if p >= 0] + [-1] * int((ref[f, b] < 0).sum())])
+            assert_topk_equivalent(gi, ri, cscores[f, b:b + 1], 1e-2)
+    assert api.li_get_last_error() == LI_OK
+
+
+def test_hs_fp8_out_of_range_candidate_reported():
+    case = synth.latent_rope_nope(B=1, L=500, G=2, seed=77)
+    qt = _absorbed(case, 1)
+    cand = torch.tensor([[3, 7, 499, 500]], dtype=torch.int32, device=DEV)  # 500: one past the cache
+    api.li_hs_refine_fp8(case.c8.to(DEV), case.cs.to(DEV), cand, qt[None].contiguous(),
+                         case.w[1:2].contiguous().to(DEV), 2)
+    from sparse_attention_lightning_score_b200._lib import LI_ERR_BOUNDS
+    assert api.li_get_last_error() == LI_ERR_BOUNDS

@@ -482,3 +482,36 @@ def test_sparse_attention_invariants():
     # no valid selection: zero
     none = np.full((2, 4), -1)
     assert np.all(oracle.sparse_attention(q, kv, none, 0.5, dv=dv) == 0.0)
+
+
+def _hs8_case(seed=21, B=2, L=120, F=2, H=3):
+    g = torch.Generator().manual_seed(seed)
+    c = torch.randn(B, L, 12, generator=g)
+    from sparse_attention_lightning_score_b200 import synth as sy
+    c8, cs = sy.encode_e4m3_cache(c.view(B * L, 12))
+    qt = torch.randn(F, B, H, 12, generator=g).to(torch.bfloat16)
+    w = torch.randn(F, B, H, generator=g)
+    return qt, w, c8.view(B, L, 12), cs.view(B, L)
+
+
+def test_hs_fp8_all_positions_as_candidates_is_full_selection():
+    qt, w, c8, cs = _hs8_case()
+    B, L = c8.shape[0], c8.shape[1]
+    cand = np.tile(np.arange(L, dtype=np.int32), (B, 1))
+    out = oracle.hs_refine_fp8(qt, w, c8, cs, cand, 7)
+    for f in range(qt.shape[0]):
+        q8, sq, _ = oracle.quantize_query(qt[f], w[f].numpy())
+        full = oracle.index_score(q8, oracle.E4M3, w[f], c8, oracle.E4M3, q_scale=sq, k_scale=cs, k_batch_rows=L, L=L)
+        idx, _ = oracle.topk(full, 7)
+        assert np.array_equal(out[f], idx)
+
+
+def test_hs_fp8_k_equal_to_candidates_and_padding():
+    qt, w, c8, cs = _hs8_case()
+    cand = np.array([[3, 17, 40, 99, -1, -1], [0, 5, 6, 7, 8, 119]], np.int32)
+    out = oracle.hs_refine_fp8(qt, w, c8, cs, cand, 6)
+    for f in range(qt.shape[0]):
+        assert out[f, 0].tolist() == [3, 17, 40, 99, -1, -1]     # pads never selected
+        assert out[f, 1].tolist() == [0, 5, 6, 7, 8, 119]
+    out = oracle.hs_refine_fp8(qt, w, c8, cs, np.full((2, 4), -1, np.int32), 3)
+    assert np.all(out == -1)
