@@ -100,89 +100,52 @@ __global__ void __launch_bounds__(128) simt_score_kernel(const SimtArgs a) {
 // once.  Partial sums over the 32 row groups are reduced with warp shuffles,
 // then across the 8 warps through shared memory.
 // ---------------------------------------------------------------------------
-constexpr int AB_BCH = 4;     // requests per pass over the registers of W
-constexpr int AB_MAXR = 8;    // rows per thread: d <= 256
+constexpr int AB_COLS = 64;   // output columns per CTA
+constexpr int AB_BMAX = 32;   // requests staged per pass
 
+__host__ __device__ constexpr size_t ab_smem(int d) {
+    return (size_t)d * AB_COLS * 2 + (size_t)AB_BMAX * (d + 1) * 4;
+}
+
+// One CTA per (head j, 64 output columns, layer): the W slice [d x 64] and up to 32 requests'
+// query rows are staged in shared memory with one round trip; thread t owns column t % 64 for the
+// requests t / 64, t / 64 + 4, ... and sums over d in its registers (fp32, in order of e), then
+// rounds once to bf16.
 __global__ void __launch_bounds__(256) absorb_kernel(const __nv_bfloat16* __restrict__ q,
                                                      const __nv_bfloat16* __restrict__ W,
                                                      __nv_bfloat16* __restrict__ qt, int B, int H, int d, int dc) {
-    __shared__ float qsh[AB_BCH][256];
-    __shared__ float red[8][AB_BCH][64];
+    extern __shared__ __align__(16) uint8_t ab_smem_raw[];
+    __nv_bfloat16* wsh = reinterpret_cast<__nv_bfloat16*>(ab_smem_raw);                 // [d][64]
+    float* qsh = reinterpret_cast<float*>(ab_smem_raw + (size_t)d * AB_COLS * 2);       // [32][d + 1]
     const int j = blockIdx.x;
-    const int c0 = blockIdx.y * 64;
+    const int c0 = blockIdx.y * AB_COLS;
     // layer blockIdx.z: its queries, decoder and output follow the previous layer's
     q += (size_t)blockIdx.z * B * H * d;
     W += (size_t)blockIdx.z * H * d * dc;
     qt += (size_t)blockIdx.z * B * H * dc;
-    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    const int rg = t >> 3;   // row group 0..31
-    const int cg = t & 7;    // 8 columns c0+8cg .. c0+8cg+7
-    // the block's slice of W: all loads first
-    uint4 wv[AB_MAXR];
-#pragma unroll
-    for (int i = 0; i < AB_MAXR; ++i) {
-        const int e = rg + 32 * i;
-        wv[i] = e < d ? __ldg(reinterpret_cast<const uint4*>(W + ((size_t)j * d + e) * dc + c0) + cg)
-                      : make_uint4(0u, 0u, 0u, 0u);
+    const int t = threadIdx.x;
+    // W slice: d rows x 128 bytes, eight 16-byte units per row
+    for (int u = t; u < d * 8; u += 256) {
+        const int e = u >> 3, v = u & 7;
+        *reinterpret_cast<uint4*>(wsh + e * AB_COLS + 8 * v) =
+            __ldg(reinterpret_cast<const uint4*>(W + ((size_t)j * d + e) * dc + c0) + v);
     }
-    for (int b0 = 0; b0 < B; b0 += AB_BCH) {
-        const int nb = min(AB_BCH, B - b0);
-        __syncthreads();
-        for (int i = t; i < AB_BCH * d; i += 256) {
-            const int bb = i / d, e = i % d;
-            qsh[bb][e] = bb < nb ? __bfloat162float(q[((size_t)(b0 + bb) * H + j) * d + e]) : 0.f;
+    const int c = t & (AB_COLS - 1);
+    for (int b0 = 0; b0 < B; b0 += AB_BMAX) {
+        const int nb = min(AB_BMAX, B - b0);
+        for (int i = t; i < nb * d; i += 256) {
+            const int bb = i / d, e = i - bb * d;
+            qsh[bb * (d + 1) + e] = __bfloat162float(q[((size_t)(b0 + bb) * H + j) * d + e]);
         }
         __syncthreads();
-        float acc[AB_BCH][8];
-#pragma unroll
-        for (int bb = 0; bb < AB_BCH; ++bb)
-#pragma unroll
-            for (int x = 0; x < 8; ++x) acc[bb][x] = 0.f;
-#pragma unroll
-        for (int i = 0; i < AB_MAXR; ++i) {
-            const int e = rg + 32 * i;
-            if (e < d) {
-                const uint32_t wp[4] = {wv[i].x, wv[i].y, wv[i].z, wv[i].w};
-                float wf[8];
-#pragma unroll
-                for (int x = 0; x < 4; ++x) {
-                    wf[2 * x] = __uint_as_float(wp[x] << 16);
-                    wf[2 * x + 1] = __uint_as_float(wp[x] & 0xffff0000u);
-                }
-#pragma unroll
-                for (int bb = 0; bb < AB_BCH; ++bb) {
-                    const float qv = qsh[bb][e];
-#pragma unroll
-                    for (int x = 0; x < 8; ++x) acc[bb][x] = fmaf(qv, wf[x], acc[bb][x]);
-                }
-            }
-        }
-        // reduce the 4 row groups of this warp (lanes that differ in bits 3, 4)
-#pragma unroll
-        for (int bb = 0; bb < AB_BCH; ++bb)
-#pragma unroll
-            for (int x = 0; x < 8; ++x) {
-                float v = acc[bb][x];
-                v += __shfl_xor_sync(0xffffffffu, v, 8);
-                v += __shfl_xor_sync(0xffffffffu, v, 16);
-                acc[bb][x] = v;
-            }
-        if (lane < 8) {
-#pragma unroll
-            for (int bb = 0; bb < AB_BCH; ++bb)
-#pragma unroll
-                for (int x = 0; x < 8; ++x) red[warp][bb][8 * cg + x] = acc[bb][x];
+        for (int bb = t >> 6; bb < nb; bb += 4) {
+            const float* qr = qsh + bb * (d + 1);
+            float acc = 0.f;
+#pragma unroll 8
+            for (int e = 0; e < d; ++e) acc = fmaf(qr[e], __bfloat162float(wsh[e * AB_COLS + c]), acc);
+            qt[((size_t)(b0 + bb) * H + j) * dc + c0 + c] = __float2bfloat16_rn(acc);
         }
         __syncthreads();
-        {
-            const int bb = t >> 6, c = t & 63;  // 256 threads = 4 requests x 64 columns
-            if (bb < nb) {
-                float sum = 0.f;
-#pragma unroll
-                for (int w = 0; w < 8; ++w) sum += red[w][bb][c];
-                qt[((size_t)(b0 + bb) * H + j) * dc + c0 + c] = __float2bfloat16_rn(sum);
-            }
-        }
     }
 }
 
@@ -263,7 +226,16 @@ li_status launch_simt_score(const SimtArgs& a, cudaStream_t st) {
 li_status launch_absorb(const void* q, const void* wdec, void* qt, int G, int B, int H, int d, int dc,
                         cudaStream_t st) {
     if (B == 0 || G == 0) return LI_OK;
-    absorb_kernel<<<dim3(H, dc / 64, G), 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(q),
+    static bool attr_done[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_done[dev]) {
+        if (cudaFuncSetAttribute(absorb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ab_smem(256)) !=
+            cudaSuccess)
+            return host_check_launch();
+        attr_done[dev] = true;
+    }
+    absorb_kernel<<<dim3(H, dc / 64, G), 256, ab_smem(d), st>>>(reinterpret_cast<const __nv_bfloat16*>(q),
                                                      reinterpret_cast<const __nv_bfloat16*>(wdec),
                                                      reinterpret_cast<__nv_bfloat16*>(qt), B, H, d, dc);
     return host_check_launch();
