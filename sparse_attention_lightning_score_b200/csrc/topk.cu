@@ -668,11 +668,11 @@ li_status launch_topk(const TopkArgs& a, cudaStream_t st) {
         const int nr = min(65535, a.rows - row0);
         cudaError_t e;
         if (a.hist) {
-            if (cs == 1) e = small ? launch_one<256, false, true>(a, row0, nr, cs, chunk, st)
+            if (cs == 1) e = small ? launch_one<512, false, true>(a, row0, nr, cs, chunk, st)
                                    : launch_one<1024, false, true>(a, row0, nr, cs, chunk, st);
             else e = launch_one<512, true, true>(a, row0, nr, cs, chunk, st);
         } else {
-            if (cs == 1) e = small ? launch_one<256, false, false>(a, row0, nr, cs, chunk, st)
+            if (cs == 1) e = small ? launch_one<512, false, false>(a, row0, nr, cs, chunk, st)
                                    : launch_one<1024, false, false>(a, row0, nr, cs, chunk, st);
             else e = launch_one<512, true, false>(a, row0, nr, cs, chunk, st);
         }
