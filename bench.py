@@ -605,7 +605,7 @@ class HsBench:
         self.sc = torch.empty((B, self.L), dtype=torch.float32, device=dev)
         self.cand = torch.empty((B, self.C), dtype=torch.int32, device=dev)
         self.out = torch.empty((3, B, KTOP), dtype=torch.int32, device=dev)
-        self.ws = torch.empty(3 * B * self.C * 4, dtype=torch.uint8, device=dev)
+        self.ws = api.li_hs_refine_workspace(B, self.C, 3, dev)
 
     def step(self, i):
         import torch
@@ -729,7 +729,7 @@ def run_table4(dev, args, clocks):
         lsc = torch.empty((1, Lx), dtype=torch.float32, device=dev)
         cand = torch.empty((1, C), dtype=torch.int32, device=dev)
         out = torch.empty((3, 1, KTOP), dtype=torch.int32, device=dev)
-        hws = torch.empty(3 * C * 4, dtype=torch.uint8, device=dev)
+        hws = api.li_hs_refine_workspace(1, C, 3, dev)
         side = torch.cuda.Stream(device=dev)
         # the same methods over DeepSeek-V3.2's FP8 latent (d_c = 192 e4m3, one scale per row)
         fcase = synth.latent_rope_nope(B=1, L=Lx, G=4, seed=5)

@@ -320,7 +320,15 @@ li_status li_latent_score_fp8(const void* q_tilde_bf16, const float* w, const vo
  * Candidates outside [0, rows of c) are reported as LI_ERR_BOUNDS by
  * li_get_last_error and are not read.  heads == 64 or 32, latent_dim == 256,
  * 1 <= followers <= 4, n_cand <= LI_TOPK_MAX_LEN.
- * workspace: li_hs_refine_workspace(...) bytes. */
+ * workspace: workspace_bytes >= li_hs_refine_workspace(...) bytes of device
+ *   memory, 16-byte aligned.  Its first part holds the candidate scores; its
+ *   last followers * batch * 8 KB (from workspace_bytes back, rounded down to
+ *   16 bytes) hold the rescoring kernel's first-digit histograms for the
+ *   follower top-k, as li_topk_hist uses them.  Zero the workspace once after
+ *   allocating it; each call leaves those histograms zero again when its
+ *   kernels finish.  If they were not zero, the result is the same, only
+ *   slower: the top-k checks each histogram against its keys, falls back to
+ *   its plain passes and reports LI_ERR_BOUNDS through li_get_last_error. */
 li_status li_hs_refine(const void* c_bf16, int64_t cache_batch_rows, int64_t cache_rows, const int32_t* cand,
                        int batch, int n_cand, const void* q_tilde_bf16, const float* w, int followers, int heads,
                        int latent_dim, int k, int32_t* out_idx, void* workspace, size_t workspace_bytes,
@@ -344,8 +352,11 @@ size_t li_hs_refine_workspace(int batch, int n_cand, int followers);
  *   - followers * batch * round_up(n_cand, 4) above that capacity returns
  *     LI_ERR_INVALID_ARG before anything is launched.
  *   - The array is shared by all calls on a device and keeps the last call's
- *     contents; nothing in it needs to start at zero.  Calls that overlap on
- *     the GPU (unordered streams) race on it: serialise them.
+ *     contents; its histogram part (the last followers * batch * 8 KB) starts
+ *     zero at load and each call leaves it zero, and a call whose histograms
+ *     overlap an earlier, larger call's scores still gives the same result.
+ *     Calls that overlap on the GPU (unordered streams) race on it: serialise
+ *     them.
  *   - The first call on a device looks up the array's device address; make
  *     that first call before any stream capture begins. */
 /* li_hs_refine over DeepSeek-V3.2's FP8 latent (LatentIndex appendix, Table 5:

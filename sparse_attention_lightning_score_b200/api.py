@@ -358,6 +358,12 @@ def li_latent_score(q_tilde: torch.Tensor, w: torch.Tensor, c: torch.Tensor, *, 
     return scores
 
 
+def li_hs_refine_workspace(batch: int, n_cand: int, followers: int, device) -> torch.Tensor:
+    """A zeroed workspace for li_hs_refine / li_hs_refine_fp8 (its histogram part stays zero between calls)."""
+    need = _lib.load().li_hs_refine_workspace(int(batch), int(n_cand), int(followers))
+    return torch.zeros(max(int(need), 16), dtype=torch.uint8, device=device)
+
+
 def li_hs_refine(c: torch.Tensor, cand: torch.Tensor, q_tilde: torch.Tensor, w: torch.Tensor, k: int, *,
                  out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None, stream=None):
     """Followers re-score the anchor's candidates and keep their own top-k.
@@ -376,7 +382,7 @@ def li_hs_refine(c: torch.Tensor, cand: torch.Tensor, q_tilde: torch.Tensor, w: 
     lib = _lib.load()
     need = lib.li_hs_refine_workspace(B, C, F)
     if workspace is None or workspace.numel() * workspace.element_size() < need:
-        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=c.device)
+        workspace = li_hs_refine_workspace(B, C, F, c.device)
     if out is None:
         out = torch.empty((F, B, k), dtype=torch.int32, device=c.device)
     st = lib.li_hs_refine(_ptr(c), batch_rows, cache_rows, _ptr(cand), B, C, _ptr(q_tilde), _ptr(w), F, H, dc, int(k),
@@ -437,7 +443,7 @@ def li_hs_refine_fp8(c8: torch.Tensor, c_scale: torch.Tensor, cand: torch.Tensor
     lib = _lib.load()
     need = lib.li_hs_refine_workspace(B, C, F)
     if workspace is None or workspace.numel() * workspace.element_size() < need:
-        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=c8.device)
+        workspace = li_hs_refine_workspace(B, C, F, c8.device)
     if out is None:
         out = torch.empty((F, B, k), dtype=torch.int32, device=c8.device)
     st = lib.li_hs_refine_fp8(_ptr(c8), _ptr(c_scale), batch_rows, cache_rows, _ptr(cand), B, C, _ptr(q_tilde),

@@ -14,7 +14,9 @@
 // the cache are reported (LI_ERR_BOUNDS) and zero-filled, never read.
 //
 // Warps: 0..3 gather producers, 4 TMEM allocator + MMA issuer, 5..8 follower
-// query preparation and epilogue.  Output: scores [F*B, round4(C)] fp32.
+// query preparation and epilogue.  Output: scores [F*B, round4(C)] fp32, and
+// (optionally) each row's first-digit histogram for the follower top-k, counted
+// by the epilogue warps with one global atomic per distinct digit per warp.
 #include "li_common.cuh"
 #include "li_kernels.cuh"
 
@@ -212,7 +214,8 @@ __global__ void __launch_bounds__(HS_THREADS, 1) hs_rescore_kernel(const HsArgs 
             const int acc = it & 1;
             const int i = (t0 + it) * HS_M + g * 32 + lane;
             const int s = i < a.C ? __ldg(cand + i) : -1;
-            if (!mbar_wait(&accf[acc], (it >> 1) & 1, a.err)) break;
+            // warp-uniform exit: the histogram below needs every lane of the warp
+            if (!__all_sync(0xffffffffu, mbar_wait(&accf[acc], (it >> 1) & 1, a.err))) break;
             tc_fence_after();
             float res[F];
 #pragma unroll
@@ -233,10 +236,11 @@ __global__ void __launch_bounds__(HS_THREADS, 1) hs_rescore_kernel(const HsArgs 
             }
             tc_fence_before();
             mbar_arrive(&acce[acc]);
-            if (i < a.C) {
 #pragma unroll
-                for (int f = 0; f < F; ++f)
-                    a.out[((size_t)f * a.B + b) * ldw + i] = s >= 0 ? res[f] : -INFINITY;
+            for (int f = 0; f < F; ++f) {
+                const float v = s >= 0 ? res[f] : -INFINITY;
+                if (i < a.C) a.out[((size_t)f * a.B + b) * ldw + i] = v;
+                if (a.hist) warp_hist_add(a.hist + ((size_t)f * a.B + b) * LI_HIST_BINS, v, i < a.C);
             }
         }
     }

@@ -18,7 +18,8 @@
 // reported (LI_ERR_BOUNDS) and zero-filled, never read.
 //
 // Warps: 0..3 gather producers, 4 TMEM allocator + MMA issuer, 5..8 follower
-// query quantisation, then the epilogue.  Output: scores [F*B, round4(C)].
+// query quantisation, then the epilogue.  Output: scores [F*B, round4(C)] and
+// (optionally) each row's first-digit histogram, as the bf16 kernel counts it.
 #include "li_common.cuh"
 #include "li_kernels.cuh"
 
@@ -257,7 +258,8 @@ __global__ void __launch_bounds__(H8_THREADS, 1) hs_rescore8_kernel(const Hs8Arg
             const int i = (t0 + it) * H8_M + g * 32 + lane;
             const int s = i < a.C ? __ldg(cand + i) : -1;
             const float scale = (s >= 0 && s < lim) ? __ldg(a.cscale + rowbase + s) : 0.f;
-            if (!mbar_wait(&accf[acc], (it >> 1) & 1, a.err)) break;
+            // warp-uniform exit: the histogram below needs every lane of the warp
+            if (!__all_sync(0xffffffffu, mbar_wait(&accf[acc], (it >> 1) & 1, a.err))) break;
             tc_fence_after();
             float res[F];
 #pragma unroll
@@ -271,10 +273,11 @@ __global__ void __launch_bounds__(H8_THREADS, 1) hs_rescore8_kernel(const Hs8Arg
             }
             tc_fence_before();
             mbar_arrive(&acce[acc]);
-            if (i < a.C) {
 #pragma unroll
-                for (int f = 0; f < F; ++f)
-                    a.out[((size_t)f * a.B + b) * ldw + i] = s >= 0 ? res[f] * scale : -INFINITY;
+            for (int f = 0; f < F; ++f) {
+                const float v = s >= 0 ? res[f] * scale : -INFINITY;
+                if (i < a.C) a.out[((size_t)f * a.B + b) * ldw + i] = v;
+                if (a.hist) warp_hist_add(a.hist + ((size_t)f * a.B + b) * LI_HIST_BINS, v, i < a.C);
             }
         }
     }

@@ -14,10 +14,12 @@
 //   - Calls with followers * batch * round_up(n_cand, 4) floats beyond that
 //     are rejected with LI_ERR_INVALID_ARG before anything is launched.
 //   - All calls on a device share the one array and it keeps the previous
-//     call's contents.  Nothing in it needs to start at zero: every score slot
-//     the selection reads is written first by the same call.  Calls that
-//     overlap on the GPU (different streams, no ordering between them) race
-//     on the array and must be serialised by the caller.
+//     call's contents.  Every score slot the selection reads is written first
+//     by the same call.  The follower top-k's histograms sit at the array's
+//     end: zero at load, left zero by every call, and only a speed-up (a
+//     histogram that disagrees with the keys sends the top-k to its plain
+//     passes).  Calls that overlap on the GPU (different streams, no ordering
+//     between them) race on the array and must be serialised by the caller.
 //   - The first call on a device looks up the array's device address (set-up);
 //     make that first call before any stream capture begins.
 #include <cuda_runtime.h>

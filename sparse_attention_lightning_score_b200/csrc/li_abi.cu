@@ -56,6 +56,14 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// The followers' first-digit histograms sit at the END of the workspace the caller gives (so
+// that a fixed scratch shared by calls of different sizes keeps them in one place).
+size_t hs_hist_bytes(int batch, int followers) { return (size_t)followers * batch * LI_HIST_BINS * sizeof(uint32_t); }
+uint32_t* hs_hist_of(void* workspace, size_t workspace_bytes, int batch, int followers) {
+    return reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) +
+                                       ((workspace_bytes - hs_hist_bytes(batch, followers)) & ~(size_t)15));
+}
+
 }  // namespace
 
 DevErr host_dev_err() {
@@ -470,7 +478,8 @@ li_status li_latent_score_fp8(const void* q_tilde_bf16, const float* w, const vo
 
 size_t li_hs_refine_workspace(int batch, int n_cand, int followers) {
     if (batch <= 0 || n_cand <= 0 || followers <= 0) return 0;
-    return (size_t)followers * batch * align_up((size_t)n_cand, 4) * sizeof(float);
+    return align_up((size_t)followers * batch * align_up((size_t)n_cand, 4) * sizeof(float), 16) +
+           hs_hist_bytes(batch, followers);
 }
 
 li_status li_hs_refine(const void* c_bf16, int64_t cache_batch_rows, int64_t cache_rows, const int32_t* cand,
@@ -496,11 +505,12 @@ li_status li_hs_refine(const void* c_bf16, int64_t cache_batch_rows, int64_t cac
     if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) return LI_ERR_INVALID_ARG;
     const int ldw = (int)align_up((size_t)n_cand, 4);
     float* sc = static_cast<float*>(workspace);
-    HsArgs h{c_bf16, cache_batch_rows, cache_rows, cand, batch, n_cand, followers, heads, q_tilde_bf16, w, sc, e};
+    uint32_t* hist = hs_hist_of(workspace, workspace_bytes, batch, followers);
+    HsArgs h{c_bf16, cache_batch_rows, cache_rows, cand, batch, n_cand, followers, heads, q_tilde_bf16, w, sc, hist, e};
     li_status s = launch_hs_rescore(h, stream);
     if (s != LI_OK) return s;
     TopkArgs t{sc, ldw, nullptr, followers * batch, n_cand, 0, 0, k, out_idx, nullptr, cand, n_cand, batch,
-               nullptr, 0, 1, e};
+               hist, 0, 1, e};
     return launch_topk(t, stream);
 }
 
@@ -527,11 +537,12 @@ li_status li_hs_refine_fp8(const void* c_e4m3, const float* c_scale, int64_t cac
     if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) return LI_ERR_INVALID_ARG;
     const int ldw = (int)align_up((size_t)n_cand, 4);
     float* sc = static_cast<float*>(workspace);
-    Hs8Args h{c_e4m3, c_scale, cache_batch_rows, cache_rows, cand, batch, n_cand, followers, q_tilde_bf16, w, sc, e};
+    uint32_t* hist = hs_hist_of(workspace, workspace_bytes, batch, followers);
+    Hs8Args h{c_e4m3, c_scale, cache_batch_rows, cache_rows, cand, batch, n_cand, followers, q_tilde_bf16, w, sc, hist, e};
     li_status s = launch_hs_rescore8(h, stream);
     if (s != LI_OK) return s;
     TopkArgs t{sc, ldw, nullptr, followers * batch, n_cand, 0, 0, k, out_idx, nullptr, cand, n_cand, batch,
-               nullptr, 0, 1, e};
+               hist, 0, 1, e};
     return launch_topk(t, stream);
 }
 

@@ -319,6 +319,15 @@ constexpr int LI_HIST_BITS = 11;
 constexpr int LI_HIST_BINS = 1 << LI_HIST_BITS;
 constexpr int LI_HIST_SHIFT = 32 - LI_HIST_BITS;
 
+// Adds each valid lane's score to the global first-digit histogram gh with one
+// atomic per distinct digit in the warp (lanes are grouped by digit).  Every
+// lane of the warp must make the call together.
+__device__ __forceinline__ void warp_hist_add(uint32_t* gh, float v, bool valid) {
+    const uint32_t bin = valid ? (order_key(v) >> LI_HIST_SHIFT) : 0xffffffffu;
+    const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+    if (valid && (int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(gh + bin, (uint32_t)__popc(peers));
+}
+
 // acc.{x,y} += a.{0,1} * b.{0,1} with one packed fp32x2 FMA (same rounding as two fmaf).
 __device__ __forceinline__ void ffma2(float2& acc, float a0, float a1, float b0, float b1) {
     asm("{\n\t.reg .b64 ra, rb, rc;\n\t"

@@ -134,6 +134,7 @@ struct HsArgs {
     const void* qt;         // bf16 [F,B,H,256]
     const float* w;         // [F,B,H]
     float* out;             // [F,B,C] candidate scores (workspace)
+    uint32_t* hist;         // optional [F*B, LI_HIST_BINS]: out's first-digit counts are added here
     DevErr err;
 };
 li_status launch_hs_rescore(const HsArgs& a, cudaStream_t st);
@@ -149,6 +150,7 @@ struct Hs8Args {
     const void* qt;         // bf16 [F,B,64,192]
     const float* w;         // [F,B,64]
     float* out;             // [F,B,round4(C)] candidate scores (workspace)
+    uint32_t* hist;         // optional [F*B, LI_HIST_BINS]: out's first-digit counts are added here
     DevErr err;
 };
 li_status launch_hs_rescore8(const Hs8Args& a, cudaStream_t st);

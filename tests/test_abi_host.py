@@ -99,7 +99,8 @@ def test_workspace_sizes():
     assert lib.li_index_score_workspace(ctypes.byref(d)) >= 8192 * 64 * (128 + 8)
     d.causal = 0
     assert lib.li_index_score_workspace(ctypes.byref(d)) == 0
-    assert lib.li_hs_refine_workspace(16, 8192, 3) == 3 * 16 * 8192 * 4
+    assert lib.li_hs_refine_workspace(16, 8192, 3) == 3 * 16 * 8192 * 4 + 3 * 16 * 2048 * 4  # scores + histograms
+    assert lib.li_hs_refine_workspace(1, 5, 2) == 2 * 8 * 4 + 2 * 2048 * 4
 
 
 def test_latent_fp8_and_layers_reject_bad_arguments_on_host():

@@ -127,6 +127,29 @@ def test_hs_fp8_matches_oracle(B, L, C, k, F, lens):
     assert api.li_get_last_error() == LI_OK
 
 
+def test_hs_fp8_histogram_path_equals_plain_passes():
+    # as for the bf16 latent: dirty histograms give the same selection, are reported and healed
+    from sparse_attention_lightning_score_b200._lib import LI_ERR_BOUNDS
+    F, C, k = 3, 8192, 2048
+    case = synth.latent_rope_nope(B=2, L=20000, G=1 + F, seed=91)
+    qts = [_absorbed(case, l) for l in range(1 + F)]
+    c8, cs = case.c8.to(DEV), case.cs.to(DEV)
+    sc = api.li_latent_score_fp8(qts[0], case.w[0].to(DEV), c8, cs)
+    cand = api.li_topk(sc, C, max_len=20000)
+    qt_f = torch.stack(qts[1:]).contiguous()
+    wf = case.w[1:].contiguous().to(DEV)
+    ws = api.li_hs_refine_workspace(2, C, F, DEV)
+    tail = ws[ws.numel() - F * 2 * 2048 * 4:]
+    out = api.li_hs_refine_fp8(c8, cs, cand, qt_f, wf, k, workspace=ws)
+    torch.cuda.synchronize()
+    assert api.li_get_last_error() == LI_OK and int(tail.count_nonzero()) == 0
+    tail.view(torch.int32)[::5] = 1
+    dirty = api.li_hs_refine_fp8(c8, cs, cand, qt_f, wf, k, workspace=ws)
+    torch.cuda.synchronize()
+    assert api.li_get_last_error() == LI_ERR_BOUNDS and int(tail.count_nonzero()) == 0
+    assert torch.equal(out, dirty)
+
+
 def test_hs_fp8_out_of_range_candidate_reported():
     case = synth.latent_rope_nope(B=1, L=500, G=2, seed=77)
     qt = _absorbed(case, 1)

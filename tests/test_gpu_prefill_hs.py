@@ -121,6 +121,30 @@ def test_hs_out_of_range_candidate_reported():
     assert api.li_get_last_error() == LI_OK
 
 
+@pytest.mark.parametrize("C,k", [(8192, 2048), (640, 100)])
+def test_hs_histogram_path_equals_plain_passes(C, k):
+    # the rescoring kernel counts each follower row's first-digit histogram for the top-k; a
+    # workspace whose histograms are dirty must give the same selection (plain passes), be
+    # reported, and be left zero
+    case = synth.latent_hs(B=2, L=20000, n_cand=C, k_top=k, seed=90)
+    c = case.c.to(DEV)
+    qts, sc, cand, qt_f = _gpu_anchor_and_followers(case, C, c)
+    w = case.w[1:].contiguous().to(DEV)
+    F = qt_f.shape[0]
+    ws = api.li_hs_refine_workspace(2, C, F, DEV)
+    tail = ws[ws.numel() - F * 2 * 2048 * 4:]
+    out = api.li_hs_refine(c, cand, qt_f, w, k, workspace=ws)
+    torch.cuda.synchronize()
+    assert api.li_get_last_error() == LI_OK and int(tail.count_nonzero()) == 0
+    tail.view(torch.int32)[::7] = 3
+    dirty = api.li_hs_refine(c, cand, qt_f, w, k, workspace=ws)
+    torch.cuda.synchronize()
+    assert api.li_get_last_error() == LI_ERR_BOUNDS and int(tail.count_nonzero()) == 0
+    assert torch.equal(out, dirty)
+    again = api.li_hs_refine(c, cand, qt_f, w, k, workspace=ws)
+    assert torch.equal(out, again) and api.li_get_last_error() == LI_OK
+
+
 @pytest.mark.parametrize("B", [1, 16])
 def test_hs_full_size(B):
     """The HS configuration at full size (L = 131072, C = 8192, 3 followers, k = 2048)."""
