@@ -353,39 +353,39 @@ __device__ __forceinline__ float relu_dot32_x2(const uint32_t (&v)[32], const fl
     return (a0.x + a0.y) + (a1.x + a1.y);
 }
 
-// e4m3(x / sq) (round to nearest even, saturating) with the quotient rounded as
-// IEEE fp32 division rounds it, at the cost of one multiply in most calls.
-// With r the correctly rounded reciprocal of sq, y = x * r lies within 2.5 ulp
-// of the correctly rounded quotient q (each of the two roundings is a relative
-// error of at most 2^-24).  y and q then round to the same e4m3 value unless an
-// e4m3 rounding midpoint lies between them.  For |y| in e4m3's normal range,
-// those midpoints are the values whose 20 low mantissa bits are 0x80000.  So
-// only a product within 8 ulp of such a point, or outside [2^-6, 512] (e4m3
-// subnormals, zero, an overflowed reciprocal, NaN), needs the division.
-//
-// (An exact division-free decision also exists: the residual M sq - x against
-// the midpoint M is exact near M and decides ties and sides.  It was checked
-// exhaustively and measured; it is built from integer and logic operations,
-// whose pipe then throttles the quantiser, so the division stays.)
-__device__ __forceinline__ bool quotient_needs_division(float y) {
-    const float ay = fabsf(y);
-    const uint32_t m = __float_as_uint(y) & 0xfffffu;
-    return !(ay >= 0x1p-6f && ay <= 512.f) || (m - 0x7fff8u) <= 16u;
-}
-
-// y[i] = x[i] / sq rounded as IEEE division, for N elements of every lane.  The
-// products are taken first; when any lane of the warp has an element that needs
-// it, the whole warp divides instead (warp-uniform, so the rare path costs no
-// divergent branch per element).  All 32 lanes must call this together.
+// y[i] = x[i] / sq rounded as IEEE fp32 division rounds it (nearest even), for
+// the e4m3 conversion that follows, without a division in the common case.
+// Method: Markstein's FMA correction of an approximate quotient (P. Markstein,
+// "Computation of elementary functions on the IBM RISC System/6000 processor",
+// IBM J. Res. Dev. 34(1), 1990; Muller et al., Handbook of Floating-Point
+// Arithmetic, the FMA-based division chapter).  With r the correctly rounded
+// reciprocal of sq:
+//   y0 = RN(x r)                      within about 2.5 ulp of x / sq
+//   y1 = RN(y0 + RN(x - y0 sq) r)     faithful (within 1 ulp)
+//   y  = RN(y1 + RN(x - y1 sq) r)     correctly rounded: the residual of a
+//                                     faithful quotient is exact with an FMA,
+//                                     and r is within half an ulp of 1/sq.
+// The residuals stay clear of underflow while sq >= 2^-90 and |x / sq| >= 2^-11;
+// smaller quotients can be off by an ulp, but every value below 2^-10 converts
+// to an e4m3 zero of the same sign either way.  A zero x keeps its sign (the
+// FMA steps would turn -0 into +0).  Scales outside [2^-90, 2^127] (tiny, or
+// inf / NaN from a non-finite head) make the whole warp divide instead.
+// (Before this, a product x r was taken and the warp divided whenever one of
+// its quotients fell within 8 ulp of an e4m3 rounding midpoint; bf16 inputs hit
+// exact midpoints so often that most warps divided.)
+// All 32 lanes must call this together.
 template <int N>
 __device__ __forceinline__ void quotients_for_e4m3(const float (&x)[N], float sq, float r, float (&y)[N]) {
-    bool need = false;
+    const bool sq_ok = sq >= 0x1p-90f && sq <= 0x1p127f;
+    if (__all_sync(0xffffffffu, sq_ok)) {
 #pragma unroll
-    for (int i = 0; i < N; ++i) {
-        y[i] = x[i] * r;
-        need |= quotient_needs_division(y[i]);
-    }
-    if (__any_sync(0xffffffffu, need)) {
+        for (int i = 0; i < N; ++i) {
+            const float y0 = __fmul_rn(x[i], r);
+            const float y1 = __fmaf_rn(__fmaf_rn(-y0, sq, x[i]), r, y0);
+            const float y2 = __fmaf_rn(__fmaf_rn(-y1, sq, x[i]), r, y1);
+            y[i] = __uint_as_float((__float_as_uint(y2) & 0x7fffffffu) | (__float_as_uint(x[i]) & 0x80000000u));
+        }
+    } else {
 #pragma unroll
         for (int i = 0; i < N; ++i) y[i] = __fdiv_rn(x[i], sq);
     }

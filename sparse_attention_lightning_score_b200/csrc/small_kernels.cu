@@ -10,35 +10,72 @@ namespace li {
 namespace {
 
 // ---------------------------------------------------------------------------
-// Query quantisation: one warp per (row, head).  Same per-(row, head) recipe
-// as the prologue of the FP8 scorer (absmax / 448 scale, the quotient rounded
-// as IEEE division rounds it, nearest-even saturating e4m3 conversion).
+// Query quantisation.  Same per-(row, head) recipe as the prologue of the FP8
+// scorer (absmax / 448 scale, the quotient rounded as IEEE division rounds it,
+// nearest-even saturating e4m3 conversion).  For d = 128 a warp takes four
+// heads at a time (8 lanes per head) and walks a grid-stride list of such
+// groups with the next two groups' loads in flight while it converts one: the
+// conversion is long enough that, without them, too few bytes are in flight to
+// keep HBM busy.  Other d: one warp per (row, head).
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) quantize_query_kernel(const __nv_bfloat16* __restrict__ q,
+constexpr int QZ_BLOCKS_PER_SM = 4;  // 64 registers a thread
+
+// the group's query elements of this lane and, on a head's first lane, its weight
+struct QzIn {
+    uint4 lo, hi;
+    float w;
+};
+
+__device__ __forceinline__ QzIn qz_load(const __nv_bfloat16* __restrict__ q, const float* __restrict__ w,
+                                        long long nheads, long long grp, int lane) {
+    const long long head = grp * 4 + (lane >> 3);
+    QzIn in{make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u), 0.f};
+    if (head < nheads) {
+        const uint4* src = reinterpret_cast<const uint4*>(q + head * 128) + 2 * (lane & 7);
+        in.lo = __ldg(src);
+        in.hi = __ldg(src + 1);
+        if (w && (lane & 7) == 0) in.w = __ldg(w + head);
+    }
+    return in;
+}
+
+// all 32 lanes call it together (the absmax shuffles span the warp's 8-lane groups)
+__device__ __forceinline__ void qz_convert(long long nheads, long long grp, int lane, const QzIn& in,
+                                           uint8_t* __restrict__ q8, float* __restrict__ sq,
+                                           float* __restrict__ w_eff) {
+    const long long head = grp * 4 + (lane >> 3);
+    float s;
+    const uint4 packed = quantize_head128_g8(in.lo, in.hi, &s);
+    if (head < nheads) {
+        reinterpret_cast<uint4*>(q8 + head * 128)[lane & 7] = packed;
+        if ((lane & 7) == 0) {
+            sq[head] = s;
+            if (w_eff) w_eff[head] = in.w * s;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256, QZ_BLOCKS_PER_SM) quantize_query_kernel(const __nv_bfloat16* __restrict__ q,
                                                              const float* __restrict__ w, long long nheads, int dim,
                                                              uint8_t* __restrict__ q8, float* __restrict__ sq,
                                                              float* __restrict__ w_eff) {
     const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
-    if (dim == 128) {  // four heads per warp, 8 lanes per head
-        const long long head = gw * 4 + (lane >> 3);
-        if (gw * 4 >= nheads) return;  // whole warp
-        const bool live = head < nheads;
-        const int l8 = lane & 7;
-        uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
-        if (live) {
-            const uint4* src = reinterpret_cast<const uint4*>(q + head * 128) + 2 * l8;
-            lo = __ldg(src);
-            hi = __ldg(src + 1);
-        }
-        float s;
-        const uint4 packed = quantize_head128_g8(lo, hi, &s);  // all lanes take part in the shuffles
-        if (live) {
-            reinterpret_cast<uint4*>(q8 + head * 128)[l8] = packed;
-            if (l8 == 0) {
-                sq[head] = s;
-                if (w_eff) w_eff[head] = w[head] * s;
+    if (dim == 128) {
+        const long long ngroups = (nheads + 3) / 4;
+        const long long stride = (long long)gridDim.x * (blockDim.x >> 5);
+        const float* wq = w_eff ? w : nullptr;
+        QzIn in_a = qz_load(q, wq, nheads, gw, lane);           // group g
+        QzIn in_b = qz_load(q, wq, nheads, gw + stride, lane);  // group g + stride
+        for (long long g = gw; g < ngroups; g += 2 * stride) {  // g is warp-uniform
+            const QzIn in_c = qz_load(q, wq, nheads, g + 2 * stride, lane);
+            qz_convert(nheads, g, lane, in_a, q8, sq, w_eff);
+            if (g + stride < ngroups) {
+                const QzIn in_d = qz_load(q, wq, nheads, g + 3 * stride, lane);
+                qz_convert(nheads, g + stride, lane, in_b, q8, sq, w_eff);
+                in_b = in_d;
             }
+            in_a = in_c;
         }
         return;
     }
@@ -196,7 +233,8 @@ li_status launch_quantize_query(const void* q, const float* w, int rows, int hea
     const long long nh = (long long)rows * heads;
     if (nh == 0) return LI_OK;
     const long long warps = dim == 128 ? (nh + 3) / 4 : nh;
-    const long long blocks = (warps * 32 + 255) / 256;
+    long long blocks = (warps * 32 + 255) / 256;
+    if (dim == 128) blocks = std::min<long long>(blocks, (long long)host_num_sms() * QZ_BLOCKS_PER_SM);
     quantize_query_kernel<<<(unsigned)blocks, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(q), w, nh, dim, q8,
                                                             sq, w_eff);
     return host_check_launch();
