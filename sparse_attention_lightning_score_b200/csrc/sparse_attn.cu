@@ -159,7 +159,6 @@ __global__ void __launch_bounds__(SA_THREADS, 1)
         tmem_relinquish();
     }
     pdl_wait();  // the selections may come from the previous kernel of the stream
-    pdl_trigger();  // the merge may be scheduled now; it waits for this grid to finish
     if (threadIdx.x == 0) {
         // the 64 query rows of the CTA's heads, first of all (nothing can be consumed before them)
         mbar_arrive_expect_tx(qfull, SA_CH * SA_QCHUNK);
@@ -381,8 +380,6 @@ __global__ void __launch_bounds__(SA_THREADS, 1)
 // the largest m_s (maxima are in the log2 domain).  One CTA per (head, request),
 // four value elements per thread.
 __global__ void __launch_bounds__(128) sparse_attn_merge_kernel(const SparseAttnArgs a) {
-    pdl_trigger();
-    pdl_wait();  // the splits' partials are complete once the main grid has finished
     const int h = blockIdx.x, b = blockIdx.y;
     const int d = threadIdx.x * 4;
     float M = -INFINITY;
@@ -434,8 +431,7 @@ li_status launch_sparse_attn(const CUtensorMap& qmap, SparseAttnArgs a, cudaStre
         return host_check_launch();
     const li_status s = host_check_launch();
     if (s != LI_OK) return s;
-    if (launch_pdl(sparse_attn_merge_kernel, dim3(a.heads, a.batch), dim3(128), 0, st, 1, a) != cudaSuccess)
-        return host_check_launch();
+    sparse_attn_merge_kernel<<<dim3(a.heads, a.batch), 128, 0, st>>>(a);
     return host_check_launch();
 }
 
