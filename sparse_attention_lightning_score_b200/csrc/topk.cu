@@ -185,7 +185,9 @@ __global__ void __launch_bounds__(NT) topk_kernel(const TopkArgs a, int row0, in
 
     pdl_trigger();
     pdl_wait();  // the scores come from the previous kernel of the stream
-    const int r = row0 + blockIdx.y;
+    // causal rows grow with the row index: the longest are dealt first, so that the short ones fill
+    // the SMs at the end of the launch
+    const int r = row0 + (a.causal ? (int)(gridDim.y - 1 - blockIdx.y) : (int)blockIdx.y);
     const int CS = gridDim.x;
     const int c = blockIdx.x;  // == cluster rank: the cluster spans gridDim.x
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
