@@ -162,11 +162,11 @@ def run_reference(args, rank):
     print(json.dumps(out), flush=True)
 
 
-def cpu_baseline_sample():
+def cpu_baseline_sample(heads=H):
     import oracle
     from sparse_attention_lightning_score_b200 import synth
     nthreads = oracle.nthreads_default()
-    case = synth.dsa_decode(B=2, L=L, k_top=KTOP, seed=1)
+    case = synth.dsa_decode(B=2, L=L, H=heads, k_top=KTOP, seed=1)
     t0 = time.perf_counter()
     n = 0
     while True:
@@ -176,11 +176,91 @@ def cpu_baseline_sample():
                                 k_scale=case.ks[r], nthreads=nthreads)
         oracle.topk(sc, KTOP)
         n += 1
-        if time.perf_counter() - t0 > 8.0 or n >= 16:
+        if time.perf_counter() - t0 > 10.0 or n >= 4096:
             break
     t = time.perf_counter() - t0
     return {"value": n * L / t, "unit": "keys/s", "cores": nthreads, "kind": "oracle",
             "sample": f"{n} request(s) of L={L} (quantise+score+top-{KTOP}) on the host, {t:.1f} s"}
+
+
+def oracle_sample(kind, case, budget_s=10.0, heads=H):
+    """The oracle as it stands, timed on the host cores on a bounded sample of a workload (the
+    cpu_baseline object of that workload's JSON line).  `case` is the workload's own synthetic input
+    on the host; the sample is whole requests (or whole causal rows) taken until `budget_s` passes,
+    so its unit matches the workload's."""
+    import numpy as np
+    import torch
+    import oracle
+    nthreads = oracle.nthreads_default()
+    t0 = time.perf_counter()
+    n, units = 0, 0
+
+    def over():
+        return time.perf_counter() - t0 > budget_s
+
+    if kind == "prefill":
+        T = case.q.shape[0]
+        Lk = case.k8.shape[0]
+        while n == 0 or not over():
+            r = T - 1 - (n * 997) % T  # rows of every length, the longest first
+            q8, sq, _ = oracle.quantize_query(case.q[r:r + 1], case.w[r:r + 1].numpy())
+            sc = oracle.index_score(q8, oracle.E4M3, case.w[r:r + 1], case.k8, oracle.E4M3, q_scale=sq,
+                                    k_scale=case.ks, causal=True, causal_offset=r, L=Lk, nthreads=nthreads)
+            oracle.topk(sc, KTOP, causal=True, causal_offset=r, max_len=Lk)
+            units += min(r + 1, Lk)
+            n += 1
+        t = time.perf_counter() - t0
+        return {"value": units / t, "unit": "keys/s (visible pairs)", "cores": nthreads, "kind": "oracle",
+                "sample": f"{n} causal row(s) of T={T} (quantise+score+top-{KTOP}), {units} pairs, {t:.1f} s"}
+    if kind in ("latent", "latent_glm5", "latent192"):
+        fp8 = kind == "latent192"
+        Bc = case.q.shape[1]
+        Lk = case.c.shape[1]
+        while n == 0 or not over():
+            b = n % Bc
+            qt = oracle.absorb(case.q[0][b:b + 1], case.w_dec[0])
+            if fp8:
+                qtb = torch.from_numpy(qt).to(torch.bfloat16)
+                q8, sq, _ = oracle.quantize_query(qtb, case.w[0][b:b + 1].numpy())
+                sc = oracle.index_score(q8, oracle.E4M3, case.w[0][b:b + 1], case.c8[b], oracle.E4M3, q_scale=sq,
+                                        k_scale=case.cs[b], nthreads=nthreads)
+            else:
+                sc = oracle.latent_score(qt, oracle.F64, case.w[0][b:b + 1], case.c[b], nthreads=nthreads)
+            oracle.topk(sc, KTOP)
+            units += Lk
+            n += 1
+        t = time.perf_counter() - t0
+        return {"value": units / t, "unit": "keys/s", "cores": nthreads, "kind": "oracle",
+                "sample": f"{n} request-layer(s) of L={Lk} (absorb+score+top-{KTOP}), {t:.1f} s"}
+    if kind in ("hs_b1", "hs_b16"):
+        Bc = case.q.shape[1]
+        Lk = case.c.shape[1]
+        C = case.n_cand if getattr(case, "n_cand", 0) else 8192
+        F = case.q.shape[0] - 1
+        while n == 0 or not over():
+            b = n % Bc
+            qt0 = oracle.absorb(case.q[0][b:b + 1], case.w_dec[0])
+            sc = oracle.latent_score(qt0, oracle.F64, case.w[0][b:b + 1], case.c[b], nthreads=nthreads)
+            cand, _ = oracle.topk(sc, C)
+            qtf = np.stack([oracle.absorb(case.q[f][b:b + 1], case.w_dec[f]) for f in range(1, F + 1)])
+            oracle.hs_refine(qtf, oracle.F64, case.w[1:, b:b + 1], case.c[b:b + 1], cand, KTOP, nthreads=nthreads)
+            units += Lk
+            n += 1
+        t = time.perf_counter() - t0
+        return {"value": units / t, "unit": "keys/s (anchor scan)", "cores": nthreads, "kind": "oracle",
+                "sample": f"{n} request(s) of L={Lk}, C={C}, {F} followers (whole HS step), {t:.1f} s"}
+    if kind == "sparse_attention":
+        q, kv, sel, scale = case
+        Bc = q.shape[0]
+        while n == 0 or not over():
+            b = n % Bc
+            oracle.sparse_attention(q[b:b + 1], kv[b:b + 1], sel[b:b + 1], scale)
+            n += 1
+        t = time.perf_counter() - t0
+        return {"value": t / n * Bc * 1e6, "unit": "µs/call", "cores": 1, "kind": "oracle",
+                "sample": f"{n} request(s) of {Bc} ({q.shape[1]} heads, {sel.shape[1]} selections, numpy fp64), "
+                          f"{t:.1f} s; value extrapolated to the whole call"}
+    raise ValueError(kind)
 
 
 # ---------------------------------------------------------------------------
@@ -466,6 +546,7 @@ class PrefillBench:
         self.api = api
         self.T = self.L = 8192
         case = synth.dsa_prefill(T=self.T, L=self.L)
+        self.case = case  # host copy, for the oracle's timed sample
         self.q, self.w = case.q.to(dev), case.w.to(dev)
         self.k8, self.ks = case.k8.to(dev), case.ks.to(dev)
         self.sc = torch.empty((self.T, self.L), dtype=torch.float32, device=dev)
@@ -528,6 +609,7 @@ class LatentBench:
             self.dc, self.key_bytes = 192, 196
         while len(self.c) * per < 1.5 * L2_BYTES:
             self.c.append(tuple(t.clone() if t is not None else None for t in self.c[0]))
+        self.case = case  # host copy, for the oracle's timed sample
         self.q = [case.q[l].to(dev) for l in range(4)]
         self.wd = [case.w_dec[l].to(dev) for l in range(4)]
         self.hist = api.li_decode_select_workspace(B, dev).view(torch.int32)[:B * 2048]
@@ -592,6 +674,7 @@ class HsBench:
         per = case.c.numel() * 2
         while len(self.c) * per < 1.5 * L2_BYTES:
             self.c.append(self.c[0].clone())
+        self.case = case  # host copy, for the oracle's timed sample
         self.q = [case.q[l].to(dev) for l in range(4)]
         self.wd = [case.w_dec[l].to(dev) for l in range(4)]
         self.qf = case.q[1:].contiguous().to(dev)
@@ -638,7 +721,7 @@ class HsBench:
         return {"step": e0.elapsed_time(e1) / steps}
 
 
-def run_consumer(dev, args, clocks):
+def run_consumer(dev, args, clocks, want_cpu=False):
     """The consumer alone: li_sparse_attention at the decode shape (B = 8 requests, 128 query heads,
     the indexer's 2048 selections out of L = 32768 cached 576-element rows), rotating through 8
     selection sets so that the gathered rows (8 x 18.9 MB) exceed L2."""
@@ -677,7 +760,7 @@ def run_consumer(dev, args, clocks):
         if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else 1590.0
     byts = B * KTOP * D * 2 + B * Ha * D * 2 + B * Ha * 512 * 4
     flops = B * Ha * KTOP * (D + 512) * 2
-    return {"metric": "sparse attention over the selection, µs per call", "value": us, "unit": "µs/call",
+    res = {"metric": "sparse attention over the selection, µs per call", "value": us, "unit": "µs/call",
             "higher_is_better": False, "dtype": "bf16",
             "config": {"workload": "sparse_attention_b8_h128_k2048_l32k", "B": B, "heads": Ha, "k": KTOP, "L": L,
                        "row": "576 bf16 (512 latent + 64 RoPE); value = first 512",
@@ -687,6 +770,9 @@ def run_consumer(dev, args, clocks):
                          "frac": byts / us / 1e3 / hbm, "algorithmic_bytes": byts,
                          "tensor_tflops": flops / us / 1e6, "tensor_frac_of_bf16": flops / us / 1e6 / bf16_peak},
             "gpu_launches": 2 * 16 * reps, "clocks": clk}
+    if want_cpu:
+        res["cpu_baseline"] = oracle_sample("sparse_attention", (q.cpu(), kv.cpu(), sels[0].cpu().numpy(), scale))
+    return res
 
 
 def run_table4(dev, args, clocks):
@@ -906,7 +992,7 @@ def run_other(args, rank, world, local_rank):
     elif args.workload == "mli":
         out = run_schedules(dev, args, clocks)
     elif args.workload == "sparse_attention":
-        out = run_consumer(dev, args, clocks)
+        out = run_consumer(dev, args, clocks, want_cpu=rank == 0 and world == 1 and not args.no_cpu_baseline)
     elif args.workload == "table4":
         out = run_table4(dev, args, clocks)
     elif args.workload == "prefill":
@@ -958,6 +1044,12 @@ def run_other(args, rank, world, local_rank):
                             "peak": hbm, "peak_source": which, "unit": "GB/s",
                             "frac": algo / (r["step"] * 1e-3) / 1e9 / hbm}, "clocks": clk}
     assert api.li_get_last_error() == 0
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and "cpu_baseline" not in out:
+        # the oracle on the host cores, on a bounded sample of the same workload
+        if args.workload == "glm5_decode":
+            out["cpu_baseline"] = cpu_baseline_sample(heads=32)
+        elif args.workload in ("prefill", "latent", "latent192", "latent_glm5", "hs_b1", "hs_b16"):
+            out["cpu_baseline"] = oracle_sample(args.workload, bx.case)
     out.update({"n_gpus": world, "steps": args.steps, "warmup": args.warmup, "scaling": "weak", "vs_baseline": None,
                 "data": "synthetic"})
     if rank == 0:

@@ -70,3 +70,27 @@ def test_clock_sampler_parses_reasons():
     assert r["sm_max_mhz"] == 1965.0 and r["samples"] == 2
     assert r["sm_mhz"] == pytest.approx((1965 + 1800) / 2)
     assert r["reasons"] == ["sw_power_cap"]
+
+
+@pytest.mark.parametrize("kind", ["prefill", "latent", "latent192", "hs_b1", "sparse_attention"])
+def test_oracle_samples_run_on_small_cases(kind):
+    # each workload's cpu_baseline: the oracle timed on a bounded sample of that workload's input
+    import numpy as np
+    import torch
+    from sparse_attention_lightning_score_b200 import synth
+    if kind == "prefill":
+        case = synth.dsa_prefill(T=300, L=300)
+    elif kind == "latent":
+        case = synth.latent_group(B=2, L=3000, G=2)
+    elif kind == "latent192":
+        case = synth.latent_rope_nope(B=2, L=3000, G=2)
+    elif kind == "hs_b1":
+        case = synth.latent_hs(B=1, L=3000, n_cand=512, k_top=128)
+    else:
+        g = torch.Generator().manual_seed(0)
+        q = torch.randn(2, 64, 576, generator=g).to(torch.bfloat16)
+        kv = torch.randn(2, 700, 576, generator=g).to(torch.bfloat16)
+        sel = np.stack([np.sort(np.random.default_rng(b).choice(700, 256, replace=False)) for b in range(2)])
+        case = (q, kv, sel.astype(np.int32), 0.05)
+    r = bench.oracle_sample(kind, case, budget_s=0.2)
+    assert r["kind"] == "oracle" and r["value"] > 0 and r["cores"] >= 1 and r["sample"]
