@@ -775,6 +775,70 @@ def run_consumer(dev, args, clocks, want_cpu=False):
     return res
 
 
+def run_lshard(dev, args, clocks):
+    """L-sharding of one long context (B = 8 requests, L = 131072), emulated on one GPU: the per-rank
+    step (li_decode_select with values over the rank's L/P slice) and the merge of the P lists
+    (li_merge_shards), for P = 2, 4, 8, beside the unsharded step.  The all-gather between them
+    (8 B per listed position, P x B x k of them) is not timed: every call here has one GPU."""
+    import torch
+    from sparse_attention_lightning_score_b200 import api, synth
+    Lt = 131072
+    case = synth.dsa_decode(B=B, L=Lt, seed=1)
+    q, w = case.q.to(dev), case.w.to(dev)
+    k8, ks = case.k8.to(dev), case.ks.to(dev)
+
+    def timed(fns, reps):
+        g = capture(fns)
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) * 1e3 / (reps * len(fns))
+
+    reps = max(3, args.steps // 4)
+    clocks.start()
+    ws = api.li_decode_select_workspace(B, dev)
+    sc = torch.empty((B, Lt), dtype=torch.float32, device=dev)
+    idx = torch.empty((B, KTOP), dtype=torch.int32, device=dev)
+    vals = torch.empty((B, KTOP), dtype=torch.float32, device=dev)
+    full_us = timed([lambda: api.li_decode_select(q, w, k8, ks, KTOP, scores=sc, workspace=ws, with_values=True,
+                                                  idx=idx, vals=vals)] * 4, reps)
+    res = {}
+    for P in (2, 4, 8):
+        sl = Lt // P
+        # every rank's slice as its own cache; copies until the slices read per replay exceed L2
+        nset = max(1, math.ceil(1.5 * L2_BYTES / (B * Lt * (D + 4))))
+        slices = [(k8[:, p * sl:(p + 1) * sl].contiguous(), ks[:, p * sl:(p + 1) * sl].contiguous())
+                  for _ in range(nset) for p in range(P)]
+        scp = torch.empty((B, sl), dtype=torch.float32, device=dev)
+        lv = torch.empty((P, B, KTOP), dtype=torch.float32, device=dev)
+        li = torch.empty((P, B, KTOP), dtype=torch.int32, device=dev)
+        for p in range(P):
+            api.li_decode_select(q, w, slices[p][0], slices[p][1], KTOP, scores=scp, workspace=ws, with_values=True,
+                                 idx=li[p], vals=lv[p])
+        ri = torch.empty((B, KTOP), dtype=torch.int32, device=dev)
+        rank_us = timed([lambda s=s: api.li_decode_select(q, w, s[0], s[1], KTOP, scores=scp, workspace=ws,
+                                                          idx=ri) for s in slices], reps)
+        mws = torch.zeros(api._lib.load().li_merge_shards_workspace(P, B, KTOP), dtype=torch.uint8, device=dev)
+        oi = torch.empty((B, KTOP), dtype=torch.int32, device=dev)
+        merge_us = timed([lambda: api.li_merge_shards(lv, li, sl, KTOP, out_idx=oi, workspace=mws)] * 8, reps)
+        # the merged selection is the unsharded one
+        assert torch.equal(oi, idx), P
+        res[str(P)] = {"rank_step_us": round(rank_us, 2), "merge_us": round(merge_us, 2),
+                       "critical_path_us_without_allgather": round(rank_us + merge_us, 2),
+                       "allgather_bytes_per_rank": P * B * KTOP * 8}
+    clk = clocks.stop()
+    return {"metric": "decode step µs at L = 131072 split along L over P ranks (rank step + merge)",
+            "value": full_us, "unit": "µs/step (unsharded)", "higher_is_better": False, "dtype": "e4m3",
+            "config": {"workload": "lshard_b8_l128k", "B": B, "L": Lt, "k": KTOP,
+                       "ranks": "emulated on one GPU, one after another; the all-gather is not timed"},
+            "lshard": res, "gpu_launches": None, "clocks": clk}
+
+
 def run_table4(dev, args, clocks):
     """An in-house analogue of the LatentIndex paper's Table 4 (decode indexer latency by context length):
     one decode token (B = 1) through one 4-layer group, µs per group, at L = 8K..128K:
@@ -995,6 +1059,8 @@ def run_other(args, rank, world, local_rank):
         out = run_consumer(dev, args, clocks, want_cpu=rank == 0 and world == 1 and not args.no_cpu_baseline)
     elif args.workload == "table4":
         out = run_table4(dev, args, clocks)
+    elif args.workload == "lshard":
+        out = run_lshard(dev, args, clocks)
     elif args.workload == "prefill":
         bx = PrefillBench(dev)
         clocks.start()
@@ -1064,7 +1130,7 @@ def main():
     ap.add_argument("--impl", default="li", choices=["li", "reference"])
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="decode", choices=["decode", "glm5_decode", "prefill", "latent", "latent192", "latent_glm5", "hs_b1", "hs_b16", "mli",
+    ap.add_argument("--workload", default="decode", choices=["decode", "glm5_decode", "prefill", "latent", "latent192", "latent_glm5", "hs_b1", "hs_b16", "mli", "lshard",
                              "sparse_attention", "table4"],
                     help="decode (default) is the benchmarked configuration; the others time the other "
                          "configurations of the parity tests")

@@ -232,7 +232,11 @@ li_status li_copy_from_host(void* dst, const void* src_mapped, size_t bytes, li_
  *        outputs stacked in shard order (as an all-gather delivers them)
  *   out_idx [rows, k_out] int32 (global positions, ascending, -1 pads),
  *   out_vals [rows, k_out] fp32 (nullable)
- *   workspace  li_merge_shards_workspace(shards, rows, k) bytes, 256-byte aligned
+ *   workspace  li_merge_shards_workspace(shards, rows, k) bytes, 256-byte aligned.
+ *              Its last rows * 8 KB hold the candidates' first-digit histograms for
+ *              the row top-k: zero the workspace once after allocating it; each call
+ *              leaves them zero again.  If they were not zero, the result is the same,
+ *              only slower, and LI_ERR_BOUNDS is reported.
  * shards * k <= LI_TOPK_MAX_LEN and shards * shard_len < 2^31.  Each shard's
  * list must hold its valid positions first; a request whose lists leave a
  * valid candidate after a pad (only possible if a shard other than the last

@@ -256,7 +256,7 @@ def li_merge_shards(vals: torch.Tensor, idx: torch.Tensor, shard_len: int, k_out
     lib = _lib.load()
     need = lib.li_merge_shards_workspace(P, R, k)
     if workspace is None or workspace.numel() < need:
-        workspace = torch.empty(max(int(need), 256), dtype=torch.uint8, device=vals.device)
+        workspace = torch.zeros(max(int(need), 256), dtype=torch.uint8, device=vals.device)  # histograms start zero
     if out_idx is None:
         out_idx = torch.empty((R, k_out), dtype=torch.int32, device=vals.device)
     if with_values and out_vals is None:

@@ -115,9 +115,10 @@ struct TopkArgs {
 li_status launch_topk(const TopkArgs& a, cudaStream_t st);
 
 // ---------------------------------------------------------------- L-sharded selection merge
+// hist (optional): [rows, LI_HIST_BINS], zero on entry; receives the valid candidates' first digits
 li_status launch_merge_prep(const float* vals, const int32_t* idx, int shards, int rows, int k, long long shard_len,
-                            float* mvals, int32_t* mpos, int32_t* mlen, long long ld, const DevErr& err,
-                            cudaStream_t st);
+                            float* mvals, int32_t* mpos, int32_t* mlen, long long ld, uint32_t* hist,
+                            const DevErr& err, cudaStream_t st);
 
 // ---------------------------------------------------------------- absorption
 li_status launch_absorb(const void* q, const void* wdec, void* qt, int G, int B, int H, int d, int dc,

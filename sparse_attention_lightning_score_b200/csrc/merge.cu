@@ -11,8 +11,9 @@
 // candidate before every pad (a shard holds fewer than k valid candidates only
 // when it is the last one the request reaches).  This kernel lays the lists of
 // each request side by side, turns local positions into global ones and counts
-// the valid candidates; the row top-k then selects over them with the global
-// positions as its position map, so ties still go to the lower position.
+// the valid candidates (and their first radix digits); the row top-k then
+// selects over them from that histogram with the global positions as its
+// position map, so ties still go to the lower position.
 #include "li_common.cuh"
 #include "li_kernels.cuh"
 
@@ -20,11 +21,19 @@ namespace li {
 
 namespace {
 
-// grid: one CTA per request row; vals / idx are [shards, rows, k]
-__global__ void __launch_bounds__(256) merge_prep_kernel(const float* __restrict__ vals, const int32_t* __restrict__ idx,
-                                                         int shards, int rows, int k, long long shard_len,
-                                                         float* __restrict__ mvals, int32_t* __restrict__ mpos,
-                                                         int32_t* __restrict__ mlen, long long ld, DevErr err) {
+constexpr int MP_THREADS = 1024;
+constexpr int MP_PER = 4;  // candidates per thread per round
+
+// grid: one CTA per request row; vals / idx are [shards, rows, k].  With hist, every valid
+// candidate's score is also counted by its first radix digit into the row's histogram, one atomic
+// per distinct digit per warp, so that the row top-k starts from it.
+__global__ void __launch_bounds__(MP_THREADS) merge_prep_kernel(const float* __restrict__ vals,
+                                                                const int32_t* __restrict__ idx, int shards, int rows,
+                                                                int k, long long shard_len, float* __restrict__ mvals,
+                                                                int32_t* __restrict__ mpos, int32_t* __restrict__ mlen,
+                                                                long long ld, uint32_t* __restrict__ hist, DevErr err) {
+    pdl_trigger();
+    pdl_wait();  // the lists may come from the previous kernel of the stream
     const int r = blockIdx.x;
     const int n = shards * k;
     __shared__ int first_pad;  // lowest slot holding a pad
@@ -34,24 +43,46 @@ __global__ void __launch_bounds__(256) merge_prep_kernel(const float* __restrict
         last_valid = -1;
     }
     __syncthreads();
+    uint32_t* gh = hist ? hist + (size_t)r * LI_HIST_BINS : nullptr;
     int fp = n, lv = -1;
-    for (int j = threadIdx.x; j < n; j += blockDim.x) {
-        const int p = j / k, i = j - p * k;
-        const size_t src = ((size_t)p * rows + r) * k + i;
-        const int32_t x = __ldg(idx + src);
-        const bool valid = x >= 0 && (long long)x < shard_len;
-        mvals[(size_t)r * ld + j] = __ldg(vals + src);
-        mpos[(size_t)r * ld + j] = valid ? (int32_t)(x + (long long)p * shard_len) : -1;
-        if (valid) lv = max(lv, j);
-        else fp = min(fp, j);
-        if (x >= shard_len) record_error(err, ERRBIT_BOUNDS);
+    // the same number of rounds in every thread: the histogram's warp votes need whole warps
+    for (int base = 0; base < n; base += MP_THREADS * MP_PER) {
+        int32_t x[MP_PER];
+        float v[MP_PER];
+#pragma unroll
+        for (int u = 0; u < MP_PER; ++u) {  // loads first, all in flight
+            const int j = base + u * MP_THREADS + (int)threadIdx.x;
+            x[u] = -1;
+            v[u] = 0.f;
+            if (j < n) {
+                const int p = j / k, i = j - p * k;
+                const size_t src = ((size_t)p * rows + r) * k + i;
+                x[u] = __ldg(idx + src);
+                v[u] = __ldg(vals + src);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < MP_PER; ++u) {
+            const int j = base + u * MP_THREADS + (int)threadIdx.x;
+            const int p = j / k;
+            const bool valid = j < n && x[u] >= 0 && (long long)x[u] < shard_len;
+            if (j < n) {
+                mvals[(size_t)r * ld + j] = v[u];
+                mpos[(size_t)r * ld + j] = valid ? (int32_t)(x[u] + (long long)p * shard_len) : -1;
+                if (valid) lv = max(lv, j);
+                else fp = min(fp, j);
+                if (x[u] >= shard_len) record_error(err, ERRBIT_BOUNDS);
+            }
+            if (gh) warp_hist_add(gh, v[u], valid);
+        }
     }
     atomicMin(&first_pad, fp);
     atomicMax(&last_valid, lv);
     __syncthreads();
     if (threadIdx.x == 0) {
         // the valid candidates must form a prefix of the row (see above); otherwise report it and
-        // keep only the prefix
+        // keep only the prefix (the histogram then disagrees with the row and the top-k runs its
+        // plain passes)
         if (last_valid >= first_pad) record_error(err, ERRBIT_BOUNDS);
         mlen[r] = first_pad;
     }
@@ -60,10 +91,12 @@ __global__ void __launch_bounds__(256) merge_prep_kernel(const float* __restrict
 }  // namespace
 
 li_status launch_merge_prep(const float* vals, const int32_t* idx, int shards, int rows, int k, long long shard_len,
-                            float* mvals, int32_t* mpos, int32_t* mlen, long long ld, const DevErr& err,
-                            cudaStream_t st) {
+                            float* mvals, int32_t* mpos, int32_t* mlen, long long ld, uint32_t* hist,
+                            const DevErr& err, cudaStream_t st) {
     if (rows <= 0) return LI_OK;
-    merge_prep_kernel<<<rows, 256, 0, st>>>(vals, idx, shards, rows, k, shard_len, mvals, mpos, mlen, ld, err);
+    if (launch_pdl(merge_prep_kernel, dim3(rows), dim3(MP_THREADS), 0, st, 1, vals, idx, shards, rows, k, shard_len,
+                   mvals, mpos, mlen, ld, hist, err) != cudaSuccess)
+        return host_check_launch();
     return host_check_launch();
 }
 

@@ -59,3 +59,32 @@ def test_lshard_merge_reports_a_list_with_a_gap():
     assert api.li_get_last_error() == LI_ERR_BOUNDS
     assert _np(out).tolist() == [[0, 1, -1]]  # only the valid prefix is merged
     assert api.li_get_last_error() == LI_OK
+
+
+def test_lshard_merge_dirty_workspace_gives_the_same_selection():
+    # the merge counts the candidates' first digits into the workspace's histograms for the row
+    # top-k; histograms that are not zero give the same result through the plain passes, are
+    # reported, and are left zero
+    case = synth.dsa_decode(B=2, L=16000, seed=81)
+    q, w, k8, ks = case.q.to(DEV), case.w.to(DEV), case.k8.to(DEV), case.ks.to(DEV)
+    P, k, sl = 4, 1024, 4000
+    vals, idx = [], []
+    for p in range(P):
+        _, ip, vp = api.li_decode_select(q, w, k8[:, p * sl:(p + 1) * sl].contiguous(),
+                                         ks[:, p * sl:(p + 1) * sl].contiguous(), k, with_values=True)
+        vals.append(vp)
+        idx.append(ip)
+    vals, idx = torch.stack(vals), torch.stack(idx)
+    from sparse_attention_lightning_score_b200 import _lib
+    ws = torch.zeros(_lib.load().li_merge_shards_workspace(P, 2, k), dtype=torch.uint8, device=DEV)
+    tail = ws[ws.numel() - 2 * 2048 * 4:]
+    clean = api.li_merge_shards(vals, idx, sl, k, workspace=ws)
+    torch.cuda.synchronize()
+    assert api.li_get_last_error() == LI_OK and int(tail.count_nonzero()) == 0
+    tail.view(torch.int32)[::3] = 2
+    dirty = api.li_merge_shards(vals, idx, sl, k, workspace=ws)
+    torch.cuda.synchronize()
+    assert api.li_get_last_error() == LI_ERR_BOUNDS and int(tail.count_nonzero()) == 0
+    assert torch.equal(clean, dirty)
+    _, full = api.li_decode_select(q, w, k8, ks, k)
+    assert torch.equal(clean, full)
