@@ -351,7 +351,7 @@ li_status li_copy_from_host(void* dst, const void* src_mapped, size_t bytes, li_
 size_t li_merge_shards_workspace(int shards, int rows, int k) {
     if (shards <= 0 || rows <= 0 || k <= 0) return 0;
     const size_t ld = align_up((size_t)shards * k, 4);
-    return align_up((size_t)rows * ld * 4, 256) * 2 + align_up((size_t)rows * 4, 256) +
+    return align_up((size_t)rows * ld * 4, 256) * 2 + align_up((size_t)rows * shards * 4, 256) +
            (size_t)rows * LI_HIST_BINS * sizeof(uint32_t);
 }
 
@@ -371,14 +371,15 @@ li_status li_merge_shards(const float* vals, const int32_t* idx, int shards, int
     const size_t ld = align_up((size_t)shards * k, 4);
     float* mvals = static_cast<float*>(workspace);
     int32_t* mpos = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + align_up((size_t)rows * ld * 4, 256));
-    int32_t* mlen = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(mpos) + align_up((size_t)rows * ld * 4, 256));
+    int32_t* parts = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(mpos) + align_up((size_t)rows * ld * 4, 256));
     // the rows' first-digit histograms close the workspace (zero before the first call, left zero)
-    uint32_t* hist = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(mlen) + align_up((size_t)rows * 4, 256));
-    li_status s = launch_merge_prep(vals, idx, shards, rows, k, shard_len, mvals, mpos, mlen, (long long)ld, hist, e,
+    uint32_t* hist =
+        reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(parts) + align_up((size_t)rows * shards * 4, 256));
+    li_status s = launch_merge_prep(vals, idx, shards, rows, k, shard_len, mvals, mpos, parts, (long long)ld, hist, e,
                                     stream);
     if (s != LI_OK) return s;
-    TopkArgs t{mvals, (long long)ld, mlen, rows, shards * k, 0, 0, k_out, out_idx, out_vals, mpos, (long long)ld, rows,
-               hist, 0, 1, e};
+    TopkArgs t{mvals, (long long)ld, nullptr, rows, shards * k, 0, 0, k_out, out_idx, out_vals, mpos, (long long)ld,
+               rows, hist, 0, 1, e, parts, shards, k};
     return launch_topk(t, stream);
 }
 

@@ -111,13 +111,20 @@ struct TopkArgs {
     int cand_cap;           // set by the launcher: candidate keys one CTA can hold
     int tokens;             // query rows per request, as for the scorer (0 or 1: one row per len entry)
     DevErr err;
+    // optional (shard merge): row r's length from nparts lists of part_k slots each,
+    // len_parts[r * nparts + p] = valid slots at the head of list p | 0x80000000 if list p has a
+    // valid slot after a pad.  The row is the valid prefix of the lists side by side; a valid slot
+    // after it is reported as a bounds error and left out.
+    const int32_t* len_parts;
+    int nparts, part_k;
 };
 li_status launch_topk(const TopkArgs& a, cudaStream_t st);
 
 // ---------------------------------------------------------------- L-sharded selection merge
-// hist (optional): [rows, LI_HIST_BINS], zero on entry; receives the valid candidates' first digits
+// parts: [rows, shards] valid-prefix counts per list (the top-k's len_parts); hist (optional):
+// [rows, LI_HIST_BINS], zero on entry, receives the valid candidates' first digits
 li_status launch_merge_prep(const float* vals, const int32_t* idx, int shards, int rows, int k, long long shard_len,
-                            float* mvals, int32_t* mpos, int32_t* mlen, long long ld, uint32_t* hist,
+                            float* mvals, int32_t* mpos, int32_t* parts, long long ld, uint32_t* hist,
                             const DevErr& err, cudaStream_t st);
 
 // ---------------------------------------------------------------- absorption

@@ -198,6 +198,25 @@ __global__ void __launch_bounds__(NT) topk_kernel(const TopkArgs a, int row0, in
     if (!a.causal && a.len && (nl < 0 || nl > a.max_len) && c == 0 && threadIdx.x == 0) record_error(a.err, ERRBIT_BOUNDS);
     nl = nl < 0 ? 0 : (nl > a.max_len ? a.max_len : nl);
     if (!a.causal) nl = nl - (tokens - 1 - r % tokens) < 0 ? 0 : nl - (tokens - 1 - r % tokens);
+    if (a.len_parts) {
+        // shard merge: the valid prefix of the lists side by side
+        const int32_t* pr = a.len_parts + (size_t)r * a.nparts;
+        const long long full = (long long)a.nparts * a.part_k;
+        long long fpad = full;
+        bool gap = false;
+        for (int p = 0; p < a.nparts; ++p) {
+            const uint32_t v = (uint32_t)__ldg(pr + p);
+            const int cnt = (int)(v & 0x7fffffffu);
+            gap |= (v >> 31) != 0u;
+            if (fpad == full) {
+                if (cnt < a.part_k) fpad = (long long)p * a.part_k + cnt;
+            } else if (cnt > 0) {
+                gap = true;
+            }
+        }
+        if (gap && c == 0 && threadIdx.x == 0) record_error(a.err, ERRBIT_BOUNDS);
+        nl = fpad < nl ? fpad : nl;
+    }
     const int n = (int)nl;
     const int k = a.k;
     const int base = c * chunk;
