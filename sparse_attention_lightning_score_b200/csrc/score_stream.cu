@@ -235,22 +235,20 @@ __global__ void __launch_bounds__(StreamCfg<NH, FP8, KBLK, STAGES, NACC, HIST>::
         } else {
             constexpr int CH = KBLK * 8;                // 16-byte chunks per query row
             constexpr int PER = C::H * CH / 128;        // chunks per thread
-            static_assert(PER % 8 == 0, "query copy batches");
-            const uint4* src =
-                reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.q) + (size_t)b * C::H * KBLK * 64);
-#pragma unroll
-            for (int g0 = 0; g0 < PER; g0 += 8) {
-                uint4 v[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) v[u] = __ldg(src + et + 128 * (g0 + u));
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int ci = et + 128 * (g0 + u);
-                    const int r = ci / CH, cc = ci % CH;
-                    *reinterpret_cast<uint4*>(qsm + (cc >> 3) * (C::H * 128) + sw128_offset(r, cc & 7)) = v[u];
-                }
+            // every 16-byte chunk straight to its swizzled place by cp.async, all in flight at once
+            const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(a.q) + (size_t)b * C::H * KBLK * 64;
+#pragma unroll 4
+            for (int g = 0; g < PER; ++g) {
+                const int ci = et + 128 * g;
+                const int r = ci / CH, cc = ci % CH;
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                                 smem_u32(qsm + (cc >> 3) * (C::H * 128) + sw128_offset(r, cc & 7))),
+                             "l"(src + (size_t)ci * 8)
+                             : "memory");
             }
+            asm volatile("cp.async.commit_group;" ::: "memory");
             if (et < C::H) wsm[et] = __ldg(a.w + (size_t)b * C::H + et);
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
         }
         if constexpr (HIST) {
             for (int i = et; i < LI_HIST_BINS; i += 32 * C::PRO_WARPS) hs[i] = 0u;
