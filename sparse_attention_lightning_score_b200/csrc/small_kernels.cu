@@ -161,12 +161,15 @@ __global__ void __launch_bounds__(256) absorb_kernel(const __nv_bfloat16* __rest
     W += (size_t)blockIdx.z * H * d * dc;
     qt += (size_t)blockIdx.z * B * H * dc;
     const int t = threadIdx.x;
-    // W slice: d rows x 128 bytes, eight 16-byte units per row
+    // W slice: d rows x 128 bytes, eight 16-byte units per row, by cp.async with every unit in
+    // flight at once (a load-then-store loop waited out one round trip per unit)
     for (int u = t; u < d * 8; u += 256) {
         const int e = u >> 3, v = u & 7;
-        *reinterpret_cast<uint4*>(wsh + e * AB_COLS + 8 * v) =
-            __ldg(reinterpret_cast<const uint4*>(W + ((size_t)j * d + e) * dc + c0) + v);
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(wsh + e * AB_COLS + 8 * v)),
+                     "l"(W + ((size_t)j * d + e) * dc + c0 + 8 * v)
+                     : "memory");
     }
+    asm volatile("cp.async.commit_group;" ::: "memory");
     const int c = t & (AB_COLS - 1);
     for (int b0 = 0; b0 < B; b0 += AB_BMAX) {
         const int nb = min(AB_BMAX, B - b0);
@@ -174,6 +177,7 @@ __global__ void __launch_bounds__(256) absorb_kernel(const __nv_bfloat16* __rest
             const int bb = i / d, e = i - bb * d;
             qsh[bb * (d + 1) + e] = __bfloat162float(q[((size_t)(b0 + bb) * H + j) * d + e]);
         }
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
         __syncthreads();
         for (int bb = t >> 6; bb < nb; bb += 4) {
             const float* qr = qsh + bb * (d + 1);
