@@ -40,7 +40,7 @@ struct HsCfg {
     static constexpr int OFF_Q = HS_STAGES * HS_STAGE_BYTES;
     static constexpr int OFF_W = OFF_Q + Q_BYTES;
     static constexpr int OFF_BAR = OFF_W + N * 4;
-    static constexpr int NBAR = 2 * HS_STAGES + 2 + 2 + 1;
+    static constexpr int NBAR = 2 * HS_STAGES + 2 + 2 + 2;  // full, empty, accf, acce, qready, qtma
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_TMEM + 16 + 1024;
     static constexpr int TMEM_COLS = (2 * N <= 128) ? 128 : ((2 * N <= 256) ? 256 : 512);
@@ -58,7 +58,8 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 template <int F, int H>
-__global__ void __launch_bounds__(HS_THREADS, 1) hs_rescore_kernel(const HsArgs a, int tiles_per_cta) {
+__global__ void __launch_bounds__(HS_THREADS, 1) hs_rescore_kernel(const __grid_constant__ CUtensorMap qmap,
+                                                                    const HsArgs a, int tiles_per_cta) {
     using C = HsCfg<F, H>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
@@ -75,6 +76,7 @@ __global__ void __launch_bounds__(HS_THREADS, 1) hs_rescore_kernel(const HsArgs 
     uint64_t* accf = empty + HS_STAGES;
     uint64_t* acce = accf + 2;
     uint64_t* qready = acce + 2;
+    uint64_t* qtma = qready + 1;  // the followers' query blocks, by TMA
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
     float* wsm = reinterpret_cast<float*>(smem + C::OFF_W);
     uint8_t* qsm = smem + C::OFF_Q;
@@ -89,6 +91,7 @@ __global__ void __launch_bounds__(HS_THREADS, 1) hs_rescore_kernel(const HsArgs 
             mbar_init(&acce[i], 128);
         }
         mbar_init(qready, 128);
+        mbar_init(qtma, 1);
         fence_mbar_init();
     }
     if (warp == 4) {
@@ -151,7 +154,7 @@ __global__ void __launch_bounds__(HS_THREADS, 1) hs_rescore_kernel(const HsArgs 
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t IDESC = idesc_f32acc(HS_M, C::N, kFmtBF16);
-            bool ok = mbar_wait(qready, 0, a.err);
+            bool ok = mbar_wait(qtma, 0, a.err);
             tc_fence_after();
             const uint32_t qaddr = smem_u32(qsm);
             int stage = 0;
@@ -182,24 +185,22 @@ __global__ void __launch_bounds__(HS_THREADS, 1) hs_rescore_kernel(const HsArgs 
         const int et = threadIdx.x - 160;  // 0..127
         constexpr int CH = HS_KBLK * 8;    // 16-byte chunks per query row
         constexpr int PER = C::N * CH / 128;  // 16 chunks per thread per follower
-        // every chunk goes straight to its swizzled place in shared memory (16-byte cp.async), all
-        // of them in flight at once; staged through registers in batches, the 96 KB of three
-        // followers' queries took about 5 us at one request
-#pragma unroll 4
-        for (int g = 0; g < PER; ++g) {
-            const int ci = et + 128 * g;
-            const int r = ci / CH, cc = ci % CH;  // r = f * H + j
-            const int f = r / H, j = r % H;
-            cp_async16(smem_u32(qsm + (cc >> 3) * (C::N * 128) + sw128_offset(r, cc & 7)),
-                       reinterpret_cast<const __nv_bfloat16*>(a.qt) + (((size_t)f * a.B + b) * H + j) * HS_DC + cc * 8,
-                       16u);
+        // the F query blocks come by TMA, one 64-element K block of H rows per load, straight into
+        // the 128-byte-swizzled K-major layout the MMA reads (register-staged, then per-thread
+        // cp.async copies of the same 96 KB took 4.9, then 3.8 us of a CTA's time at one request)
+        if (et == 0) {
+            mbar_arrive_expect_tx(qtma, (uint32_t)(F * HS_KBLK * H * 128));
+#pragma unroll
+            for (int f = 0; f < F; ++f)
+#pragma unroll
+                for (int kb = 0; kb < HS_KBLK; ++kb)
+                    tma_load_2d(qsm + kb * (C::N * 128) + f * H * 128, &qmap, kb * 64, (f * a.B + b) * H, qtma,
+                                l2_policy_evict_last());
         }
-        cp_async_commit();
         for (int r = et; r < C::N; r += 128) {
             const int f = r / H, j = r % H;
             wsm[r] = __ldg(a.w + ((size_t)f * a.B + b) * H + j);
         }
-        cp_async_wait<0>();
         fence_proxy_async_smem();
         mbar_arrive(qready);
         asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -240,6 +241,9 @@ __global__ void __launch_bounds__(HS_THREADS, 1) hs_rescore_kernel(const HsArgs 
             }
         }
     }
+    // the query blocks' TMA must have landed before the CTA may leave (the MMA issuer waited for
+    // them unless it gave up)
+    if (threadIdx.x == 160) (void)mbar_wait(qtma, 0, a.err);
     __syncwarp();
     __syncthreads();
     if (warp == 4) {
@@ -249,7 +253,7 @@ __global__ void __launch_bounds__(HS_THREADS, 1) hs_rescore_kernel(const HsArgs 
 }
 
 template <int F, int H>
-li_status launch_f(const HsArgs& a, cudaStream_t st) {
+li_status launch_f(const CUtensorMap& qmap, const HsArgs& a, cudaStream_t st) {
     using C = HsCfg<F, H>;
     static bool attr_done[64] = {};
     int dev = 0;
@@ -265,29 +269,29 @@ li_status launch_f(const HsArgs& a, cudaStream_t st) {
     int cpr = max(1, sms / max(1, a.B));
     int tpc = max(1, (ntiles + cpr - 1) / cpr);
     cpr = (ntiles + tpc - 1) / tpc;
-    hs_rescore_kernel<F, H><<<dim3(cpr, a.B), HS_THREADS, C::SMEM, st>>>(a, tpc);
+    hs_rescore_kernel<F, H><<<dim3(cpr, a.B), HS_THREADS, C::SMEM, st>>>(qmap, a, tpc);
     return host_check_launch();
 }
 
 }  // namespace
 
-li_status launch_hs_rescore(const HsArgs& a, cudaStream_t st) {
+li_status launch_hs_rescore(const CUtensorMap& qmap, const HsArgs& a, cudaStream_t st) {
     if (a.B <= 0 || a.C <= 0) return LI_OK;
     if (a.H == 64) {
         switch (a.F) {
-        case 1: return launch_f<1, 64>(a, st);
-        case 2: return launch_f<2, 64>(a, st);
-        case 3: return launch_f<3, 64>(a, st);
-        case 4: return launch_f<4, 64>(a, st);
+        case 1: return launch_f<1, 64>(qmap, a, st);
+        case 2: return launch_f<2, 64>(qmap, a, st);
+        case 3: return launch_f<3, 64>(qmap, a, st);
+        case 4: return launch_f<4, 64>(qmap, a, st);
         default: return LI_ERR_UNSUPPORTED;
         }
     }
     if (a.H == 32) {
         switch (a.F) {
-        case 1: return launch_f<1, 32>(a, st);
-        case 2: return launch_f<2, 32>(a, st);
-        case 3: return launch_f<3, 32>(a, st);
-        case 4: return launch_f<4, 32>(a, st);
+        case 1: return launch_f<1, 32>(qmap, a, st);
+        case 2: return launch_f<2, 32>(qmap, a, st);
+        case 3: return launch_f<3, 32>(qmap, a, st);
+        case 4: return launch_f<4, 32>(qmap, a, st);
         default: return LI_ERR_UNSUPPORTED;
         }
     }

@@ -512,7 +512,12 @@ li_status li_hs_refine(const void* c_bf16, int64_t cache_batch_rows, int64_t cac
     float* sc = static_cast<float*>(workspace);
     uint32_t* hist = hs_hist_of(workspace, workspace_bytes, batch, followers);
     HsArgs h{c_bf16, cache_batch_rows, cache_rows, cand, batch, n_cand, followers, heads, q_tilde_bf16, w, sc, hist, e};
-    li_status s = launch_hs_rescore(h, stream);
+    if ((uint64_t)followers * batch * heads >= (1ull << 31)) return LI_ERR_UNSUPPORTED;
+    CUtensorMap qmap;
+    if (!encode_map_2d(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q_tilde_bf16, 256, (uint64_t)followers * batch * heads,
+                       512, 64, (uint32_t)heads))
+        return LI_ERR_CUDA;
+    li_status s = launch_hs_rescore(qmap, h, stream);
     if (s != LI_OK) return s;
     TopkArgs t{sc, ldw, nullptr, followers * batch, n_cand, 0, 0, k, out_idx, nullptr, cand, n_cand, batch,
                hist, 0, 1, e};

@@ -145,7 +145,8 @@ struct HsArgs {
     uint32_t* hist;         // optional [F*B, LI_HIST_BINS]: out's first-digit counts are added here
     DevErr err;
 };
-li_status launch_hs_rescore(const HsArgs& a, cudaStream_t st);
+// qmap: q~ as [F * B * H, 256] bf16, box 64 x H, 128-byte swizzle
+li_status launch_hs_rescore(const CUtensorMap& qmap, const HsArgs& a, cudaStream_t st);
 
 // HS over DeepSeek-V3.2's FP8 latent: e4m3 rows of 192 with one fp32 scale per row, 64 heads per follower
 struct Hs8Args {
