@@ -13,8 +13,11 @@
 // scored -inf so the following top-k never prefers them; candidates outside
 // the cache are reported (LI_ERR_BOUNDS) and zero-filled, never read.
 //
+// The followers' query blocks (F x 4 K blocks of H rows) come by TMA from a
+// tensor map over q~, straight into the same layout.
+//
 // Warps: 0..3 gather producers, 4 TMEM allocator + MMA issuer, 5..8 follower
-// query preparation and epilogue.  Output: scores [F*B, round4(C)] fp32, and
+// weights (one thread issues the query TMA) and epilogue.  Output: scores [F*B, round4(C)] fp32, and
 // (optionally) each row's first-digit histogram for the follower top-k, counted
 // by the epilogue warps with one global atomic per distinct digit per warp.
 #include "li_common.cuh"
