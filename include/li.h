@@ -132,6 +132,21 @@ li_status li_index_score(const void* q, const float* w, const void* k, const flo
 /* Bytes of device workspace li_index_score needs for this descriptor. */
 size_t li_index_score_workspace(const li_score_desc* desc);
 
+/* Workspace sizes by operation, in the one-call form (op, rows, max_len, k).
+ * Each call's own *_workspace function gives the exact size for its full
+ * argument set; this one returns a size that is enough for every call of the
+ * operation with these sizes (a workspace larger than needed is accepted):
+ *   LI_OP_SCORE          li_index_score over `rows` query rows of 64 heads x 128
+ *                        (the causal prefill form; the decode forms need none)
+ *   LI_OP_TOPK           li_topk: 0 (it takes no workspace)
+ *   LI_OP_HS             li_hs_refine / li_hs_refine_fp8 with batch = rows,
+ *                        n_cand = max_len and any follower count up to 4
+ *   LI_OP_DECODE_SELECT  li_decode_select over `rows` rows (zero it once)
+ * k is accepted for the form's sake and changes no size.  An unknown op or a
+ * negative size returns 0. */
+typedef enum { LI_OP_SCORE = 0, LI_OP_TOPK = 1, LI_OP_HS = 2, LI_OP_DECODE_SELECT = 3 } li_op;
+size_t li_workspace_size(int op, int rows, int max_len, int k);
+
 /* ------------------------------------------------------------------------ */
 /* Top-k selection                                                           */
 /* ------------------------------------------------------------------------ */
@@ -340,29 +355,6 @@ li_status li_hs_refine(const void* c_bf16, int64_t cache_batch_rows, int64_t cac
 
 size_t li_hs_refine_workspace(int batch, int n_cand, int followers);
 
-/* Capacity, in floats (4 MiB), of the fixed scratch behind li_hs_refine_noalloc. */
-#define LI_HS_NOALLOC_MAX_SCRATCH_FLOATS 1048576
-
-/* li_hs_refine without a workspace argument, for callers that cannot
- * allocate device memory: for example code inside an engine that owns and
- * budgets all device memory and forbids allocation while serving, or a
- * plugin that receives only its inputs and outputs.  The pages have no
- * counterpart to this call; it exists only for such callers.
- *
- * Same arguments, results and errors as li_hs_refine.  The followers'
- * candidate scores go to a file-scope device array of
- * LI_HS_NOALLOC_MAX_SCRATCH_FLOATS floats that every GPU loading the library
- * holds until the process exits; the call allocates nothing.
- *   - followers * batch * round_up(n_cand, 4) above that capacity returns
- *     LI_ERR_INVALID_ARG before anything is launched.
- *   - The array is shared by all calls on a device and keeps the last call's
- *     contents; its histogram part (the last followers * batch * 8 KB) starts
- *     zero at load and each call leaves it zero, and a call whose histograms
- *     overlap an earlier, larger call's scores still gives the same result.
- *     Calls that overlap on the GPU (unordered streams) race on it: serialise
- *     them.
- *   - The first call on a device looks up the array's device address; make
- *     that first call before any stream capture begins. */
 /* li_hs_refine over DeepSeek-V3.2's FP8 latent (LatentIndex appendix, Table 5:
  * 64 RoPE + 128 NoPE dimensions), the cache li_latent_score_fp8 scans: e4m3 rows
  * of 192 bytes with one fp32 scale per row.  Each follower's absorbed query is
@@ -378,9 +370,38 @@ li_status li_hs_refine_fp8(const void* c_e4m3, const float* c_scale, int64_t cac
                            int followers, int heads, int latent_dim, int k, int32_t* out_idx, void* workspace,
                            size_t workspace_bytes, li_stream_t stream);
 
+/* Capacity, in floats (4 MiB), of the fixed scratch behind li_hs_refine_noalloc. */
+#define LI_HS_NOALLOC_MAX_SCRATCH_FLOATS 1048576
+
+/* li_hs_refine without a workspace argument, for callers that cannot
+ * allocate device memory: for example code inside an engine that owns and
+ * budgets all device memory and forbids allocation while serving, or a
+ * plugin that receives only its inputs and outputs.  The pages have no
+ * counterpart to this call; it exists only for such callers.
+ *
+ * Same arguments, results and errors as li_hs_refine.  The workspace
+ * li_hs_refine would take -- the followers' candidate scores and the follower
+ * top-k's histograms -- is a file-scope device array of
+ * LI_HS_NOALLOC_MAX_SCRATCH_FLOATS floats that every GPU loading the library
+ * holds until the process exits; the call allocates nothing.
+ *   - Limit: li_hs_refine_workspace(batch, n_cand, followers) must not exceed
+ *     4 * LI_HS_NOALLOC_MAX_SCRATCH_FLOATS bytes (4 MiB); a larger call returns
+ *     LI_ERR_INVALID_ARG before anything is launched.  For example one
+ *     follower and 4 requests take at most 260,096 candidates, three followers
+ *     and 16 requests at most 19,796.
+ *   - The array is shared by all calls on a device and keeps the last call's
+ *     contents.  Each call clears its own histograms (the array's last
+ *     followers * batch * 8 KB) with one cudaMemsetAsync on `stream` before its
+ *     kernels, so what an earlier call of other sizes left there changes
+ *     neither the result nor the status.  Calls that overlap on the GPU
+ *     (unordered streams) race on the array: serialise them.
+ *   - The first call on a device looks up the array's device address and
+ *     caches it for the process; make that first call before any stream
+ *     capture begins.  After cudaDeviceReset the cached address is stale. */
 li_status li_hs_refine_noalloc(const void* c_bf16, int64_t cache_batch_rows, int64_t cache_rows, const int32_t* cand,
                                int batch, int n_cand, const void* q_tilde_bf16, const float* w, int followers,
                                int heads, int latent_dim, int k, int32_t* out_idx, li_stream_t stream);
+
 
 /* ------------------------------------------------------------------------ */
 /* The consumer: sparse attention over a selection                           */

@@ -11,18 +11,25 @@
 // Limits and sharing:
 //   - The array holds LI_HS_NOALLOC_MAX_SCRATCH_FLOATS floats (4 MiB).  Every
 //     GPU that loads the library reserves it until the process exits.
-//   - Calls with followers * batch * round_up(n_cand, 4) floats beyond that
-//     are rejected with LI_ERR_INVALID_ARG before anything is launched.
+//   - A call is accepted when li_hs_refine_workspace(batch, n_cand, followers)
+//     -- the candidate scores plus the follower top-k's histograms -- fits in
+//     those 4 MiB; a larger one returns LI_ERR_INVALID_ARG before anything is
+//     launched.
 //   - All calls on a device share the one array and it keeps the previous
 //     call's contents.  Every score slot the selection reads is written first
-//     by the same call.  The follower top-k's histograms sit at the array's
-//     end: zero at load, left zero by every call, and only a speed-up (a
-//     histogram that disagrees with the keys sends the top-k to its plain
-//     passes).  Calls that overlap on the GPU (different streams, no ordering
-//     between them) race on the array and must be serialised by the caller.
+//     by the same call.  The histograms sit at the array's end, where an
+//     earlier call with other sizes may have left scores, so every call
+//     clears its own histograms on its stream (cudaMemsetAsync, no
+//     allocation) before its kernels run.  Calls that overlap on the GPU
+//     (different streams, no ordering between them) race on the array and
+//     must be serialised by the caller.
 //   - The first call on a device looks up the array's device address (set-up);
-//     make that first call before any stream capture begins.
+//     make that first call before any stream capture begins.  The address is
+//     cached per device for the life of the process: after cudaDeviceReset
+//     the array is a new allocation and this cache no longer names it.
 #include <cuda_runtime.h>
+
+#include <atomic>
 
 #include "li.h"
 
@@ -33,10 +40,14 @@ static __device__ __align__(256) float g_hs_noalloc_scratch[LI_HS_NOALLOC_MAX_SC
 
 constexpr int kMaxDevices = 64;
 
+// one follower row's first-digit histogram in li_hs_refine's workspace: 2048 bins of uint32
+constexpr size_t kHistBytesPerRow = 8192;
+
 // Host code cannot use g_hs_noalloc_scratch's name as a device address (on the
 // host it names a stand-in object); the address is fetched per device, with
-// that device current, and cached.
-float* g_scratch_addr[kMaxDevices] = {};
+// that device current, and cached (atomically: several host threads may make
+// their first call at once; each then stores the same address).
+std::atomic<float*> g_scratch_addr[kMaxDevices];
 
 li_status scratch_for_current_device(float** out) {
     int dev = 0;
@@ -45,16 +56,18 @@ li_status scratch_for_current_device(float** out) {
         return LI_ERR_CUDA;
     }
     if (dev < 0 || dev >= kMaxDevices) return LI_ERR_UNSUPPORTED;
-    if (!g_scratch_addr[dev]) {
+    float* a = g_scratch_addr[dev].load(std::memory_order_acquire);
+    if (!a) {
         void* p = nullptr;
         const cudaError_t e = cudaGetSymbolAddress(&p, g_hs_noalloc_scratch);
         if (e != cudaSuccess || !p) {
             cudaGetLastError();
             return LI_ERR_CUDA;
         }
-        g_scratch_addr[dev] = static_cast<float*>(p);
+        a = static_cast<float*>(p);
+        g_scratch_addr[dev].store(a, std::memory_order_release);
     }
-    *out = g_scratch_addr[dev];
+    *out = a;
     return LI_OK;
 }
 
@@ -70,6 +83,17 @@ extern "C" li_status li_hs_refine_noalloc(const void* c_bf16, int64_t cache_batc
     float* scratch = nullptr;
     const li_status s = scratch_for_current_device(&scratch);
     if (s != LI_OK) return s;
+    // this call's histograms are the last followers * batch * 8 KB of the workspace it is given (the
+    // layout li_hs_refine documents); an earlier call with other sizes may have left scores there
+    const size_t hist_bytes = (size_t)followers * batch * kHistBytesPerRow;
+    if (hist_bytes == 0 || n_cand == 0)
+        return li_hs_refine(c_bf16, cache_batch_rows, cache_rows, cand, batch, n_cand, q_tilde_bf16, w, followers,
+                            heads, latent_dim, k, out_idx, scratch, sizeof(g_hs_noalloc_scratch), stream);
+    uint8_t* hist = reinterpret_cast<uint8_t*>(scratch) + (sizeof(g_hs_noalloc_scratch) - hist_bytes);
+    if (cudaMemsetAsync(hist, 0, hist_bytes, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return LI_ERR_CUDA;
+    }
     return li_hs_refine(c_bf16, cache_batch_rows, cache_rows, cand, batch, n_cand, q_tilde_bf16, w, followers, heads,
                         latent_dim, k, out_idx, scratch, sizeof(g_hs_noalloc_scratch), stream);
 }
