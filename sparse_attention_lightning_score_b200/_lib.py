@@ -15,6 +15,7 @@ LI_OK, LI_ERR_INVALID_ARG, LI_ERR_UNSUPPORTED, LI_ERR_CUDA, LI_ERR_TIMEOUT, LI_E
 LI_DTYPE_F32, LI_DTYPE_BF16, LI_DTYPE_E4M3 = 0, 1, 2
 LI_TOPK_MAX_LEN = 262144
 LI_HS_NOALLOC_MAX_SCRATCH_FLOATS = 1048576
+LI_OP_SCORE, LI_OP_TOPK, LI_OP_HS, LI_OP_DECODE_SELECT = range(4)
 
 vp = ctypes.c_void_p
 i32 = ctypes.c_int
@@ -34,6 +35,7 @@ SIGNATURES = {
     "li_quantize_query": (i32, [vp, vp, i32, i32, i32, vp, vp, vp, vp]),
     "li_index_score": (i32, [vp, vp, vp, vp, i64, vp, vp, i64, ctypes.POINTER(ScoreDesc), vp, sz, vp]),
     "li_index_score_workspace": (sz, [ctypes.POINTER(ScoreDesc)]),
+    "li_workspace_size": (sz, [i32, i32, i32, i32]),
     "li_topk": (i32, [vp, i64, vp, i32, i32, i32, i32, i32, vp, vp, vp]),
     "li_decode_select": (i32, [vp, vp, vp, vp, i64, vp, vp, i64, ctypes.POINTER(ScoreDesc), i32, vp, vp, vp, sz,
                                vp]),

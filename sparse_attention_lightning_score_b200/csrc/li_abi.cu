@@ -487,6 +487,32 @@ size_t li_hs_refine_workspace(int batch, int n_cand, int followers) {
            hs_hist_bytes(batch, followers);
 }
 
+size_t li_workspace_size(int op, int rows, int max_len, int k) {
+    (void)k;
+    if (rows < 0 || max_len < 0) return 0;
+    switch (op) {
+    case LI_OP_SCORE: {
+        li_score_desc d{};
+        d.rows = rows;
+        d.heads = 64;
+        d.dim = 128;
+        d.max_len = max_len;
+        d.causal = 1;
+        d.q_dtype = LI_DTYPE_BF16;
+        d.k_dtype = LI_DTYPE_E4M3;
+        return li_index_score_workspace(&d);
+    }
+    case LI_OP_TOPK: return 0;
+    case LI_OP_HS: return li_hs_refine_workspace(rows, max_len, 4);
+    case LI_OP_DECODE_SELECT: {
+        li_score_desc d{};
+        d.rows = rows;
+        return li_decode_select_workspace(&d);
+    }
+    }
+    return 0;
+}
+
 li_status li_hs_refine(const void* c_bf16, int64_t cache_batch_rows, int64_t cache_rows, const int32_t* cand,
                        int batch, int n_cand, const void* q_tilde_bf16, const float* w, int followers, int heads,
                        int latent_dim, int k, int32_t* out_idx, void* workspace, size_t workspace_bytes,

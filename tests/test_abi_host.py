@@ -32,6 +32,24 @@ def test_library_exports_every_declared_symbol():
         assert name in _lib.SIGNATURES, name
 
 
+def test_workspace_size_by_operation_matches_each_calls_own_size():
+    """The one-call workspace form (op, rows, max_len, k) against the per-call sizes."""
+    lib = _lib.load()
+    for rows in [1, 8, 8192]:
+        d = _lib.ScoreDesc(rows, 64, 128, 8192, 1, 0, _lib.LI_DTYPE_BF16, _lib.LI_DTYPE_E4M3)
+        assert lib.li_workspace_size(_lib.LI_OP_SCORE, rows, 8192, 2048) == lib.li_index_score_workspace(ctypes.byref(d))
+        d.causal = 0
+        assert lib.li_workspace_size(_lib.LI_OP_DECODE_SELECT, rows, 32768, 2048) == \
+            lib.li_decode_select_workspace(ctypes.byref(d))
+        assert lib.li_workspace_size(_lib.LI_OP_TOPK, rows, 32768, 2048) == 0
+    for B, C in [(1, 8192), (16, 8192), (3, 100)]:
+        need = lib.li_workspace_size(_lib.LI_OP_HS, B, C, 2048)
+        assert need == lib.li_hs_refine_workspace(B, C, 4)
+        assert all(need >= lib.li_hs_refine_workspace(B, C, F) for F in (1, 2, 3))
+    assert lib.li_workspace_size(99, 8, 100, 16) == 0
+    assert lib.li_workspace_size(_lib.LI_OP_HS, -1, 100, 16) == 0
+
+
 def test_status_strings():
     assert _lib.status_string(_lib.LI_OK) == "LI_OK"
     assert _lib.status_string(_lib.LI_ERR_TIMEOUT) == "LI_ERR_TIMEOUT"
