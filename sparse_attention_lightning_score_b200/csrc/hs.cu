@@ -43,7 +43,7 @@ struct HsCfg {
     static constexpr int OFF_Q = HS_STAGES * HS_STAGE_BYTES;
     static constexpr int OFF_W = OFF_Q + Q_BYTES;
     static constexpr int OFF_BAR = OFF_W + N * 4;
-    static constexpr int NBAR = 2 * HS_STAGES + 2 + 2 + 2;  // full, empty, accf, acce, qready, qtma
+    static constexpr int NBAR = 2 * HS_STAGES + 2 + 2 + 1;  // full, empty, accf, acce, qtma
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_TMEM + 16 + 1024;
     static constexpr int TMEM_COLS = (2 * N <= 128) ? 128 : ((2 * N <= 256) ? 256 : 512);
@@ -78,8 +78,7 @@ __global__ void __launch_bounds__(HS_THREADS, 1) hs_rescore_kernel(const __grid_
     uint64_t* empty = full + HS_STAGES;
     uint64_t* accf = empty + HS_STAGES;
     uint64_t* acce = accf + 2;
-    uint64_t* qready = acce + 2;
-    uint64_t* qtma = qready + 1;  // the followers' query blocks, by TMA
+    uint64_t* qtma = acce + 2;  // the followers' query blocks, by TMA
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
     float* wsm = reinterpret_cast<float*>(smem + C::OFF_W);
     uint8_t* qsm = smem + C::OFF_Q;
@@ -93,7 +92,6 @@ __global__ void __launch_bounds__(HS_THREADS, 1) hs_rescore_kernel(const __grid_
             mbar_init(&accf[i], 1);
             mbar_init(&acce[i], 128);
         }
-        mbar_init(qready, 128);
         mbar_init(qtma, 1);
         fence_mbar_init();
     }
@@ -204,8 +202,7 @@ __global__ void __launch_bounds__(HS_THREADS, 1) hs_rescore_kernel(const __grid_
             const int f = r / H, j = r % H;
             wsm[r] = __ldg(a.w + ((size_t)f * a.B + b) * H + j);
         }
-        fence_proxy_async_smem();
-        mbar_arrive(qready);
+        // the head weights, visible to every epilogue thread
         asm volatile("bar.sync 1, 128;" ::: "memory");
 
         // ------------------------------------------------------------ epilogue
