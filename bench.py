@@ -11,8 +11,11 @@ reads its keys from HBM.  Under torchrun each rank runs its own batch of
 requests (weak scaling, no collective on the data path); the time is the max
 over ranks.
 
-Prints ONE JSON line (rank 0).  `--impl reference` times the fp64 CPU oracle
-on the same workload instead (a bounded sample of it).
+Prints ONE JSON line (rank 0).  Besides the decode step it carries the L
+sweep (8K-128K) and the causal prefill (T = L = 8192: quantise + score, and
+the step with its top-2048) against the FP8 tensor peak measured in the same
+run (`--no-sweep`, `--no-prefill` skip them).  `--impl reference` times the
+fp64 CPU oracle on the same workload instead (a bounded sample of it).
 """
 from __future__ import annotations
 
@@ -35,6 +38,7 @@ WORKLOAD = "dsa_decode_b8_l32k"
 B, L, H, D, KTOP = 8, 32768, 64, 128, 2048
 L2_BYTES = 126 * 1024 * 1024
 SCORER_KERNEL = "stream_score_kernel"
+PREFILL_KERNELS = "quantize_query_kernel + prefill_score_kernel"
 
 
 def peaks():
@@ -487,6 +491,18 @@ def run_li(args, rank, world, local_rank):
                               "score_hbm_frac": round(B * Lx * decode_bytes_per_key() / (sc_ms * 1e-3) / 1e9 / hbm,
                                                       3)}
             del bx
+    prefill = None
+    if not args.no_prefill and rank == 0:
+        fp8 = fp8_peak_tflops()
+        px = PrefillBench(dev)
+        clocks = ClockSampler(local_rank)
+        clocks.start()
+        time.sleep(0.3)
+        r = px.run(max(10, args.steps // 2), args.warmup)
+        pclk = clocks.stop()
+        prefill = prefill_record(r, px, pclk, fp8)
+        del px
+        assert api.li_get_last_error() == 0
     if dist:
         dist.barrier()
         dist.destroy_process_group()
@@ -520,6 +536,8 @@ def run_li(args, rank, world, local_rank):
     }
     if sweep:
         out["sweep"] = sweep
+    if prefill:
+        out["prefill"] = prefill
     if world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline_sample()
     print(json.dumps(out), flush=True)
@@ -528,13 +546,83 @@ def run_li(args, rank, world, local_rank):
 # ---------------------------------------------------------------------------
 # other configurations (parity-test workloads; timed on request with --workload)
 # ---------------------------------------------------------------------------
+_FP8_PEAK = None
+
+
 def fp8_peak_tflops():
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(p):
-        d = json.load(open(p))
-        # FP8 dense = 2 x the measured bf16 dense rate (nominal 4.5 : 2.25 PF ratio)
-        return 2.0 * float(d["bf16_tflops"]), 2.0 * float(d["bf16_tflops_sustained"]), "measured bf16 x 2"
-    return 2 * 1590.0, 2 * 1400.0, "fallback bf16 x 2"
+    """Dense FP8 (e4m3) tensor-core rate of this GPU, measured the way the bf16 figures of
+    MEASURED_PEAKS.json were: an 8192^3 GEMM (2 * 8192^3 flops) timed with CUDA events, the best
+    of 10 launches (burst) and the rate of back-to-back launches over 4 s (sustained).  The GEMM
+    is torch._scaled_mm, e4m3 x e4m3 -> bf16 with tensor-wise scales, in both of cuBLAS's
+    accumulation modes; the faster one is taken.  Measured once per process.
+    Returns (burst TF/s, sustained TF/s, source)."""
+    global _FP8_PEAK
+    if _FP8_PEAK is not None:
+        return _FP8_PEAK
+    import torch
+    try:
+        n = 8192
+        g = torch.Generator(device="cuda").manual_seed(0)
+        a = torch.randn(n, n, device="cuda", generator=g).to(torch.float8_e4m3fn)
+        bt = torch.randn(n, n, device="cuda", generator=g).to(torch.float8_e4m3fn)
+        one = torch.ones((), device="cuda")
+        flops = 2.0 * n ** 3
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+        def mm(fast):
+            return torch._scaled_mm(a, bt.t(), one, one, out_dtype=torch.bfloat16, use_fast_accum=fast)
+
+        best, best_mode = 0.0, False
+        for fast in (False, True):
+            for _ in range(3):
+                mm(fast)
+            torch.cuda.synchronize()
+            for _ in range(10):
+                e0.record()
+                mm(fast)
+                e1.record()
+                torch.cuda.synchronize()
+                tf = flops / (e0.elapsed_time(e1) * 1e-3) / 1e12
+                if tf > best:
+                    best, best_mode = tf, fast
+        count = 0
+        t_end = time.time() + 4.0
+        e0.record()
+        while time.time() < t_end:
+            for _ in range(50):
+                mm(best_mode)
+            count += 50
+            e1.record()
+            e1.synchronize()
+        e1.record()
+        torch.cuda.synchronize()
+        sust = count * flops / (e0.elapsed_time(e1) * 1e-3) / 1e12
+        del a, bt
+        src = ("measured: torch._scaled_mm e4m3 8192^3, best of 10 and 4 s back to back "
+               f"({'fast' if best_mode else 'fp32'} accumulation)")
+        _FP8_PEAK = (best, sust, src)
+    except Exception as exc:  # no FP8 GEMM in this torch build: the nominal 2:1 ratio to measured bf16
+        p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+        if os.path.exists(p):
+            d = json.load(open(p))
+            _FP8_PEAK = (2.0 * float(d["bf16_tflops"]), 2.0 * float(d["bf16_tflops_sustained"]),
+                         f"measured bf16 x 2 (FP8 GEMM unavailable: {type(exc).__name__})")
+        else:
+            _FP8_PEAK = (2 * 1590.0, 2 * 1400.0, "fallback bf16 x 2")
+    return _FP8_PEAK
+
+
+def prefill_record(r, bx, clk, fp8):
+    """The causal prefill's figures against the FP8 tensor peak (algorithmic flops: visible
+    (t, s) pairs x 2 * H * d)."""
+    burst, sust, src = fp8
+    flops = bx.pairs * 2 * H * D
+    tf = flops / (r["score"] * 1e-3) / 1e12
+    return {"workload": "dsa_prefill_t8k", "T": bx.T, "L": bx.L, "H": H, "d": D, "k": KTOP,
+            "score_ms": r["score"], "step_ms": r["step"], "topk_ms": r["topk"],
+            "tflops": tf, "frac_of_fp8_burst": tf / burst, "frac_of_fp8_sustained": tf / sust,
+            "fp8_peak_tflops": {"burst": burst, "sustained": sust, "source": src},
+            "pairs_per_s": bx.pairs / (r["step"] * 1e-3), "kernels": PREFILL_KERNELS, "clocks": clk}
 
 
 class PrefillBench:
@@ -1033,7 +1121,6 @@ def run_other(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     hbm, which = peaks()
-    fp8_burst, fp8_sust, fp8_src = fp8_peak_tflops()
     clocks = ClockSampler(local_rank)
     if args.workload == "glm5_decode":
         # GLM-5's indexer shape (32 heads, d = 128, FP8 keys) on the decode step of the default workload
@@ -1062,6 +1149,7 @@ def run_other(args, rank, world, local_rank):
     elif args.workload == "lshard":
         out = run_lshard(dev, args, clocks)
     elif args.workload == "prefill":
+        fp8_burst, fp8_sust, fp8_src = fp8_peak_tflops()
         bx = PrefillBench(dev)
         clocks.start()
         r = bx.run(args.steps, args.warmup)
@@ -1071,7 +1159,7 @@ def run_other(args, rank, world, local_rank):
         out = {"metric": METRIC, "value": bx.pairs / (r["step"] * 1e-3), "unit": "keys/s (visible pairs)",
                "ms_per_step": r["step"], "higher_is_better": True, "dtype": "e4m3",
                "config": {"workload": "dsa_prefill_t8k", "T": bx.T, "L": bx.L, "H": H, "d": D, "k": KTOP},
-               "roofline": {"bound": "tensor", "kernel": "quantize_query_kernel + prefill_score_kernel",
+               "roofline": {"bound": "tensor", "kernel": PREFILL_KERNELS,
                             "achieved": achieved, "peak": fp8_burst, "peak_source": fp8_src, "unit": "TFLOP/s",
                             "frac": achieved / fp8_burst, "frac_of_sustained": achieved / fp8_sust,
                             "score_ms": r["score"]},
@@ -1130,6 +1218,8 @@ def main():
     ap.add_argument("--impl", default="li", choices=["li", "reference"])
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="skip the causal prefill record (and the FP8 peak it is measured against)")
     ap.add_argument("--workload", default="decode", choices=["decode", "glm5_decode", "prefill", "latent", "latent192", "latent_glm5", "hs_b1", "hs_b16", "mli", "lshard",
                              "sparse_attention", "table4"],
                     help="decode (default) is the benchmarked configuration; the others time the other "
