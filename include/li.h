@@ -170,10 +170,10 @@ li_status li_topk(const float* scores, int64_t scores_ld, const int32_t* len, in
  * 0) followed by li_topk(k_top) on the same scores, with identical results.
  * The difference is internal.  The pages run the indexer as a full scan that
  * scores every visible position, with top-k after it (IndexCache explainer,
- * Symbol Map), and this call keeps that order.  While
- * writing each score, the scorer also counts it by the top 11 bits of the
- * selection's order key.  The top-k takes its first radix digit from those
- * counts instead of sweeping the row for it.
+ * Symbol Map), and this call keeps that order.  While writing each score, the
+ * scorer also counts it by the top 11 bits of the selection's order key.  The
+ * top-k takes its first radix digit from those counts instead of sweeping the
+ * row for it.
  *   q, w, k, k_scale, cache_batch_rows, len, scores, scores_ld, desc
  *           as li_index_score (desc->causal must be 0; tensor-core path only:
  *           BF16 query, E4M3 keys, heads 64 or 32, dim 128).  scores_ld must be a
@@ -192,11 +192,29 @@ li_status li_decode_select(const void* q, const float* w, const void* k, const f
                            const int32_t* len, float* scores, int64_t scores_ld, const li_score_desc* desc, int k_top,
                            int32_t* idx, float* vals, void* workspace, size_t workspace_bytes, li_stream_t stream);
 
-/* Bytes of zeroed device workspace li_decode_select needs (0 when desc->rows <= 0). */
+/* Bytes of zeroed device workspace li_decode_select needs: desc->rows * 8 KB,
+ * rounded up to 256 (0 when desc->rows <= 0); the other fields do not change
+ * it.  It is also the histogram buffer li_decode_score_hist and li_topk_hist
+ * take. */
 size_t li_decode_select_workspace(const li_score_desc* desc);
 
-/* The two halves of li_decode_select, for callers that place them
- * separately; li_decode_select is exactly this pair on one stream.
+/* li_decode_select as its two kernels, for callers that place or time them
+ * separately; li_decode_select is exactly this pair on one stream, with the
+ * same arguments and workspace.
+ * li_decode_select_score: the scan (li_decode_score_hist into the workspace).
+ * li_decode_select_finish: the top-k from the scores and the workspace's
+ *   counts (li_topk_hist); leaves the workspace zero.  Its result equals
+ *   li_topk's (causal 0) on the same scores. */
+li_status li_decode_select_score(const void* q, const float* w, const void* k, const float* k_scale,
+                                 int64_t cache_batch_rows, const int32_t* len, float* scores, int64_t scores_ld,
+                                 const li_score_desc* desc, void* workspace, size_t workspace_bytes,
+                                 li_stream_t stream);
+li_status li_decode_select_finish(const float* scores, int64_t scores_ld, const int32_t* len,
+                                  const li_score_desc* desc, int k_top, int32_t* idx, float* vals, void* workspace,
+                                  size_t workspace_bytes, li_stream_t stream);
+
+/* The same pair with the histogram as a plain argument (the form the latent
+ * scan, the HS followers and the shard merge use as well).
  * li_decode_score_hist: li_index_score in its decode form (same arguments and
  *   restrictions as li_decode_select).  For every score it writes, it also
  *   adds 1 to hist[r * 2048 + (key >> 21)], where key is the score's order key

@@ -40,6 +40,8 @@ SIGNATURES = {
     "li_decode_select": (i32, [vp, vp, vp, vp, i64, vp, vp, i64, ctypes.POINTER(ScoreDesc), i32, vp, vp, vp, sz,
                                vp]),
     "li_decode_select_workspace": (sz, [ctypes.POINTER(ScoreDesc)]),
+    "li_decode_select_score": (i32, [vp, vp, vp, vp, i64, vp, vp, i64, ctypes.POINTER(ScoreDesc), vp, sz, vp]),
+    "li_decode_select_finish": (i32, [vp, i64, vp, ctypes.POINTER(ScoreDesc), i32, vp, vp, vp, sz, vp]),
     "li_decode_score_hist": (i32, [vp, vp, vp, vp, i64, vp, vp, i64, ctypes.POINTER(ScoreDesc), vp, vp]),
     "li_topk_hist": (i32, [vp, i64, vp, i32, i32, i32, vp, vp, vp, i32, vp]),
     "li_absorb_query": (i32, [vp, vp, vp, i32, i32, i32, i32, vp]),

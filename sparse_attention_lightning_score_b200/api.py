@@ -152,11 +152,18 @@ def li_topk(scores: torch.Tensor, k: int, *, lens: Optional[torch.Tensor] = None
     return (idx, vals) if with_values else idx
 
 
-def li_decode_select_workspace(rows: int, device) -> torch.Tensor:
-    """A zeroed workspace for li_decode_select over `rows` requests (it stays zero between calls)."""
-    desc = score_desc(rows, 64, 128, 0)
+def li_decode_select_workspace(rows: int, device, max_len: int = 0) -> torch.Tensor:
+    """A zeroed workspace for li_decode_select over `rows` rows: one 2048-bin histogram per row,
+    which every call leaves zero again (also the histogram buffer of li_decode_score_hist /
+    li_topk_hist / li_latent_score_hist).  `max_len` does not change its size."""
+    desc = score_desc(rows, 64, 128, int(max_len))
     need = _lib.load().li_decode_select_workspace(ctypes.byref(desc))
     return torch.zeros(max(int(need), 256), dtype=torch.uint8, device=device)
+
+
+def li_decode_select_hist_bytes(rows: int) -> int:
+    """Bytes of li_decode_select's workspace that hold the histograms (zero between calls)."""
+    return rows * 2048 * 4
 
 
 def li_decode_select(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, k_scale: torch.Tensor, k_top: int, *,
@@ -167,7 +174,8 @@ def li_decode_select(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, k_scale:
 
     Same arguments as li_index_score's decode form (q bf16 [B,64,128], k e4m3 [B,L,128] or [L,128],
     k_scale) and li_topk's k / outputs.  `workspace` is a zeroed buffer from li_decode_select_workspace
-    (made here when omitted); it is left zero again for the next call.
+    for these rows and this length (made here when omitted); its histograms are left zero again for
+    the next call.
     """
     _need(q, "q", torch.bfloat16)
     _need(w, "w", torch.float32)
@@ -185,7 +193,7 @@ def li_decode_select(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, k_scale:
     if scores is None:
         scores = torch.empty((R, _round4(L)), dtype=torch.float32, device=q.device)
     if workspace is None:
-        workspace = li_decode_select_workspace(R, q.device)
+        workspace = li_decode_select_workspace(R, q.device, L)
     if idx is None:  # (idx / vals may also be page-locked host tensors: the top-k writes them directly)
         idx = torch.empty((R, k_top), dtype=torch.int32, device=q.device)
     if with_values and vals is None:
@@ -196,6 +204,53 @@ def li_decode_select(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, k_scale:
                               _stream(stream))
     _lib.check("li_decode_select", st)
     return (scores, idx, vals) if with_values else (scores, idx)
+
+
+def li_decode_select_score(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, k_scale: torch.Tensor,
+                           workspace: torch.Tensor, *, lens: Optional[torch.Tensor] = None,
+                           scores: Optional[torch.Tensor] = None, tokens_per_request: int = 1, stream=None):
+    """First kernel of li_decode_select: the scores, plus the counts in the workspace's histograms."""
+    _need(q, "q", torch.bfloat16)
+    _need(w, "w", torch.float32)
+    _need(k, "k")
+    _need(k_scale, "k_scale", torch.float32)
+    if k.dtype == torch.float8_e4m3fn:
+        k = k.view(torch.uint8)
+    R, H, d = q.shape
+    L = k.shape[-2]
+    batch_rows = k.shape[1] if k.dim() == 3 else 0
+    if lens is not None:
+        _need(lens, "lens", torch.int32)
+    if scores is None:
+        scores = torch.empty((R, _round4(L)), dtype=torch.float32, device=q.device)
+    desc = score_desc(R, H, d, L, tokens_per_request=tokens_per_request)
+    st = _lib.load().li_decode_select_score(_ptr(q), _ptr(w), _ptr(k), _ptr(k_scale), batch_rows, _ptr(lens),
+                                            _ptr(scores), scores.stride(0), ctypes.byref(desc), _ptr(workspace),
+                                            workspace.numel(), _stream(stream))
+    _lib.check("li_decode_select_score", st)
+    return scores
+
+
+def li_decode_select_finish(scores: torch.Tensor, k_top: int, workspace: torch.Tensor, *, heads: int = 64,
+                            max_len: Optional[int] = None, lens: Optional[torch.Tensor] = None,
+                            with_values: bool = False, idx=None, vals=None, tokens_per_request: int = 1, stream=None):
+    """Second kernel of li_decode_select: the top-k from the scores and the workspace's counts."""
+    _need(scores, "scores", torch.float32)
+    rows, ld = scores.shape
+    if max_len is None:
+        max_len = ld
+    if lens is not None:
+        _need(lens, "lens", torch.int32)
+    if idx is None:
+        idx = torch.empty((rows, k_top), dtype=torch.int32, device=scores.device)
+    if with_values and vals is None:
+        vals = torch.empty((rows, k_top), dtype=torch.float32, device=scores.device)
+    desc = score_desc(rows, heads, 128, int(max_len), tokens_per_request=tokens_per_request)
+    st = _lib.load().li_decode_select_finish(_ptr(scores), ld, _ptr(lens), ctypes.byref(desc), int(k_top), _ptr(idx),
+                                             _ptr(vals) if with_values else None, _ptr(workspace), workspace.numel(),
+                                             _stream(stream))
+    _lib.check("li_decode_select_finish", st)
+    return (idx, vals) if with_values else idx
 
 
 def li_decode_score_hist(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, k_scale: torch.Tensor,

@@ -301,31 +301,78 @@ li_status li_topk_hist(const float* scores, int64_t scores_ld, const int32_t* le
     return launch_topk(a, stream);
 }
 
-li_status li_decode_select(const void* q, const float* w, const void* k, const float* k_scale, int64_t cache_batch_rows,
-                           const int32_t* len, float* scores, int64_t scores_ld, const li_score_desc* desc, int k_top,
-                           int32_t* idx, float* vals, void* workspace, size_t workspace_bytes, li_stream_t stream) {
+}  // extern "C"
+
+namespace li {
+namespace {
+
+// The checks li_decode_select and its two halves share.
+li_status check_decode_select(const void* q, const float* w, const void* k, const float* k_scale,
+                              int64_t cache_batch_rows, const float* scores, int64_t scores_ld,
+                              const li_score_desc* desc, int k_top, bool need_idx, const int32_t* idx,
+                              const void* workspace, size_t workspace_bytes) {
     if (!desc) return LI_ERR_INVALID_ARG;
     const li_score_desc d = *desc;
     if (d.rows < 0 || d.heads <= 0 || d.dim <= 0 || d.max_len < 0 || cache_batch_rows < 0 || d.causal)
         return LI_ERR_INVALID_ARG;
-    if (k_top < 1 || k_top > LI_TOPK_MAX_LEN || d.max_len > LI_TOPK_MAX_LEN) return LI_ERR_INVALID_ARG;
+    if (need_idx && (k_top < 1 || k_top > LI_TOPK_MAX_LEN)) return LI_ERR_INVALID_ARG;
+    if (d.max_len > LI_TOPK_MAX_LEN) return LI_ERR_INVALID_ARG;
     if (d.rows == 0) return LI_OK;
     if (d.q_dtype != LI_DTYPE_BF16 || d.k_dtype != LI_DTYPE_E4M3) return LI_ERR_UNSUPPORTED;
     if ((d.heads != 64 && d.heads != 32) || d.dim != 128) return LI_ERR_UNSUPPORTED;
-    if (!idx || !workspace || workspace_bytes < li_decode_select_workspace(&d) || !aligned(workspace, 256))
+    if ((need_idx && !idx) || !workspace || workspace_bytes < li_decode_select_workspace(&d) ||
+        !aligned(workspace, 256))
         return LI_ERR_INVALID_ARG;
     if (d.tokens_per_request > 1 && d.rows % d.tokens_per_request != 0) return LI_ERR_INVALID_ARG;
     if (d.max_len > 0) {
-        if (!q || !w || !k || !k_scale || !scores || scores_ld < d.max_len || (scores_ld % 4) != 0)
-            return LI_ERR_INVALID_ARG;
-        if (!aligned(k, 16) || !aligned(q, 16) || !aligned(scores, 16)) return LI_ERR_INVALID_ARG;
+        if (!scores || scores_ld < d.max_len || (scores_ld % 4) != 0) return LI_ERR_INVALID_ARG;
+        if (!aligned(scores, 16)) return LI_ERR_INVALID_ARG;
+        if (!need_idx) {
+            if (!q || !w || !k || !k_scale) return LI_ERR_INVALID_ARG;
+            if (!aligned(k, 16) || !aligned(q, 16)) return LI_ERR_INVALID_ARG;
+        }
     }
-    uint32_t* hist = static_cast<uint32_t*>(workspace);
-    const li_status s = li_decode_score_hist(q, w, k, k_scale, cache_batch_rows, len, scores, scores_ld, desc, hist,
-                                             stream);
+    return LI_OK;
+}
+
+}  // namespace
+}  // namespace li
+
+extern "C" {
+
+li_status li_decode_select_score(const void* q, const float* w, const void* k, const float* k_scale,
+                                 int64_t cache_batch_rows, const int32_t* len, float* scores, int64_t scores_ld,
+                                 const li_score_desc* desc, void* workspace, size_t workspace_bytes,
+                                 li_stream_t stream) {
+    li_status s = check_decode_select(q, w, k, k_scale, cache_batch_rows, scores, scores_ld, desc, 1, false, nullptr,
+                                      workspace, workspace_bytes);
+    if (s != LI_OK || desc->rows == 0 || desc->max_len == 0) return s;
+    return li_decode_score_hist(q, w, k, k_scale, cache_batch_rows, len, scores, scores_ld, desc,
+                                static_cast<uint32_t*>(workspace), stream);
+}
+
+li_status li_decode_select_finish(const float* scores, int64_t scores_ld, const int32_t* len,
+                                  const li_score_desc* desc, int k_top, int32_t* idx, float* vals, void* workspace,
+                                  size_t workspace_bytes, li_stream_t stream) {
+    li_status s = check_decode_select(nullptr, nullptr, nullptr, nullptr, 0, scores, scores_ld, desc, k_top, true,
+                                      idx, workspace, workspace_bytes);
+    if (s != LI_OK || desc->rows == 0) return s;
+    const li_score_desc d = *desc;
+    return li_topk_hist(scores, d.max_len > 0 ? scores_ld : 4, len, d.rows, d.max_len, k_top, idx, vals,
+                        static_cast<uint32_t*>(workspace), d.tokens_per_request, stream);
+}
+
+li_status li_decode_select(const void* q, const float* w, const void* k, const float* k_scale, int64_t cache_batch_rows,
+                           const int32_t* len, float* scores, int64_t scores_ld, const li_score_desc* desc, int k_top,
+                           int32_t* idx, float* vals, void* workspace, size_t workspace_bytes, li_stream_t stream) {
+    li_status s = check_decode_select(q, w, k, k_scale, cache_batch_rows, scores, scores_ld, desc, k_top, true, idx,
+                                      workspace, workspace_bytes);
+    if (s != LI_OK || desc->rows == 0) return s;
+    s = li_decode_select_score(q, w, k, k_scale, cache_batch_rows, len, scores, scores_ld, desc, workspace,
+                               workspace_bytes, stream);
     if (s != LI_OK) return s;
-    return li_topk_hist(scores, d.max_len > 0 ? scores_ld : 4, len, d.rows, d.max_len, k_top, idx, vals, hist,
-                        d.tokens_per_request, stream);
+    return li_decode_select_finish(scores, desc->max_len > 0 ? scores_ld : 4, len, desc, k_top, idx, vals, workspace,
+                                   workspace_bytes, stream);
 }
 
 li_status li_host_device_pointer(const void* host_ptr, void** dev_ptr) {
@@ -507,6 +554,7 @@ size_t li_workspace_size(int op, int rows, int max_len, int k) {
     case LI_OP_DECODE_SELECT: {
         li_score_desc d{};
         d.rows = rows;
+        d.max_len = max_len;
         return li_decode_select_workspace(&d);
     }
     }

@@ -269,7 +269,7 @@ class DecodeLayerStack:
         self.sel = torch.empty(step.n_slots, self.B, self.k, dtype=torch.int32, device=self.out.device)
         self.scores = torch.empty(step.n_slots, self.B, (self.L + 3) // 4 * 4, dtype=torch.float32,
                                   device=self.out.device)
-        self.hist = [self.api.li_decode_select_workspace(self.B, self.out.device) for _ in range(step.n_slots)]
+        self.hist = [self.api.li_decode_select_workspace(self.B, self.out.device, self.L) for _ in range(step.n_slots)]
         self.att_ws = self.api.li_sparse_attention_workspace(self.B, self.qa[0].shape[1], self.k, self.out.device)
         return step
 

@@ -39,6 +39,7 @@ def test_workspace_size_by_operation_matches_each_calls_own_size():
         d = _lib.ScoreDesc(rows, 64, 128, 8192, 1, 0, _lib.LI_DTYPE_BF16, _lib.LI_DTYPE_E4M3)
         assert lib.li_workspace_size(_lib.LI_OP_SCORE, rows, 8192, 2048) == lib.li_index_score_workspace(ctypes.byref(d))
         d.causal = 0
+        d.max_len = 32768
         assert lib.li_workspace_size(_lib.LI_OP_DECODE_SELECT, rows, 32768, 2048) == \
             lib.li_decode_select_workspace(ctypes.byref(d))
         assert lib.li_workspace_size(_lib.LI_OP_TOPK, rows, 32768, 2048) == 0
@@ -164,6 +165,13 @@ def test_graph_calls_check_arguments_on_host():
     assert lib.li_graph_instantiate(ctypes.c_void_p(256), 1, None) == _lib.LI_ERR_INVALID_ARG
     assert lib.li_graph_launch(None, None) == _lib.LI_ERR_INVALID_ARG
     assert lib.li_graph_destroy(None) == _lib.LI_OK
+
+
+def test_decode_select_workspace_is_one_histogram_per_row():
+    lib = _lib.load()
+    for L in (0, 1000, 32768, 262144):
+        d = _lib.ScoreDesc(8, 64, 128, L, 0, 0, _lib.LI_DTYPE_BF16, _lib.LI_DTYPE_E4M3)
+        assert lib.li_decode_select_workspace(ctypes.byref(d)) == 8 * 2048 * 4
 
 
 def test_multi_token_descriptor_checked_on_host():

@@ -35,6 +35,10 @@ def _two_calls(q, w, k8, ks, lens, k_top):
     return sc, idx, vals
 
 
+def _hist_zero(ws, rows):
+    return int(ws[:api.li_decode_select_hist_bytes(rows)].count_nonzero()) == 0
+
+
 def _assert_same(got, want, lens):
     sc, idx, vals = got
     sc_r, idx_r, vals_r = want
@@ -56,11 +60,36 @@ def _assert_same(got, want, lens):
 def test_decode_select_matches_score_then_topk(B, L, lens, k_top):
     case = synth.dsa_decode(B=B, L=L, seed=40 + B, lens=lens)
     q, w, k8, ks, ln = _dev(case)
-    ws = api.li_decode_select_workspace(B, DEV)
+    ws = api.li_decode_select_workspace(B, DEV, L)
     got = api.li_decode_select(q, w, k8, ks, k_top, lens=ln, workspace=ws, with_values=True)
     _assert_same(got, _two_calls(q, w, k8, ks, ln, k_top), ln)
     assert api.li_get_last_error() == LI_OK
-    assert int(ws.count_nonzero()) == 0
+    assert _hist_zero(ws, B)
+
+
+def test_decode_select_halves_equal_the_call():
+    case = synth.dsa_decode(B=4, L=20000, seed=31, lens=[20000, 15000, 2049, 300])
+    q, w, k8, ks, ln = _dev(case)
+    ws = api.li_decode_select_workspace(4, DEV, 20000)
+    sc = api.li_decode_select_score(q, w, k8, ks, ws, lens=ln)
+    idx, vals = api.li_decode_select_finish(sc, 2048, ws, max_len=20000, lens=ln, with_values=True)
+    _assert_same((sc, idx, vals), _two_calls(q, w, k8, ks, ln, 2048), ln)
+    assert api.li_get_last_error() == LI_OK
+    assert _hist_zero(ws, 4)
+
+
+def test_decode_select_many_long_rows():
+    # 300 rows of 70,000 positions over one shared cache: more rows than SMs, one scorer CTA and one
+    # top-k CTA per row, slices far above the cluster top-k's 4K
+    case = synth.dsa_decode(B=1, L=70000, seed=33)
+    g = torch.Generator().manual_seed(33)
+    q = torch.randn(300, 64, 128, generator=g).to(torch.bfloat16).to(DEV)
+    w = (torch.randn(300, 64, generator=g) * 0.1).to(DEV)
+    k8, ks = case.k8[0].to(DEV), case.ks[0].to(DEV)
+    lens = torch.randint(60000, 70001, (300,), generator=g, dtype=torch.int32).to(DEV)
+    got = api.li_decode_select(q, w, k8, ks, 2048, lens=lens, with_values=True)
+    _assert_same(got, _two_calls(q, w, k8, ks, lens, 2048), lens)
+    assert api.li_get_last_error() == LI_OK
 
 
 def test_decode_select_against_oracle():
@@ -78,14 +107,14 @@ def test_decode_select_against_oracle():
 
 
 def test_decode_select_workspace_reused_across_steps():
-    ws = api.li_decode_select_workspace(4, DEV)
+    ws = api.li_decode_select_workspace(4, DEV, 9000)
     for seed in (1, 2, 3):
         case = synth.dsa_decode(B=4, L=9000, seed=seed, lens=[9000, 7000, 3000, 2100])
         q, w, k8, ks, ln = _dev(case)
         got = api.li_decode_select(q, w, k8, ks, 2048, lens=ln, workspace=ws, with_values=True)
         _assert_same(got, _two_calls(q, w, k8, ks, ln, 2048), ln)
     assert api.li_get_last_error() == LI_OK
-    assert int(ws.count_nonzero()) == 0
+    assert _hist_zero(ws, 4)
 
 
 def test_decode_select_shared_cache_and_many_rows():
@@ -106,22 +135,22 @@ def test_decode_select_all_scores_equal():
     case = synth.dsa_decode(B=2, L=40000, seed=5)
     q, _, k8, ks, ln = _dev(case)
     w = torch.zeros(2, 64, device=DEV)
-    ws = api.li_decode_select_workspace(2, DEV)
+    ws = api.li_decode_select_workspace(2, DEV, 40000)
     sc, idx = api.li_decode_select(q, w, k8, ks, 2048, lens=ln, workspace=ws)
     assert np.array_equal(_np(idx), np.tile(np.arange(2048, dtype=np.int32), (2, 1)))
     assert api.li_get_last_error() == LI_OK
-    assert int(ws.count_nonzero()) == 0
+    assert _hist_zero(ws, 2)
 
 
 def test_decode_select_dirty_workspace_is_reported_and_healed():
     case = synth.dsa_decode(B=3, L=12000, seed=6)
     q, w, k8, ks, ln = _dev(case)
-    ws = api.li_decode_select_workspace(3, DEV)
+    ws = api.li_decode_select_workspace(3, DEV, 12000)
     ws.view(torch.int32)[::7] = 3  # counts that describe no row
     got = api.li_decode_select(q, w, k8, ks, 2048, lens=ln, workspace=ws, with_values=True)
     _assert_same(got, _two_calls(q, w, k8, ks, ln, 2048), ln)
     assert api.li_get_last_error() == LI_ERR_BOUNDS
-    assert int(ws.count_nonzero()) == 0
+    assert _hist_zero(ws, 3)
     got = api.li_decode_select(q, w, k8, ks, 2048, lens=ln, workspace=ws, with_values=True)
     _assert_same(got, _two_calls(q, w, k8, ks, ln, 2048), ln)
     assert api.li_get_last_error() == LI_OK
