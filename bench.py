@@ -297,9 +297,10 @@ class DecodeBench:
     """Decode-step launches over rotating key caches, as graphs.
 
     A step is li_decode_select: the scorer (which also counts each row's first
-    radix digit into a histogram) and the top-k that starts from it.  The two
-    kernels are also timed alone through the call's two halves: the scorer
-    into a scratch histogram, the top-k from a saved histogram restored by a
+    radix digit into a histogram and leaves its keys bucketed by that digit)
+    and the selection from those buckets.  The two kernels are also timed
+    alone through the call's two halves: the scorer into a scratch workspace,
+    the selection from a saved workspace whose histograms are restored by a
     device copy before each launch (the copy's own time is subtracted)."""
 
     def __init__(self, dev, Lx, seed, heads=H):
@@ -313,27 +314,28 @@ class DecodeBench:
         self.q, self.w = self.case.q.to(dev), self.case.w.to(dev)
         self.sc = torch.empty((B, Lx), dtype=torch.float32, device=dev)
         self.idx = torch.empty((B, KTOP), dtype=torch.int32, device=dev)
-        self.ws = api.li_decode_select_workspace(B, dev)
-        nh = B * 2048
-        self.hist_scratch = api.li_decode_select_workspace(B, dev).view(torch.int32)[:nh]
-        # scores + their histogram for the top-k-only timing
+        self.ws = api.li_decode_select_workspace(B, dev, Lx)
+        self.ws_scratch = api.li_decode_select_workspace(B, dev, Lx)
+        # scores + a workspace the scorer filled, for the selection-only timing
+        nh = api.li_decode_select_hist_bytes(B)
         self.sc_t = torch.empty_like(self.sc)
         self.idx_t = torch.empty_like(self.idx)
-        self.hist_saved = api.li_decode_select_workspace(B, dev).view(torch.int32)[:nh]
-        self.hist_t = api.li_decode_select_workspace(B, dev).view(torch.int32)[:nh]
+        self.ws_t = api.li_decode_select_workspace(B, dev, Lx)
         kk, ss = self.sets[0]
-        api.li_decode_score_hist(self.q, self.w, kk, ss, self.hist_saved, scores=self.sc_t)
+        api.li_decode_select_score(self.q, self.w, kk, ss, self.ws_t, scores=self.sc_t)
+        self.hist_saved = self.ws_t[:nh].clone()
+        self.hist_t = self.ws_t[:nh]
 
     def score(self, i):
         kk, ss = self.sets[i % self.n]
-        self.api.li_decode_score_hist(self.q, self.w, kk, ss, self.hist_scratch, scores=self.sc)
+        self.api.li_decode_select_score(self.q, self.w, kk, ss, self.ws_scratch, scores=self.sc)
 
     def restore(self):
         self.hist_t.copy_(self.hist_saved)
 
     def topk(self):
         self.restore()
-        self.api.li_topk_hist(self.sc_t, KTOP, self.hist_t, idx=self.idx_t)
+        self.api.li_decode_select_finish(self.sc_t, KTOP, self.ws_t, heads=self.heads, max_len=self.Lx, idx=self.idx_t)
 
     def step(self, i):
         kk, ss = self.sets[i % self.n]
@@ -446,10 +448,32 @@ def run_li(args, rank, world, local_rank):
         [ms, score_ms, topk_ms, direct_ms, single_ms], device=dev)
     launches = 2 * args.steps
 
-    # ---- end to end through the public API: each step copies the pinned host
-    # query/weights in, scores + selects, and copies the indices out, as one
-    # graph-captured DecodeIndexer step (one indexer per rotating cache copy)
-    from sparse_attention_lightning_score_b200.step import DecodeIndexer
+    # ---- end to end through the public API.  Throughput: K independent steps as one DecodePipeline
+    # graph, each step copying its own pinned host query/weights in and its selected positions out,
+    # the copies of neighbouring steps overlapping its kernels.  Latency: the same step alone as one
+    # graph-captured DecodeIndexer step (copy in -> li_decode_select -> copy out), back to back.
+    from sparse_attention_lightning_score_b200.step import DecodeIndexer, DecodePipeline
+    pipe = DecodePipeline([bench.sets[i % bench.n] for i in range(args.steps)], H, KTOP)
+    for i in range(args.steps):
+        pipe.q_host[i].copy_(bench.case.q)
+        pipe.w_host[i].copy_(bench.case.w)
+    for _ in range(max(1, args.warmup // 2)):
+        pipe.run(sync=False)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record()
+    pipe.run(sync=False)
+    a1.record()
+    torch.cuda.synchronize()
+    e2e_ms = a0.elapsed_time(a1) / args.steps
+    # the selections that came back to the host match the device-side graph's
+    bench.step_graphs[(args.steps - 1) % bench.n].replay()
+    torch.cuda.synchronize()
+    assert torch.equal(pipe.idx_host[args.steps - 1], bench.idx.cpu())
+    h2d, d2h = pipe.h2d_bytes_per_step, pipe.d2h_bytes_per_step
+    del pipe
     indexers = [DecodeIndexer(kk, ss, H, KTOP) for kk, ss in bench.sets]
     for ix in indexers:
         ix.q_host.copy_(bench.case.q)
@@ -457,23 +481,14 @@ def run_li(args, rank, world, local_rank):
     for i in range(args.warmup):
         indexers[i % len(indexers)].step(sync=False)
     torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
-    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a0.record()
     for i in range(args.steps):
         indexers[i % len(indexers)].step(sync=False)
     a1.record()
     torch.cuda.synchronize()
-    e2e_ms = a0.elapsed_time(a1) / args.steps
-    (e2e_ms,) = li_dist.max_over_ranks([e2e_ms], device=dev)
-    # the selections that came back to the host match the device-side graph's
-    ref_idx = bench.idx.clone()
-    bench.step_graphs[(args.steps - 1) % bench.n].replay()
-    torch.cuda.synchronize()
-    assert torch.equal(indexers[(args.steps - 1) % len(indexers)].idx_host, bench.idx.cpu())
-    h2d, d2h = indexers[0].h2d_bytes, indexers[0].d2h_bytes
-    del indexers, ref_idx
+    lat_ms = a0.elapsed_time(a1) / args.steps
+    e2e_ms, lat_ms = li_dist.max_over_ranks([e2e_ms, lat_ms], device=dev)
+    del indexers
     assert api.li_get_last_error() == 0
 
     sweep = None
@@ -530,7 +545,10 @@ def run_li(args, rank, world, local_rank):
         "direct_us_per_step": direct_ms * 1e3, "graph_per_step_us": single_ms * 1e3,
         "e2e": {"value": world * B * L / (e2e_ms * 1e-3), "unit": "keys/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-                "api": "DecodeIndexer.step (graph: H2D q,w -> li_decode_select -> D2H indices)"},
+                "api": "DecodePipeline.run: K independent steps in one graph, each H2D q,w -> li_decode_select "
+                       "-> D2H indices, neighbouring steps' copies overlapping its kernels",
+                "latency_ms_per_step": lat_ms,
+                "latency_api": "DecodeIndexer.step (one step per graph: H2D q,w -> li_decode_select -> D2H indices)"},
         "gpu_launches": launches,
         "clocks": clk,
     }
@@ -889,7 +907,7 @@ def run_lshard(dev, args, clocks):
 
     reps = max(3, args.steps // 4)
     clocks.start()
-    ws = api.li_decode_select_workspace(B, dev)
+    ws = api.li_decode_select_workspace(B, dev, Lt)
     sc = torch.empty((B, Lt), dtype=torch.float32, device=dev)
     idx = torch.empty((B, KTOP), dtype=torch.int32, device=dev)
     vals = torch.empty((B, KTOP), dtype=torch.float32, device=dev)
@@ -949,7 +967,7 @@ def run_table4(dev, args, clocks):
         ks = [dcase.ks.to(dev).clone() for _ in range(ncopy)]
         q = [dcase.q.to(dev)] * 4
         w = [dcase.w.to(dev)] * 4
-        ws = [api.li_decode_select_workspace(1, dev) for _ in range(4)]
+        ws = [api.li_decode_select_workspace(1, dev, Lx) for _ in range(4)]
         sc = torch.empty((1, Lx), dtype=torch.float32, device=dev)
         idx = torch.empty((4, 1, KTOP), dtype=torch.int32, device=dev)
         C = min(8192, Lx)

@@ -58,7 +58,7 @@ class DecodeIndexer:
         self.w_host = self.in_host[qbytes:].view(torch.float32).view(B, heads)
         self.scores = torch.empty((B, (L + 3) // 4 * 4), dtype=torch.float32, device=dev)
         self.idx_dev = torch.empty((B, k), dtype=torch.int32, device=dev)
-        self.ws = api.li_decode_select_workspace(B, dev)
+        self.ws = api.li_decode_select_workspace(B, dev, L)
         self.idx_host = torch.empty((B, k), dtype=torch.int32).pin_memory()
         self._launch()  # warm-up: loads the module, sets kernel attributes, checks arguments
         torch.cuda.synchronize(dev)
@@ -98,3 +98,113 @@ class DecodeIndexer:
     @property
     def d2h_bytes(self) -> int:
         return self.idx_host.numel() * 4
+
+
+class DecodePipeline:
+    """Independent decode-indexer steps back to back, with their transfers overlapped.
+
+    A serving engine that runs the indexer of many independent steps (other
+    layers' indexers, other request batches) does not need step i's selection
+    before step i+1's inputs can move.  Here ``steps`` such steps form one CUDA
+    graph on three streams:
+
+        copy stream 1:  H2D(i)   H2D(i+1)   H2D(i+2) ...
+        main stream:          select(i)  select(i+1)  select(i+2) ...
+        copy stream 2:                 D2H(i)     D2H(i+1) ...
+
+    Step i's inputs come from its own page-locked host buffer into device
+    slot i % 2 while step i-1's kernels run; its selected positions go from
+    device slot i % 2 to its own page-locked host buffer while step i+1's
+    kernels run.  Every step still copies its own inputs in and its own result
+    out; only the waiting is overlapped.  The slots are reused two steps later,
+    after their previous step's kernels (inputs) and result copy (outputs)
+    have finished.  Every kernel in the graph is an li kernel.
+
+    caches: a list of ``steps`` (k8, ks) key caches, one per step (a cache may
+    repeat); heads, k, lens as for ``DecodeIndexer``.  The host inputs are
+    ``q_host[i]`` (bf16 [B,H,d]) and ``w_host[i]`` (fp32 [B,H]); ``run()``
+    replays the graph and returns the list of pinned int32 [B, k] results.
+    """
+
+    def __init__(self, caches, heads: int, k: int, lens: Optional[torch.Tensor] = None):
+        self.caches = list(caches)
+        k8, ks = self.caches[0]
+        if not (k8.is_cuda and ks.is_cuda):
+            raise ValueError("the key caches must be resident on a CUDA device")
+        B, L, d = k8.shape
+        self.B, self.L, self.d, self.H, self.k, self.lens = B, L, d, heads, k, lens
+        self.steps = S = len(self.caches)
+        dev = k8.device
+        qbytes = B * heads * d * 2
+        self.nbytes = nbytes = qbytes + B * heads * 4
+        self.in_host = [torch.zeros(nbytes, dtype=torch.uint8).pin_memory() for _ in range(S)]
+        self.q_host = [t[:qbytes].view(torch.bfloat16).view(B, heads, d) for t in self.in_host]
+        self.w_host = [t[qbytes:].view(torch.float32).view(B, heads) for t in self.in_host]
+        self.idx_host = [torch.empty((B, k), dtype=torch.int32).pin_memory() for _ in range(S)]
+        self.in_dev = [torch.zeros(nbytes, dtype=torch.uint8, device=dev) for _ in range(2)]
+        self.q_dev = [t[:qbytes].view(torch.bfloat16).view(B, heads, d) for t in self.in_dev]
+        self.w_dev = [t[qbytes:].view(torch.float32).view(B, heads) for t in self.in_dev]
+        self.idx_dev = [torch.empty((B, k), dtype=torch.int32, device=dev) for _ in range(2)]
+        self.scores = torch.empty((B, (L + 3) // 4 * 4), dtype=torch.float32, device=dev)
+        self.ws = api.li_decode_select_workspace(B, dev, L)
+        self.s_in = torch.cuda.Stream(device=dev)
+        self.s_out = torch.cuda.Stream(device=dev)
+        self._select(0, torch.cuda.current_stream(dev))  # warm-up: module, kernel attributes, argument checks
+        torch.cuda.synchronize(dev)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self._capture(torch.cuda.current_stream(dev))
+
+    def _select(self, i, stream):
+        j = i % 2
+        k8, ks = self.caches[i]
+        api.li_decode_select(self.q_dev[j], self.w_dev[j], k8, ks, self.k, lens=self.lens, scores=self.scores,
+                             workspace=self.ws, idx=self.idx_dev[j], stream=stream)
+
+    def _capture(self, main):
+        fork = torch.cuda.Event()
+        fork.record(main)
+        self.s_in.wait_event(fork)
+        self.s_out.wait_event(fork)
+        done_sel, done_out = [], []
+        for i in range(self.steps):
+            j = i % 2
+            with torch.cuda.stream(self.s_in):
+                if i >= 2:
+                    self.s_in.wait_event(done_sel[i - 2])  # slot j's inputs were read by step i - 2
+                self.in_dev[j].copy_(self.in_host[i], non_blocking=True)
+                arrived = torch.cuda.Event()
+                arrived.record(self.s_in)
+            main.wait_event(arrived)
+            if i >= 2:
+                main.wait_event(done_out[i - 2])  # slot j's result of step i - 2 has been copied out
+            self._select(i, main)
+            ev = torch.cuda.Event()
+            ev.record(main)
+            done_sel.append(ev)
+            with torch.cuda.stream(self.s_out):
+                self.s_out.wait_event(ev)
+                self.idx_host[i].copy_(self.idx_dev[j], non_blocking=True)
+                ev_o = torch.cuda.Event()
+                ev_o.record(self.s_out)
+                done_out.append(ev_o)
+        main.wait_event(done_out[-1])
+        joined = torch.cuda.Event()
+        joined.record(self.s_in)
+        main.wait_event(joined)
+
+    def run(self, sync: bool = True):
+        """Replay the ``steps`` steps; returns the pinned host results (valid once the stream has
+        been synchronised: ``sync=True`` waits)."""
+        self.graph.replay()
+        if sync:
+            torch.cuda.current_stream().synchronize()
+        return self.idx_host
+
+    @property
+    def h2d_bytes_per_step(self) -> int:
+        return self.nbytes
+
+    @property
+    def d2h_bytes_per_step(self) -> int:
+        return self.B * self.k * 4

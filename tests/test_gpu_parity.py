@@ -341,6 +341,30 @@ def test_decode_indexer_graph_step():
     assert api.li_get_last_error() == LI_OK
 
 
+def test_decode_pipeline_matches_single_steps():
+    """Five independent steps in one pipelined graph (transfers overlapped with the kernels, device
+    slots reused two steps later) select exactly what five separate graph steps select."""
+    from sparse_attention_lightning_score_b200.step import DecodeIndexer, DecodePipeline
+    cases = [synth.dsa_decode(B=3, L=6000, k_top=500, seed=70 + i) for i in range(3)]
+    caches = [(c.k8.to(DEV), c.ks.to(DEV)) for c in cases]
+    order = [0, 1, 2, 1, 0]
+    pipe = DecodePipeline([caches[i] for i in order], heads=64, k=500)
+    g = torch.Generator().manual_seed(77)
+    qs = [torch.randn(3, 64, 128, generator=g).to(torch.bfloat16) for _ in order]
+    ws = [torch.randn(3, 64, generator=g) * 0.1 for _ in order]
+    for i in range(len(order)):
+        pipe.q_host[i].copy_(qs[i])
+        pipe.w_host[i].copy_(ws[i])
+    for rep in range(2):  # the same graph twice: slots and host buffers are reused
+        got = [t.clone() for t in pipe.run()]
+        for i, c in enumerate(order):
+            one = DecodeIndexer(caches[c][0], caches[c][1], heads=64, k=500)
+            want = one.step(qs[i], ws[i]).clone()
+            assert torch.equal(got[i], want), (rep, i)
+    assert pipe.h2d_bytes_per_step == 3 * 64 * 128 * 2 + 3 * 64 * 4 and pipe.d2h_bytes_per_step == 3 * 500 * 4
+    assert api.li_get_last_error() == LI_OK
+
+
 def test_copy_from_host_kernel():
     src = torch.arange(1000 * 16 + 7, dtype=torch.uint8).pin_memory()  # a tail that is not 16 bytes
     dst = torch.zeros(src.numel(), dtype=torch.uint8, device=DEV)
