@@ -74,7 +74,7 @@ __global__ void __launch_bounds__(StreamCfg<NH, FP8, KBLK, STAGES, NACC, HIST>::
     const int b = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     pdl_trigger();  // the next kernel of the stream may be scheduled; it waits for this one itself
-    if (blockIdx.x * a.tiles_per_cta >= (a.max_len + C::M - 1) / C::M) return;  // no tile for any length
+    if ((int)blockIdx.x >= (a.max_len + C::M - 1) / C::M) return;  // no tile for any length
 
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* empty = full + STAGES;
@@ -144,8 +144,11 @@ __global__ void __launch_bounds__(StreamCfg<NH, FP8, KBLK, STAGES, NACC, HIST>::
     }
     len_b = max(0, len_b - (tokens - 1 - b % tokens));
     const int ntiles = (len_b + C::M - 1) / C::M;
-    const int t0 = blockIdx.x * a.tiles_per_cta;
-    const int nt = min(t0 + a.tiles_per_cta, ntiles) - t0;
+    // tiles are dealt round robin: CTA c takes tiles c, c + G, c + 2G, ... (G = CTAs per request), so
+    // that every CTA reads from the whole of its request's cache
+    const int t0 = blockIdx.x;
+    const int tstride = gridDim.x;
+    const int nt = t0 < ntiles ? (ntiles - t0 + tstride - 1) / tstride : 0;
     if (nt <= 0) goto done;  // uniform over the CTA
 
     if (warp == 0) {
@@ -158,7 +161,7 @@ __global__ void __launch_bounds__(StreamCfg<NH, FP8, KBLK, STAGES, NACC, HIST>::
             uint32_t ph = 0;
             bool ok = true;
             for (int it = 0; ok && it < nt; ++it) {
-                const int y = (int)(rowbase + (long long)(t0 + it) * C::M);
+                const int y = (int)(rowbase + (long long)(t0 + it * tstride) * C::M);
                 for (int kb = 0; kb < KBLK; ++kb) {
                     // FP8: the last stage's buffer first holds the query row, until it is quantised
                     if (FP8 && stage == STAGES - 1 && ph == 0u && !mbar_wait(qready, 0, a.err)) { ok = false; break; }
@@ -266,7 +269,7 @@ __global__ void __launch_bounds__(StreamCfg<NH, FP8, KBLK, STAGES, NACC, HIST>::
         for (int it = 0; it < nt; ++it) {
             const int acc = it % NACC;
             const uint32_t aph = (uint32_t)(it / NACC) & 1u;
-            const int s = (t0 + it) * C::M + g * 32 + lane;
+            const int s = (t0 + it * tstride) * C::M + g * 32 + lane;
             float sk = 1.f;
             if (FP8 && s < len_b) sk = __ldg(a.kscale + srow + s);
             if (!mbar_wait(&accf[acc], aph, a.err)) break;
