@@ -297,8 +297,8 @@ class DecodeBench:
     """Decode-step launches over rotating key caches, as graphs.
 
     A step is li_decode_select: the scorer (which also counts each row's first
-    radix digit into a histogram and leaves its keys bucketed by that digit)
-    and the selection from those buckets.  The two kernels are also timed
+    radix digit into a histogram) and the top-k that starts from that
+    histogram.  The two kernels are also timed
     alone through the call's two halves: the scorer into a scratch workspace,
     the selection from a saved workspace whose histograms are restored by a
     device copy before each launch (the copy's own time is subtracted)."""
