@@ -315,6 +315,10 @@ class DecodeBench:
         self.sc = torch.empty((B, Lx), dtype=torch.float32, device=dev)
         self.idx = torch.empty((B, KTOP), dtype=torch.int32, device=dev)
         self.ws = api.li_decode_select_workspace(B, dev, Lx)
+        # a second set for the pipelined timing: two independent steps in flight on two streams
+        self.sc2 = torch.empty_like(self.sc)
+        self.idx2 = torch.empty_like(self.idx)
+        self.ws2 = api.li_decode_select_workspace(B, dev, Lx)
         self.ws_scratch = api.li_decode_select_workspace(B, dev, Lx)
         # scores + a workspace the scorer filled, for the selection-only timing
         nh = api.li_decode_select_hist_bytes(B)
@@ -341,6 +345,12 @@ class DecodeBench:
         kk, ss = self.sets[i % self.n]
         self.api.li_decode_select(self.q, self.w, kk, ss, KTOP, scores=self.sc, workspace=self.ws, idx=self.idx)
 
+    def step_on(self, i, stream):
+        """Step i on `stream` with the buffer set of its parity (the pipelined timing)."""
+        kk, ss = self.sets[i % self.n]
+        sc, ws, idx = (self.sc, self.ws, self.idx) if i % 2 == 0 else (self.sc2, self.ws2, self.idx2)
+        self.api.li_decode_select(self.q, self.w, kk, ss, KTOP, scores=sc, workspace=ws, idx=idx, stream=stream)
+
     def build_graphs(self, warmup):
         import torch
         for i in range(warmup):
@@ -355,6 +365,25 @@ class DecodeBench:
         self.score_launches = self.n * reps
         self.topk_graph = capture([self.topk] * 16)
         self.topk_launches = 16
+        # the same steps, independent, alternating over two streams: step i's top-k overlaps step
+        # i+1's scorer (an even number of steps, so that every set is used in both parities)
+        self.pipe_n = 2 * self.n
+        self.pipe_streams = [torch.cuda.Stream(device=self.sc.device) for _ in range(2)]
+        self.pipe_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.pipe_graph):
+            main = torch.cuda.current_stream()
+            fork = torch.cuda.Event()
+            fork.record(main)
+            for st in self.pipe_streams:
+                st.wait_event(fork)
+            for i in range(self.pipe_n):
+                st = self.pipe_streams[i % 2]
+                with torch.cuda.stream(st):
+                    self.step_on(i, st)
+            for st in self.pipe_streams:
+                ev = torch.cuda.Event()
+                ev.record(st)
+                main.wait_event(ev)
         self.restore_graph = capture([self.restore] * 16)
         for g in self.step_graphs:
             g.replay()
@@ -362,6 +391,7 @@ class DecodeBench:
         self.score_graph.replay()
         self.topk_graph.replay()
         self.restore_graph.replay()
+        self.pipe_graph.replay()
         torch.cuda.synchronize()
 
     def time_steps(self, steps):
@@ -377,6 +407,11 @@ class DecodeBench:
         e1.record()
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / steps
+
+    def time_pipelined(self, steps):
+        """At least `steps` independent steps, two in flight (whole pipelined graphs); time per step."""
+        reps = max(1, -(-steps // self.pipe_n))
+        return self._time_graph(self.pipe_graph, self.pipe_n, reps)
 
     def time_steps_single(self, steps):
         """The same steps, one graph launch per step."""
@@ -444,36 +479,42 @@ def run_li(args, rank, world, local_rank):
     topk_ms = bench.time_kernel("topk")
     direct_ms = bench.time_direct(args.steps)
     single_ms = bench.time_steps_single(args.steps)
-    ms, score_ms, topk_ms, direct_ms, single_ms = li_dist.max_over_ranks(
-        [ms, score_ms, topk_ms, direct_ms, single_ms], device=dev)
+    pipe_dev_ms = bench.time_pipelined(args.steps)
+    ms, score_ms, topk_ms, direct_ms, single_ms, pipe_dev_ms = li_dist.max_over_ranks(
+        [ms, score_ms, topk_ms, direct_ms, single_ms, pipe_dev_ms], device=dev)
     launches = 2 * args.steps
 
     # ---- end to end through the public API.  Throughput: K independent steps as one DecodePipeline
     # graph, each step copying its own pinned host query/weights in and its selected positions out,
-    # the copies of neighbouring steps overlapping its kernels.  Latency: the same step alone as one
-    # graph-captured DecodeIndexer step (copy in -> li_decode_select -> copy out), back to back.
+    # the copies of neighbouring steps overlapping its kernels; the headline e2e keeps the steps'
+    # kernels on one stream, as `value` does, and the pipelined figure lets two steps' kernels
+    # overlap.  Latency: the same step alone as one graph-captured DecodeIndexer step (copy in ->
+    # li_decode_select -> copy out), back to back.
     from sparse_attention_lightning_score_b200.step import DecodeIndexer, DecodePipeline
-    pipe = DecodePipeline([bench.sets[i % bench.n] for i in range(args.steps)], H, KTOP)
-    for i in range(args.steps):
-        pipe.q_host[i].copy_(bench.case.q)
-        pipe.w_host[i].copy_(bench.case.w)
-    for _ in range(max(1, args.warmup // 2)):
-        pipe.run(sync=False)
-    torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
     a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a0.record()
-    pipe.run(sync=False)
-    a1.record()
-    torch.cuda.synchronize()
-    e2e_ms = a0.elapsed_time(a1) / args.steps
-    # the selections that came back to the host match the device-side graph's
-    bench.step_graphs[(args.steps - 1) % bench.n].replay()
-    torch.cuda.synchronize()
-    assert torch.equal(pipe.idx_host[args.steps - 1], bench.idx.cpu())
-    h2d, d2h = pipe.h2d_bytes_per_step, pipe.d2h_bytes_per_step
-    del pipe
+    e2e = {}
+    for nstreams in (1, 2):
+        pipe = DecodePipeline([bench.sets[i % bench.n] for i in range(args.steps)], H, KTOP, streams=nstreams)
+        for i in range(args.steps):
+            pipe.q_host[i].copy_(bench.case.q)
+            pipe.w_host[i].copy_(bench.case.w)
+        for _ in range(max(1, args.warmup // 2)):
+            pipe.run(sync=False)
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        a0.record()
+        pipe.run(sync=False)
+        a1.record()
+        torch.cuda.synchronize()
+        e2e[nstreams] = a0.elapsed_time(a1) / args.steps
+        # the selections that came back to the host match the device-side graph's
+        bench.step_graphs[(args.steps - 1) % bench.n].replay()
+        torch.cuda.synchronize()
+        assert torch.equal(pipe.idx_host[args.steps - 1], bench.idx.cpu())
+        h2d, d2h = pipe.h2d_bytes_per_step, pipe.d2h_bytes_per_step
+        del pipe
+    e2e_ms, pipe_e2e_ms = e2e[1], e2e[2]
     indexers = [DecodeIndexer(kk, ss, H, KTOP) for kk, ss in bench.sets]
     for ix in indexers:
         ix.q_host.copy_(bench.case.q)
@@ -487,7 +528,7 @@ def run_li(args, rank, world, local_rank):
     a1.record()
     torch.cuda.synchronize()
     lat_ms = a0.elapsed_time(a1) / args.steps
-    e2e_ms, lat_ms = li_dist.max_over_ranks([e2e_ms, lat_ms], device=dev)
+    e2e_ms, pipe_e2e_ms, lat_ms = li_dist.max_over_ranks([e2e_ms, pipe_e2e_ms, lat_ms], device=dev)
     del indexers
     assert api.li_get_last_error() == 0
 
@@ -501,7 +542,9 @@ def run_li(args, rank, world, local_rank):
             st_ms = bx.time_steps(max(20, args.steps))
             sc_ms = bx.time_kernel("score")
             tk_ms = bx.time_kernel("topk")
+            pp_ms = bx.time_pipelined(max(20, args.steps))
             sweep[str(Lx)] = {"us_per_step": round(st_ms * 1e3, 2), "score_us": round(sc_ms * 1e3, 2),
+                              "pipelined_us_per_step": round(pp_ms * 1e3, 2),
                               "topk_us": round(tk_ms * 1e3, 2), "keys_per_s": B * Lx / (st_ms * 1e-3),
                               "score_hbm_frac": round(B * Lx * decode_bytes_per_key() / (sc_ms * 1e-3) / 1e9 / hbm,
                                                       3)}
@@ -545,10 +588,16 @@ def run_li(args, rank, world, local_rank):
         "direct_us_per_step": direct_ms * 1e3, "graph_per_step_us": single_ms * 1e3,
         "e2e": {"value": world * B * L / (e2e_ms * 1e-3), "unit": "keys/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-                "api": "DecodePipeline.run: K independent steps in one graph, each H2D q,w -> li_decode_select "
-                       "-> D2H indices, neighbouring steps' copies overlapping its kernels",
+                "api": "DecodePipeline(streams=1).run: K independent steps in one graph, each H2D q,w -> "
+                       "li_decode_select -> D2H indices, neighbouring steps' copies overlapping its kernels, "
+                       "the steps' kernels one after another",
                 "latency_ms_per_step": lat_ms,
                 "latency_api": "DecodeIndexer.step (one step per graph: H2D q,w -> li_decode_select -> D2H indices)"},
+        "pipelined": {"us_per_step": pipe_dev_ms * 1e3, "keys_per_s": world * B * L / (pipe_dev_ms * 1e-3),
+                      "e2e_us_per_step": pipe_e2e_ms * 1e3, "e2e_keys_per_s": world * B * L / (pipe_e2e_ms * 1e-3),
+                      "how": "the same independent steps, two in flight on two streams with their own scores and "
+                             "workspaces (step i's top-k overlaps step i+1's scorer); device-only, and end to end "
+                             "through DecodePipeline(streams=2) with the same copies as e2e"},
         "gpu_launches": launches,
         "clocks": clk,
     }

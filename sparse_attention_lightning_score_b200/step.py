@@ -104,12 +104,12 @@ class DecodePipeline:
     """Independent decode-indexer steps back to back, with their transfers overlapped.
 
     A serving engine that runs the indexer of many independent steps (other
-    layers' indexers, other request batches) does not need step i's selection
-    before step i+1's inputs can move.  Here ``steps`` such steps form one CUDA
-    graph on three streams:
+    request batches, micro-batches in flight together) does not need step i's
+    selection before step i+1's inputs can move.  Here ``steps`` such steps
+    form one CUDA graph:
 
         copy stream 1:  H2D(i)   H2D(i+1)   H2D(i+2) ...
-        main stream:          select(i)  select(i+1)  select(i+2) ...
+        compute:              select(i)  select(i+1)  select(i+2) ...
         copy stream 2:                 D2H(i)     D2H(i+1) ...
 
     Step i's inputs come from its own page-locked host buffer into device
@@ -120,13 +120,19 @@ class DecodePipeline:
     after their previous step's kernels (inputs) and result copy (outputs)
     have finished.  Every kernel in the graph is an li kernel.
 
+    ``streams`` compute streams take the steps in turn (step i on stream
+    i % streams), each with its own scores and workspace.  With one, the
+    steps' kernels run one after another.  With two, step i's top-k (a chain
+    of short, latency-bound phases on a few dozen SMs) overlaps step i+1's
+    scorer, which streams the cache at HBM bandwidth.
+
     caches: a list of ``steps`` (k8, ks) key caches, one per step (a cache may
     repeat); heads, k, lens as for ``DecodeIndexer``.  The host inputs are
     ``q_host[i]`` (bf16 [B,H,d]) and ``w_host[i]`` (fp32 [B,H]); ``run()``
     replays the graph and returns the list of pinned int32 [B, k] results.
     """
 
-    def __init__(self, caches, heads: int, k: int, lens: Optional[torch.Tensor] = None):
+    def __init__(self, caches, heads: int, k: int, lens: Optional[torch.Tensor] = None, streams: int = 2):
         self.caches = list(caches)
         k8, ks = self.caches[0]
         if not (k8.is_cuda and ks.is_cuda):
@@ -134,6 +140,9 @@ class DecodePipeline:
         B, L, d = k8.shape
         self.B, self.L, self.d, self.H, self.k, self.lens = B, L, d, heads, k, lens
         self.steps = S = len(self.caches)
+        if streams not in (1, 2):
+            raise ValueError("streams must be 1 or 2")
+        self.nstreams = streams
         dev = k8.device
         qbytes = B * heads * d * 2
         self.nbytes = nbytes = qbytes + B * heads * 4
@@ -145,10 +154,11 @@ class DecodePipeline:
         self.q_dev = [t[:qbytes].view(torch.bfloat16).view(B, heads, d) for t in self.in_dev]
         self.w_dev = [t[qbytes:].view(torch.float32).view(B, heads) for t in self.in_dev]
         self.idx_dev = [torch.empty((B, k), dtype=torch.int32, device=dev) for _ in range(2)]
-        self.scores = torch.empty((B, (L + 3) // 4 * 4), dtype=torch.float32, device=dev)
-        self.ws = api.li_decode_select_workspace(B, dev, L)
+        self.scores = [torch.empty((B, (L + 3) // 4 * 4), dtype=torch.float32, device=dev) for _ in range(streams)]
+        self.ws = [api.li_decode_select_workspace(B, dev, L) for _ in range(streams)]
         self.s_in = torch.cuda.Stream(device=dev)
         self.s_out = torch.cuda.Stream(device=dev)
+        self.s_comp = [torch.cuda.Stream(device=dev) for _ in range(streams)] if streams > 1 else []
         self._select(0, torch.cuda.current_stream(dev))  # warm-up: module, kernel attributes, argument checks
         torch.cuda.synchronize(dev)
         self.graph = torch.cuda.CUDAGraph()
@@ -156,31 +166,35 @@ class DecodePipeline:
             self._capture(torch.cuda.current_stream(dev))
 
     def _select(self, i, stream):
-        j = i % 2
+        j, c = i % 2, i % self.nstreams
         k8, ks = self.caches[i]
-        api.li_decode_select(self.q_dev[j], self.w_dev[j], k8, ks, self.k, lens=self.lens, scores=self.scores,
-                             workspace=self.ws, idx=self.idx_dev[j], stream=stream)
+        api.li_decode_select(self.q_dev[j], self.w_dev[j], k8, ks, self.k, lens=self.lens, scores=self.scores[c],
+                             workspace=self.ws[c], idx=self.idx_dev[j], stream=stream)
 
     def _capture(self, main):
         fork = torch.cuda.Event()
         fork.record(main)
         self.s_in.wait_event(fork)
         self.s_out.wait_event(fork)
+        for s in self.s_comp:
+            s.wait_event(fork)
         done_sel, done_out = [], []
         for i in range(self.steps):
             j = i % 2
+            comp = self.s_comp[i % self.nstreams] if self.s_comp else main
             with torch.cuda.stream(self.s_in):
                 if i >= 2:
                     self.s_in.wait_event(done_sel[i - 2])  # slot j's inputs were read by step i - 2
                 self.in_dev[j].copy_(self.in_host[i], non_blocking=True)
                 arrived = torch.cuda.Event()
                 arrived.record(self.s_in)
-            main.wait_event(arrived)
+            comp.wait_event(arrived)
             if i >= 2:
-                main.wait_event(done_out[i - 2])  # slot j's result of step i - 2 has been copied out
-            self._select(i, main)
+                comp.wait_event(done_out[i - 2])  # slot j's result of step i - 2 has been copied out
+            # step i - streams, on the same compute stream, used this stream's scores and workspace
+            self._select(i, comp)
             ev = torch.cuda.Event()
-            ev.record(main)
+            ev.record(comp)
             done_sel.append(ev)
             with torch.cuda.stream(self.s_out):
                 self.s_out.wait_event(ev)
@@ -189,9 +203,10 @@ class DecodePipeline:
                 ev_o.record(self.s_out)
                 done_out.append(ev_o)
         main.wait_event(done_out[-1])
-        joined = torch.cuda.Event()
-        joined.record(self.s_in)
-        main.wait_event(joined)
+        for s in [self.s_in] + self.s_comp:
+            joined = torch.cuda.Event()
+            joined.record(s)
+            main.wait_event(joined)
 
     def run(self, sync: bool = True):
         """Replay the ``steps`` steps; returns the pinned host results (valid once the stream has

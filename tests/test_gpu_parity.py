@@ -341,14 +341,16 @@ def test_decode_indexer_graph_step():
     assert api.li_get_last_error() == LI_OK
 
 
-def test_decode_pipeline_matches_single_steps():
+@pytest.mark.parametrize("streams", [1, 2])
+def test_decode_pipeline_matches_single_steps(streams):
     """Five independent steps in one pipelined graph (transfers overlapped with the kernels, device
-    slots reused two steps later) select exactly what five separate graph steps select."""
+    slots reused two steps later; with two compute streams, neighbouring steps' kernels overlap too)
+    select exactly what five separate graph steps select."""
     from sparse_attention_lightning_score_b200.step import DecodeIndexer, DecodePipeline
     cases = [synth.dsa_decode(B=3, L=6000, k_top=500, seed=70 + i) for i in range(3)]
     caches = [(c.k8.to(DEV), c.ks.to(DEV)) for c in cases]
     order = [0, 1, 2, 1, 0]
-    pipe = DecodePipeline([caches[i] for i in order], heads=64, k=500)
+    pipe = DecodePipeline([caches[i] for i in order], heads=64, k=500, streams=streams)
     g = torch.Generator().manual_seed(77)
     qs = [torch.randn(3, 64, 128, generator=g).to(torch.bfloat16) for _ in order]
     ws = [torch.randn(3, 64, generator=g) * 0.1 for _ in order]
@@ -362,6 +364,31 @@ def test_decode_pipeline_matches_single_steps():
             want = one.step(qs[i], ws[i]).clone()
             assert torch.equal(got[i], want), (rep, i)
     assert pipe.h2d_bytes_per_step == 3 * 64 * 128 * 2 + 3 * 64 * 4 and pipe.d2h_bytes_per_step == 3 * 500 * 4
+    assert api.li_get_last_error() == LI_OK
+
+
+def test_decode_pipeline_two_streams_full_size():
+    """The benchmarked shape (8 requests of 32768 keys, k = 2048), six independent steps over three
+    caches with ragged lengths, two compute streams: every step's selection equals that step alone."""
+    from sparse_attention_lightning_score_b200.step import DecodeIndexer, DecodePipeline
+    lens = torch.tensor([32768, 30000, 2048, 2049, 17, 32767, 20000, 4096], dtype=torch.int32)
+    cases = [synth.dsa_decode(B=8, L=32768, seed=90 + i) for i in range(3)]
+    caches = [(c.k8.to(DEV), c.ks.to(DEV)) for c in cases]
+    order = [0, 1, 2, 0, 1, 2]
+    pipe = DecodePipeline([caches[i] for i in order], heads=64, k=2048, lens=lens.to(DEV), streams=2)
+    g = torch.Generator().manual_seed(91)
+    qs = [torch.randn(8, 64, 128, generator=g).to(torch.bfloat16) for _ in order]
+    ws = [torch.randn(8, 64, generator=g) * 0.1 for _ in order]
+    for i in range(len(order)):
+        pipe.q_host[i].copy_(qs[i])
+        pipe.w_host[i].copy_(ws[i])
+    got = [t.clone() for t in pipe.run()]
+    got2 = [t.clone() for t in pipe.run()]
+    for i, c in enumerate(order):
+        one = DecodeIndexer(caches[c][0], caches[c][1], heads=64, k=2048, lens=lens.to(DEV))
+        want = one.step(qs[i], ws[i]).clone()
+        assert torch.equal(got[i], want), i
+        assert torch.equal(got2[i], want), i
     assert api.li_get_last_error() == LI_OK
 
 
