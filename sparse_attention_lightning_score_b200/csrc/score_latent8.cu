@@ -58,7 +58,7 @@ __global__ void __launch_bounds__(L8_THREADS, 2) latent8_score_kernel(const __gr
     const int b = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     pdl_trigger();
-    if (blockIdx.x * a.tiles_per_cta >= (a.max_len + L8_M - 1) / L8_M) return;  // no tile for any length
+    if ((int)blockIdx.x >= (a.max_len + L8_M - 1) / L8_M) return;  // no tile for any length
 
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L8_OFF_BAR);
     uint64_t* empty = full + L8_STAGES;
@@ -98,8 +98,11 @@ __global__ void __launch_bounds__(L8_THREADS, 2) latent8_score_kernel(const __gr
         len_b = len_b < 0 ? 0 : a.max_len;
     }
     const int ntiles = (len_b + L8_M - 1) / L8_M;
-    const int t0 = blockIdx.x * a.tiles_per_cta;
-    const int nt = min(t0 + a.tiles_per_cta, ntiles) - t0;
+    // tiles are dealt round robin: CTA c takes tiles c, c + G, c + 2G, ... (G = CTAs per request), so
+    // that every CTA reads from the whole of its request's cache
+    const int t0 = blockIdx.x;
+    const int tstride = gridDim.x;
+    const int nt = t0 < ntiles ? (ntiles - t0 + tstride - 1) / tstride : 0;
     if (nt <= 0) goto done;  // uniform over the CTA
 
     if (warp == 0) {
@@ -112,7 +115,7 @@ __global__ void __launch_bounds__(L8_THREADS, 2) latent8_score_kernel(const __gr
             uint32_t ph = 0;
             bool ok = true;
             for (int it = 0; ok && it < nt; ++it) {
-                const int y = (int)(rowbase + (long long)(t0 + it) * L8_M);
+                const int y = (int)(rowbase + (long long)(t0 + it * tstride) * L8_M);
                 for (int kb = 0; kb < L8_KBLK; ++kb) {
                     if (!mbar_wait(&empty[stage], ph ^ 1u, a.err)) { ok = false; break; }
                     mbar_arrive_expect_tx(&full[stage], L8_STAGE_BYTES);
@@ -215,7 +218,7 @@ __global__ void __launch_bounds__(L8_THREADS, 2) latent8_score_kernel(const __gr
         for (int it = 0; it < nt; ++it) {
             const int acc = it % L8_NACC;
             const uint32_t aph = (uint32_t)(it / L8_NACC) & 1u;
-            const int s = (t0 + it) * L8_M + g * 32 + lane;
+            const int s = (t0 + it * tstride) * L8_M + g * 32 + lane;
             const float sk = s < len_b ? __ldg(a.cscale + srow + s) : 1.f;
             if (!mbar_wait(&accf[acc], aph, a.err)) break;
             tc_fence_after();
@@ -233,14 +236,6 @@ __global__ void __launch_bounds__(L8_THREADS, 2) latent8_score_kernel(const __gr
                 if constexpr (HIST) atomicAdd(&hs[order_key(sc) >> LI_HIST_SHIFT], 1u);
             }
         }
-        if constexpr (HIST) {
-            asm volatile("bar.sync 2, 128;" ::: "memory");
-            uint32_t* gh = a.hist + (size_t)b * LI_HIST_BINS;
-            for (int i = et; i < LI_HIST_BINS; i += 128) {
-                const uint32_t v = hs[i];
-                if (v) atomicAdd(gh + i, v);
-            }
-        }
     }
 done:
     __syncwarp();
@@ -248,6 +243,21 @@ done:
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, L8_NACC * L8_H);
+    }
+    if constexpr (HIST) {
+        // every epilogue count is in (the barrier above): all warps add the non-empty bins to the
+        // request's histogram, four bins per shared-memory load
+        if (nt > 0) {
+            uint32_t* gh = a.hist + (size_t)b * LI_HIST_BINS;
+            const uint4* h4 = reinterpret_cast<const uint4*>(hs);
+            for (int i = threadIdx.x; i < LI_HIST_BINS / 4; i += L8_THREADS) {
+                const uint4 v = h4[i];
+                if (v.x) atomicAdd(gh + 4 * i, v.x);
+                if (v.y) atomicAdd(gh + 4 * i + 1, v.y);
+                if (v.z) atomicAdd(gh + 4 * i + 2, v.z);
+                if (v.w) atomicAdd(gh + 4 * i + 3, v.w);
+            }
+        }
     }
 }
 
@@ -263,7 +273,8 @@ li_status launch_impl(const CUtensorMap& map, const Latent8Args& args, int batch
         attr_done[dev] = true;
     }
     const int sms = host_num_sms();
-    int cpr = max(1, (2 * sms) / max(1, batch));  // two CTAs per SM in total, spread over the requests
+    // two CTAs per SM in total, spread over the requests, each with about the same number of tiles
+    int cpr = max(1, (2 * sms) / max(1, batch));
     int tpc = max(1, (ntiles_max + cpr - 1) / cpr);
     cpr = (ntiles_max + tpc - 1) / tpc;
     Latent8Args a = args;
