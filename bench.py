@@ -815,9 +815,15 @@ class LatentBench:
 class HsBench:
     """HS decode at L=131072: anchor absorb + scan + top-8192, 3 follower absorbs + refine.
 
-    The followers' absorption does not depend on the anchor, so its one launch (all three
-    layers) runs on a second stream while the anchor absorbs, scans and selects; the refine
-    waits for both.  The anchor's scan counts its first radix digit for the top-8192."""
+    The anchor's scan counts its first radix digit for the top-8192.  Two layouts of the same
+    calls, chosen by batch size:
+      - B < 8: all four layers are absorbed in one launch, then the anchor's scan and top-k and the
+        followers' refine follow on the same stream, so each kernel starts under a programmatic
+        dependency on the previous one (at one request the absorption is latency-bound and its
+        four layers cost about what one does);
+      - B >= 8: the followers' absorption (one launch, three layers) runs on a second stream while
+        the anchor absorbs, scans and selects, and the refine waits for both (the followers'
+        absorption would lengthen the anchor's chain by several µs)."""
 
     def __init__(self, dev, B):
         import torch
@@ -844,10 +850,20 @@ class HsBench:
         self.cand = torch.empty((B, self.C), dtype=torch.int32, device=dev)
         self.out = torch.empty((3, B, KTOP), dtype=torch.int32, device=dev)
         self.ws = api.li_hs_refine_workspace(B, self.C, 3, dev)
+        self.one_stream = B < 8
+        self.q_all = torch.stack(self.q).contiguous()
+        self.wd_all = torch.stack(self.wd).contiguous()
+        self.qt_all = torch.empty((4, B, H, 256), dtype=torch.bfloat16, device=dev)
 
     def step(self, i):
         import torch
         c = self.c[i % len(self.c)]
+        if self.one_stream:
+            self.api.li_absorb_query_layers(self.q_all, self.wd_all, out=self.qt_all)
+            self.api.li_latent_score_hist(self.qt_all[0], self.w0, c, self.hist, scores=self.sc)
+            self.api.li_topk_hist(self.sc, self.C, self.hist, idx=self.cand)
+            self.api.li_hs_refine(c, self.cand, self.qt_all[1:], self.wf, KTOP, out=self.out, workspace=self.ws)
+            return
         main = torch.cuda.current_stream()
         self.side.wait_stream(main)
         with torch.cuda.stream(self.side):
@@ -1000,8 +1016,8 @@ def run_table4(dev, args, clocks):
       dsa         4 layers x li_decode_select (FP8 keys, 64 heads, d = 128, top-2048);
       indexcache  1 indexer layer of the 4 (the other 3 reuse its selection: no kernel);
       latentindex 4 layers x (absorb + bf16 latent scan over the shared d_c = 256 cache + top-2048);
-      hs          anchor (absorb + scan + top-C, C = min(8192, L)) + 3 followers (one absorb launch on a
-                  side stream, gather-once rescoring, top-2048);
+      hs          all four layers absorbed in one launch, the anchor's scan + top-C (C = min(8192, L)),
+                  then the 3 followers' gather-once rescoring and top-2048, on one stream;
       *_fp8       the same two over DeepSeek-V3.2's d_c = 192 e4m3 latent with per-row scales.
     Every layer reads its own cache copies, rotated so that a group's working set exceeds L2."""
     import torch
@@ -1027,15 +1043,15 @@ def run_table4(dev, args, clocks):
         ql = [lcase.q[l].to(dev) for l in range(4)]
         wdl = [lcase.w_dec[l].to(dev) for l in range(4)]
         wl = [lcase.w[l].to(dev) for l in range(4)]
-        qf, wdf, wf = lcase.q[1:].contiguous().to(dev), lcase.w_dec[1:].contiguous().to(dev), lcase.w[1:].contiguous().to(dev)
+        wf = lcase.w[1:].contiguous().to(dev)
         qt = torch.empty((1, H, 256), dtype=torch.bfloat16, device=dev)
-        qtf = torch.empty((3, 1, H, 256), dtype=torch.bfloat16, device=dev)
+        ql_all, wdl_all = torch.stack(ql).contiguous(), torch.stack(wdl).contiguous()
+        qt_all = torch.empty((4, 1, H, 256), dtype=torch.bfloat16, device=dev)
         hist = api.li_decode_select_workspace(1, dev).view(torch.int32)[:2048]
         lsc = torch.empty((1, Lx), dtype=torch.float32, device=dev)
         cand = torch.empty((1, C), dtype=torch.int32, device=dev)
         out = torch.empty((3, 1, KTOP), dtype=torch.int32, device=dev)
         hws = api.li_hs_refine_workspace(1, C, 3, dev)
-        side = torch.cuda.Stream(device=dev)
         # the same methods over DeepSeek-V3.2's FP8 latent (d_c = 192 e4m3, one scale per row)
         fcase = synth.latent_rope_nope(B=1, L=Lx, G=4, seed=5)
         fper = Lx * 196
@@ -1044,10 +1060,10 @@ def run_table4(dev, args, clocks):
         q8l = [fcase.q[l].to(dev) for l in range(4)]
         wd8 = [fcase.w_dec[l].to(dev) for l in range(4)]
         w8 = [fcase.w[l].to(dev) for l in range(4)]
-        qf8, wdf8, wf8 = (fcase.q[1:].contiguous().to(dev), fcase.w_dec[1:].contiguous().to(dev),
-                          fcase.w[1:].contiguous().to(dev))
+        wf8 = fcase.w[1:].contiguous().to(dev)
         qt8 = torch.empty((1, H, 192), dtype=torch.bfloat16, device=dev)
-        qtf8 = torch.empty((3, 1, H, 192), dtype=torch.bfloat16, device=dev)
+        q8_all, wd8_all = torch.stack(q8l).contiguous(), torch.stack(wd8).contiguous()
+        qt8_all = torch.empty((4, 1, H, 192), dtype=torch.bfloat16, device=dev)
 
         def dsa(i, layers=4):
             for l in range(layers):
@@ -1063,15 +1079,10 @@ def run_table4(dev, args, clocks):
 
         def hs(i):
             c = cs[i % lcopy]
-            main = torch.cuda.current_stream()
-            side.wait_stream(main)
-            with torch.cuda.stream(side):
-                api.li_absorb_query_layers(qf, wdf, out=qtf)
-            api.li_absorb_query(ql[0], wdl[0], out=qt)
-            api.li_latent_score_hist(qt, wl[0], c, hist, scores=lsc)
+            api.li_absorb_query_layers(ql_all, wdl_all, out=qt_all)
+            api.li_latent_score_hist(qt_all[0], wl[0], c, hist, scores=lsc)
             api.li_topk_hist(lsc, C, hist, idx=cand)
-            main.wait_stream(side)
-            api.li_hs_refine(c, cand, qtf, wf, KTOP, out=out, workspace=hws)
+            api.li_hs_refine(c, cand, qt_all[1:], wf, KTOP, out=out, workspace=hws)
 
         def latent8(i):
             c8, cs8 = c8s[i % fcopy]
@@ -1082,15 +1093,10 @@ def run_table4(dev, args, clocks):
 
         def hs8(i):
             c8, cs8 = c8s[i % fcopy]
-            main = torch.cuda.current_stream()
-            side.wait_stream(main)
-            with torch.cuda.stream(side):
-                api.li_absorb_query_layers(qf8, wdf8, out=qtf8)
-            api.li_absorb_query(q8l[0], wd8[0], out=qt8)
-            api.li_latent_score_fp8(qt8, w8[0], c8, cs8, hist=hist, scores=lsc)
+            api.li_absorb_query_layers(q8_all, wd8_all, out=qt8_all)
+            api.li_latent_score_fp8(qt8_all[0], w8[0], c8, cs8, hist=hist, scores=lsc)
             api.li_topk_hist(lsc, C, hist, idx=cand)
-            main.wait_stream(side)
-            api.li_hs_refine_fp8(c8, cs8, cand, qtf8, wf8, KTOP, out=out, workspace=hws)
+            api.li_hs_refine_fp8(c8, cs8, cand, qt8_all[1:], wf8, KTOP, out=out, workspace=hws)
 
         res = {"L": Lx}
         for name, fn in (("dsa", lambda i: dsa(i)), ("indexcache", lambda i: dsa(i, 1)), ("latentindex", latent),
