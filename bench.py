@@ -531,6 +531,13 @@ def run_li(args, rank, world, local_rank):
     e2e_ms, pipe_e2e_ms, lat_ms = li_dist.max_over_ranks([e2e_ms, pipe_e2e_ms, lat_ms], device=dev)
     del indexers
     assert api.li_get_last_error() == 0
+    # every collective of the run is behind us: the group closes before rank 0's sweep and prefill
+    # legs, so the other ranks neither wait on them nor run into the group's timeout
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
 
     sweep = None
     if not args.no_sweep and rank == 0:
@@ -561,11 +568,6 @@ def run_li(args, rank, world, local_rank):
         prefill = prefill_record(r, px, pclk, fp8)
         del px
         assert api.li_get_last_error() == 0
-    if dist:
-        dist.barrier()
-        dist.destroy_process_group()
-    if rank != 0:
-        return
 
     hbm, which = peaks()
     units = B * L
