@@ -28,9 +28,9 @@
 // a block-wide scan (warp shuffles) that finds the digit of the k-th key.
 //
 // Compaction: the slice's counts above / at the threshold are exchanged over
-// the cluster once, then the slice is written in order, 4 keys per thread per
-// tile, positions from a block-wide scan.  No output depends on the order of
-// any atomic operation.
+// the cluster once, then the slice is written in order, 4 or 8 consecutive
+// keys per thread per sweep, positions from a block-wide scan.  No output
+// depends on the order of any atomic operation.
 //
 // With a histogram from the decode scorer (HIST): its LI_HIST_BITS-bit digit
 // is the first pass, found by one block-wide scan in every CTA with no cluster
@@ -98,12 +98,30 @@ struct TopkShape {
     }
 };
 
+// KPT consecutive keys of the slice from shared memory (keys at or past cnt read as 0); i0 % 4 == 0.
+template <int KPT>
+__device__ __forceinline__ void load_keys(const uint4* t, int i0, int cnt, uint32_t (&kk)[KPT]) {
+#pragma unroll
+    for (int q = 0; q < KPT / 4; ++q) {
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (i0 + 4 * q < cnt) v = t[(i0 >> 2) + q];
+        kk[4 * q] = v.x;
+        kk[4 * q + 1] = v.y;
+        kk[4 * q + 2] = v.z;
+        kk[4 * q + 3] = v.w;
+    }
+}
+
 // Thread t < OWNERS owns the BPT contiguous bins BINS-BPT(t+1) .. BINS-BPT*t-1
 // (descending positions BPT*t .. BPT*t+BPT-1).
 template <int NT, bool CLUSTER, bool HIST>
 __global__ void __launch_bounds__(NT) topk_kernel(const TopkArgs a, int row0, int chunk) {
     using S = TopkShape<NT, CLUSTER>;
     constexpr int BPT = S::BPT, NW = S::WARPS, NCOPY = S::NCOPY, BINS = S::BINS;
+    // keys per thread in the candidate and compaction sweeps: 4 for the 1024-thread cluster CTAs
+    // (slices of at most 4096 keys, so every thread has keys and one block-wide scan covers the
+    // slice), 8 otherwise
+    constexpr int KPT = (CLUSTER && NT == 1024) ? 4 : 8;
     static_assert(BPT == 1 || BPT == 2 || BPT == 4 || BPT == 8, "bins per owner");
     extern __shared__ uint4 tk_dyn[];
     uint32_t* keys = reinterpret_cast<uint32_t*>(tk_dyn);
@@ -220,17 +238,15 @@ __global__ void __launch_bounds__(NT) topk_kernel(const TopkArgs a, int row0, in
         if (total_h != (uint32_t)n && c == 0 && threadIdx.x == 0) record_error(a.err, ERRBIT_BOUNDS);
         if (total_h == (uint32_t)n && inbin_h <= (uint32_t)a.cand_cap) {
             // ---- this slice's candidates (keys in bin b1, in position order) and its count of keys
-            // above the bin: eight consecutive keys per thread, offsets from one block-wide scan
+            // above the bin: KPT consecutive keys per thread, offsets from one block-wide scan
             uint32_t ncand = 0u, nabove = 0u;
-            for (int tb = 0, flip = 0; tb < cnt; tb += NT * 8, flip ^= 1) {
-                const int i0 = tb + threadIdx.x * 8;
-                uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
-                if (i0 < cnt) v0 = tk_dyn[i0 >> 2];
-                if (i0 + 4 < cnt) v1 = tk_dyn[(i0 >> 2) + 1];
-                const uint32_t kk[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            for (int tb = 0, flip = 0; tb < cnt; tb += NT * KPT, flip ^= 1) {
+                const int i0 = tb + threadIdx.x * KPT;
+                uint32_t kk[KPT];
+                load_keys<KPT>(tk_dyn, i0, cnt, kk);
                 uint32_t cm = 0u, na = 0u;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
+                for (int e = 0; e < KPT; ++e) {
                     const uint32_t d = kk[e] >> LI_HIST_SHIFT;
                     const bool valid = i0 + e < cnt;
                     cm |= (valid && d == b1) ? 1u << e : 0u;
@@ -241,7 +257,7 @@ __global__ void __launch_bounds__(NT) topk_kernel(const TopkArgs a, int row0, in
                 const uint32_t excl = block_scan1<NW>(packed, wsum[flip], &tot) - packed;
                 uint32_t slot = ncand + (excl & 0xffffu);
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
+                for (int e = 0; e < KPT; ++e)
                     if (cm & (1u << e)) {
                         if (slot < (uint32_t)a.cand_cap) cand[slot] = kk[e];
                         ++slot;
@@ -487,18 +503,16 @@ __global__ void __launch_bounds__(NT) topk_kernel(const TopkArgs a, int row0, in
     const int quota = ties ? max(0, krem - (int)eq_before) : 0;
     const int out_base = (int)gt_before + (ties ? min((int)eq_before, krem) : 0);
 
-    // ---- ordered compaction of the slice: eight consecutive keys per thread, positions from a
-    // block-wide scan per NT * 8 keys
+    // ---- ordered compaction of the slice: KPT consecutive keys per thread, positions from a
+    // block-wide scan per NT * KPT keys
     int carry_gt = 0, carry_eq = 0;
-    for (int tb = 0, flip = 1; tb < cnt; tb += NT * 8, flip ^= 1) {
-        const int i0 = tb + threadIdx.x * 8;
-        uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
-        if (i0 < cnt) v0 = tk_dyn[i0 >> 2];
-        if (i0 + 4 < cnt) v1 = tk_dyn[(i0 >> 2) + 1];
-        const uint32_t kk[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    for (int tb = 0, flip = 1; tb < cnt; tb += NT * KPT, flip ^= 1) {
+        const int i0 = tb + threadIdx.x * KPT;
+        uint32_t kk[KPT];
+        load_keys<KPT>(tk_dyn, i0, cnt, kk);
         uint32_t gm = 0u, em = 0u;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
+        for (int e = 0; e < KPT; ++e) {
             const bool valid = i0 + e < cnt;
             if (valid && (ties ? kk[e] > T : kk[e] >= T)) gm |= 1u << e;
             else if (valid && ties && kk[e] == T) em |= 1u << e;
@@ -510,7 +524,7 @@ __global__ void __launch_bounds__(NT) topk_kernel(const TopkArgs a, int row0, in
         int eb = carry_eq + (int)(excl & 0xffffu);
         if (gm | em) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
+            for (int e = 0; e < KPT; ++e) {
                 int pos = -1;
                 if (gm & (1u << e)) {
                     pos = out_base + gb + min(eb, quota);
