@@ -639,10 +639,10 @@ li_status launch_topk(const TopkArgs& a, cudaStream_t st) {
         if (a.hist) {
             if (cs == 1) e = small ? launch_one<512, false, true>(a, row0, nr, cs, chunk, st)
                                    : launch_one<1024, false, true>(a, row0, nr, cs, chunk, st);
-            // slices of up to 4096 keys in clusters of 4 or 8, 32 CTAs or more: 1024 threads (measured
-            // faster in the decode step at B = 8, L = 16K-32K); the rest keep 512 (1024 was slower for
-            // one request's row, the HS followers' and the shard merge's 2-CTA rows, and 8K-key slices)
-            else if (chunk <= TK_SLICE && cs >= 4 && cs <= 8 && (long long)nr * cs >= 32)
+            // slices of up to 4096 keys in clusters of 2 to 8: 1024 threads, four keys each in the
+            // sweeps (measured faster in the decode step at B = 8, L = 8K-32K, and no slower for the
+            // HS followers' 2-CTA rows); longer slices keep 512 (1024 was much slower on 8K-key slices)
+            else if (chunk <= TK_SLICE && cs >= 2 && cs <= 8)
                 e = launch_one<1024, true, true>(a, row0, nr, cs, chunk, st);
             else e = launch_one<512, true, true>(a, row0, nr, cs, chunk, st);
         } else {
